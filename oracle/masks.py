@@ -1,0 +1,68 @@
+"""Block masks of the two layouts (oracle; test infrastructure only).
+
+Source: "Striped Attention: Faster Ring Attention for Causal Transformers"
+review, GetMask 函数 (procedures GETMASKRINGATTENTION and
+GETMASKSTRIPEDATTENTION), and the causal matrix C of 三 技术架构 / 核心公式.
+
+Reading taken (the pages are ambiguous here): (j, k) = (query block, key
+block).  The printed rules only agree with C when the MASK is indexed as
+MASK[x, y] with x = KEY-local index and y = QUERY-local index:
+
+* ring:    j < k: everything blocked; j = k: blocked where y < x (the query
+  precedes the key); j > k: nothing blocked.  The ring procedure prints no
+  initialisation; it is read as zero-initialised like the striped one.
+* striped: j < k: blocked where y <= x; j >= k: blocked where y < x.
+
+Both procedures below return boolean arrays in that printed orientation
+(True = -inf).  ``mask_from_positions`` derives the same blocks from the
+original token positions and C, in the conventional [query, key]
+orientation; the pins check that one is the transpose of the other.
+"""
+
+import numpy as np
+
+from .partition import CONTIGUOUS, STRIPED, token_of
+
+
+def getmask_ring(j, k, c):
+    """GETMASKRINGATTENTION(j, k): MASK[x (key), y (query)], True = -inf."""
+    mask = np.zeros((c, c), dtype=bool)
+    if j < k:
+        mask[:, :] = True
+    elif j == k:
+        for x in range(c):
+            for y in range(c):
+                if y < x:
+                    mask[x, y] = True
+    return mask
+
+
+def getmask_striped(j, k, c):
+    """GETMASKSTRIPEDATTENTION(j, k): MASK[x (key), y (query)], True = -inf."""
+    mask = np.zeros((c, c), dtype=bool)
+    for x in range(c):
+        for y in range(c):
+            if j < k and y <= x:
+                mask[x, y] = True
+            elif j >= k and y < x:
+                mask[x, y] = True
+    return mask
+
+
+def getmask(j, k, c, layout):
+    if layout == CONTIGUOUS:
+        return getmask_ring(j, k, c)
+    if layout == STRIPED:
+        return getmask_striped(j, k, c)
+    raise ValueError(layout)
+
+
+def mask_from_positions(j, k, N, P, layout, causal=True):
+    """Blocked[query-local, key-local] for query shard j against key shard k,
+    taken from C over original token positions."""
+    c = N // P
+    qpos = np.array([token_of(j, x, N, P, layout) for x in range(c)])
+    kpos = np.array([token_of(k, y, N, P, layout) for y in range(c)])
+    if not causal:
+        return np.zeros((c, c), dtype=bool)
+    return kpos[None, :] > qpos[:, None]

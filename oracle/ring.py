@@ -1,0 +1,87 @@
+"""The blockwise ring method restated step by step, in float64 (oracle).
+
+Test infrastructure only.  Used on tiny inputs to check the method's own
+invariants (its result equals the plain definition in ``attention``), never
+as the source of expected GPU values at scale.
+
+Steps, in the order of "ICLR 2024論文解説: Ring Attention":
+
+* ステップ1 -- split Q, K, V into P blocks of c = N/P rows (contiguous), or
+  stripe them (Striped review, 分区策略对比; see ``partition``).
+* ステップ2 -- device j keeps Q_j; in each of P rounds it holds one K/V block
+  and passes it on to device j+1, so in round r it holds block (j - r) mod P
+  (the 実装例 sends to rank+1 and receives from rank-1).
+* ステップ3 -- fold each round in with online softmax.  The printed
+  recurrence is incomplete: it shows O_j = diag(l_{j-1}/l_j) O_{j-1} +
+  exp(S_j - m_j)/l_j V_j without defining l_j and without the factor that
+  re-bases O_{j-1} from the old max to the new one.  Reading taken
+  (consistent with the 実装例, which rescales both the running sum and the
+  unnormalised output by exp(row_max - new_max)):
+
+      m_j = max(m_{j-1}, rowmax(S_j))
+      l_j = exp(m_{j-1} - m_j) l_{j-1} + rowsum(exp(S_j - m_j))
+      O_j = diag(exp(m_{j-1} - m_j) l_{j-1} / l_j) O_{j-1}
+            + diag(1 / l_j) exp(S_j - m_j) V_j            (normalised form)
+
+  The 実装例 keeps O unnormalised and divides by l once at the end
+  (``normalise_each_round=False``); both forms are offered so that the pins
+  show they agree.
+* Causal blocks are masked with GetMask(j, block) (Striped review, GetMask 函数);
+  a row with every key of a block masked contributes nothing to that round
+  (the pages are silent; exp(-inf) = 0 with the running max left unchanged).
+"""
+
+import numpy as np
+
+from .masks import getmask
+from .partition import shard_len
+
+
+def ring_attention(q, k, v, P, layout, causal, scale, normalise_each_round=False,
+                   round_order=None):
+    """Blockwise ring attention over P virtual devices.
+
+    q, k, v: [N, d] in LAYOUT order (already partitioned).  Returns O [N, dv]
+    and lse [N] in layout order.  ``round_order``: optional permutation of
+    range(P) giving the order in which the rounds are folded in (the merge is
+    order-independent; the ring order is the default).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    N = q.shape[0]
+    c = shard_len(N, P)
+    out = np.empty((N, v.shape[1]))
+    lse_out = np.empty(N)
+    rounds = list(range(P)) if round_order is None else list(round_order)
+    for j in range(P):                       # device j, its Q block stays put
+        qj = q[j * c:(j + 1) * c]
+        m = np.full(c, -np.inf)
+        l = np.zeros(c)
+        o = np.zeros((c, v.shape[1]))
+        for r in rounds:
+            kb = (j - r) % P                 # block held by device j in round r
+            kj = k[kb * c:(kb + 1) * c]
+            vj = v[kb * c:(kb + 1) * c]
+            s = (qj @ kj.T) * float(scale)
+            if causal:
+                blocked = getmask(j, kb, c, layout).T   # -> [query, key]
+                s = np.where(blocked, -np.inf, s)
+            m_new = np.maximum(m, np.max(s, axis=1))
+            m_sub = np.where(np.isneginf(m_new), 0.0, m_new)
+            p = np.exp(s - m_sub[:, None])
+            alpha = np.exp(m - m_sub)
+            l_new = alpha * l + np.sum(p, axis=1)
+            if normalise_each_round:
+                with np.errstate(invalid="ignore", divide="ignore"):
+                    keep = np.where(l_new > 0, alpha * l / l_new, 0.0)
+                    inv = np.where(l_new > 0, 1.0 / l_new, 0.0)
+                o = keep[:, None] * o + inv[:, None] * (p @ vj)
+            else:
+                o = alpha[:, None] * o + p @ vj
+            m, l = m_new, l_new
+        if not normalise_each_round:
+            o = o / l[:, None]
+        out[j * c:(j + 1) * c] = o
+        lse_out[j * c:(j + 1) * c] = m + np.log(l)
+    return out, lse_out

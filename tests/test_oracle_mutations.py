@@ -1,0 +1,142 @@
+"""Planted mistakes: each pin must catch a plausible error in the oracle.
+
+Every test below swaps one oracle function for a copy with a single planted
+mistake (a dropped term, a wrong sign or index, a transposed operand) and
+checks that at least one pin of test_oracle_*.py then fails.  The mistakes
+are planted in the oracle, on the CPU only.
+"""
+
+import numpy as np
+import pytest
+
+import tests.test_oracle_attention as TA
+import tests.test_oracle_partition_masks_work as TP
+from oracle import attention as att
+from oracle import masks, merge, partition, ring, work
+from oracle.partition import CONTIGUOUS, STRIPED
+
+
+def _attention_mutant(kind):
+    def f(q, k, v, scale, causal, q_pos=None, k_pos=None):
+        q, k, v = (np.asarray(a, dtype=np.float64) for a in (q, k, v))
+        nq, nk = q.shape[-2], k.shape[-2]
+        if kind == "transposed":
+            s = np.matmul(k, np.swapaxes(q, -1, -2)) * scale
+        elif kind == "no_scale":
+            s = np.matmul(q, np.swapaxes(k, -1, -2))
+        else:
+            s = np.matmul(q, np.swapaxes(k, -1, -2)) * scale
+        if causal:
+            qp = np.arange(nq) if q_pos is None else np.asarray(q_pos)
+            kp = np.arange(nk) if k_pos is None else np.asarray(k_pos)
+            if kind == "mask_includes_diagonal":
+                blocked = kp[None, :] >= qp[:, None]
+                blocked[:, 0] = False            # keep row 0 finite
+            elif kind == "mask_flipped":
+                blocked = kp[None, :] < qp[:, None]
+            else:
+                blocked = kp[None, :] > qp[:, None]
+            s = np.where(blocked, -np.inf, s)
+        mx = np.max(s, axis=-1, keepdims=True)
+        e = np.exp(s - mx)
+        den = np.sum(e, axis=-1, keepdims=True)
+        if kind == "no_normalise":
+            den = np.ones_like(den)
+        o = (e / den) @ v
+        lse = (mx + np.log(den))[..., 0]
+        return o, lse
+    return f
+
+
+@pytest.mark.parametrize("kind", ["transposed", "no_scale", "mask_includes_diagonal",
+                                  "mask_flipped", "no_normalise"])
+def test_attention_mutants_fail_brute_force_pin(monkeypatch, kind):
+    monkeypatch.setattr(att, "attention", _attention_mutant(kind))
+    with pytest.raises(AssertionError):
+        for causal in (True, False):
+            TA.test_definition_equals_pure_python_brute_force(causal, 7, 4, 5, 0.5)
+            TA.test_definition_equals_pure_python_brute_force(causal, 12, 6, 3, 1.3)
+
+
+def _ring_mutant(kind):
+    def f(q, k, v, P, layout, causal, scale, normalise_each_round=False, round_order=None):
+        N = q.shape[0]
+        c = N // P
+        out = np.empty((N, v.shape[1]))
+        lse_out = np.empty(N)
+        for j in range(P):
+            qj = q[j * c:(j + 1) * c]
+            m = np.full(c, -np.inf)
+            l = np.zeros(c)
+            o = np.zeros((c, v.shape[1]))
+            for r in range(P):
+                kb = (j - r) % P
+                kj, vj = k[kb * c:(kb + 1) * c], v[kb * c:(kb + 1) * c]
+                s = (qj @ kj.T) * scale
+                if causal:
+                    blocked = masks.getmask(j, kb, c, layout)
+                    if kind != "mask_not_transposed":
+                        blocked = blocked.T
+                    s = np.where(blocked, -np.inf, s)
+                m_new = np.maximum(m, np.max(s, axis=1))
+                m_sub = np.where(np.isneginf(m_new), 0.0, m_new)
+                p = np.exp(s - m_sub[:, None])
+                alpha = np.exp(m - m_sub)
+                if kind == "no_rescale":
+                    alpha = np.where(np.isneginf(m), 0.0, 1.0)
+                if kind == "rescale_sum_only":
+                    o = o + p @ vj
+                else:
+                    o = alpha[:, None] * o + p @ vj
+                l = alpha * l + np.sum(p, axis=1)
+                m = m_new
+            out[j * c:(j + 1) * c] = o / l[:, None]
+            lse_out[j * c:(j + 1) * c] = m + np.log(l)
+        return out, lse_out
+    return f
+
+
+@pytest.mark.parametrize("kind", ["mask_not_transposed", "no_rescale", "rescale_sum_only"])
+def test_ring_mutants_fail_exactness_pin(monkeypatch, kind):
+    monkeypatch.setattr(ring, "ring_attention", _ring_mutant(kind))
+    with pytest.raises(AssertionError):
+        for layout in (CONTIGUOUS, STRIPED):
+            TA.test_blockwise_ring_equals_full_softmax(layout, True, 24, 4, False)
+
+
+def test_partition_mutant_fails_golden(monkeypatch, golden_dir):
+    def swapped(shard, local, N, P, layout):
+        c = N // P
+        return shard * c + local if layout == STRIPED else local * P + shard
+    monkeypatch.setattr(partition, "token_of", swapped)
+    with pytest.raises(AssertionError):
+        TP.test_worked_stripe_example(golden_dir)
+
+
+def test_getmask_mutant_fails_position_pin(monkeypatch):
+    def wrong(j, k, c):
+        mask = np.zeros((c, c), dtype=bool)
+        for x in range(c):
+            for y in range(c):
+                if (j < k and y < x) or (j >= k and y <= x):   # strictness swapped
+                    mask[x, y] = True
+        return mask
+    monkeypatch.setattr(masks, "getmask_striped", wrong)
+    with pytest.raises(AssertionError):
+        TP.test_getmask_equals_causal_C_over_positions(STRIPED, 3, 4)
+
+
+def test_work_mutant_fails_brute_force_pin(monkeypatch):
+    monkeypatch.setattr(work, "work_striped_printed",
+                        lambda i, j, c: c * (c - 1) // 2 if i >= j else c * (c + 1) // 2)
+    with pytest.raises(AssertionError):
+        TP.test_work_counts_brute_force_equal_closed_forms(STRIPED, 3, 4)
+
+
+def test_merge_mutant_fails_split_pin(monkeypatch):
+    def wrong(o_a, lse_a, o_b, lse_b):
+        lse = np.logaddexp(lse_a, lse_b)
+        return (np.exp(lse_a)[..., None] * o_a + np.exp(lse_b)[..., None] * o_b), lse
+    monkeypatch.setattr(merge, "lse_merge", wrong)
+    with pytest.raises(AssertionError):
+        TA.test_lse_merge_of_key_halves_equals_full(7)
