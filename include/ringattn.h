@@ -1,0 +1,196 @@
+/*
+ * ringattn.h -- C ABI of the B200 (sm_100a) exact blockwise attention library
+ * (libringattn.so).
+ *
+ * The library computes exact causal (or full) softmax attention the way Ring
+ * Attention and Striped Attention organise it: the sequence is split into P
+ * virtual shards; each shard's query block stays put while the key/value
+ * blocks visit it in ring order, one block per round, and every round is
+ * folded in with an online softmax (running max m, running normaliser l,
+ * output rescaled when m grows).  Fully masked tiles are skipped.
+ *
+ * Sources for the operations (page title, section):
+ *   - "ICLR 2024論文解説: Ring Attention -- 複数GPU間でのブロックワイズ分散
+ *     アテンションによる超長コンテキスト処理": ステップ1 (contiguous split),
+ *     ステップ2 (ring rounds), ステップ3 (online-softmax recurrence; scores
+ *     scaled by 1/sqrt(d)), 実装例 (unnormalised accumulator, one final
+ *     division by the row sum).
+ *   - "Striped Attention: Faster Ring Attention for Causal Transformers"
+ *     (paper review): 核心公式 (CausalAttn = Softmax(QK^T + C)V), 分区策略对比
+ *     (token t on device t mod P), GetMask 函数 (block masks), 分块与分瓦片
+ *     (skip fully masked tiles), 位置编码处理 (position ids striped alike).
+ *   - 1cademy, "Computing Attention Weights in Sequence Parallelism": the
+ *     softmax denominator as a sum of per-node partial sums (lse merge).
+ *
+ * Conventions for every entry point:
+ *   - All pointers marked "device" are CUDA device pointers on the current
+ *     device; the caller allocates and owns every buffer.  The library never
+ *     allocates device memory and keeps no pointer after a call returns.
+ *   - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL =
+ *     the legacy default stream).  A return of RA_OK means the work was
+ *     validated and enqueued, not that it finished.
+ *   - Arguments are validated on the host before anything is launched; an
+ *     invalid call returns a non-zero status and launches nothing.  No entry
+ *     point aborts, prints, or traps on the device.
+ *   - Tensors are dense row-major.  [B, H, N, d] bf16 means element
+ *     (b, h, n, i) at ((b*H + h)*N + n)*d + i, two bytes each.
+ *   - Thread safety: calls may be made from several host threads; each call
+ *     only reads its arguments.
+ */
+#ifndef RINGATTN_H_
+#define RINGATTN_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int ra_status;
+
+/* Status codes. */
+#define RA_OK 0
+#define RA_ERR_NULL 1        /* a required pointer is NULL                     */
+#define RA_ERR_ALIGN 2       /* a pointer is not 16-byte aligned               */
+#define RA_ERR_SHAPE 3       /* sizes out of range, or N not a multiple of P   */
+#define RA_ERR_HEADDIM 4     /* head dimension d not supported (64 or 128)     */
+#define RA_ERR_LAYOUT 5      /* unknown layout / flag bits                     */
+#define RA_ERR_SCALE 6       /* scale not finite or not > 0                    */
+#define RA_ERR_DTYPE 7       /* unknown dtype code                             */
+#define RA_ERR_ALIAS 8       /* input and output buffers overlap               */
+#define RA_ERR_CUDA 9        /* a CUDA runtime/driver call failed              */
+#define RA_ERR_DEVICE 10     /* current device is not sm_100 (B200)            */
+#define RA_ERR_DEVICE_FAULT 11 /* a kernel gave up a bounded wait (see below)  */
+
+/* Layouts (low byte of `layout`). */
+#define RA_CONTIGUOUS 0      /* shard j = tokens [j*c, (j+1)*c)  (Ring)        */
+#define RA_STRIPED 1         /* shard j = tokens j, j+P, j+2P, ...  (Striped)  */
+
+/* Optional scheduling flag for ra_attn_fwd, OR-ed into `layout`.
+ * Default ("owner" schedule): each virtual shard j is served by its own fixed
+ * group of floor(#SM / P) streaming multiprocessors, which walk that shard's
+ * query tiles through all P rounds -- the per-device work of the ring, so
+ * the wall time is set by the most loaded shard as on P real devices.
+ * RA_SCHED_FREE: every SM takes work from every shard (a single-GPU
+ * load-balanced schedule; same results, same tile skipping). */
+#define RA_SCHED_FREE 0x100
+
+/* Element types for ra_partition. */
+#define RA_BF16 0
+#define RA_F32 1
+#define RA_I32 2
+
+/* Human-readable text for a status code (static storage; never NULL). */
+const char* ra_status_string(ra_status status);
+
+/* Library version, as major*10000 + minor*100 + patch. */
+int ra_version(void);
+
+/*
+ * ra_partition -- move rows between token order and layout order.
+ *
+ * Defined by the placements of "Striped Attention" review 分区策略对比 and
+ * Ring Attention explainer ステップ1: with c = N/P, layout slot s = j*c + x
+ * (shard j, local index x) holds token t = x*P + j (RA_STRIPED) or
+ * t = j*c + x (RA_CONTIGUOUS).  Position ids are moved the same way
+ * (Striped review, 位置编码处理): pass the int32 ids as [1, 1, N, 1] RA_I32.
+ *
+ *   src, dst  device, [B, H, N, d] of `dtype` (bf16 = 2 bytes, f32/i32 = 4).
+ *             Must not overlap (RA_ERR_ALIAS); 16-byte aligned when a row
+ *             (d * element size) is a multiple of 16 bytes, else 4-byte
+ *             aligned.
+ *   inverse   0: token order -> layout order  (dst[.,.,s,:] = src[.,.,t(s),:])
+ *             1: layout order -> token order  (dst[.,.,t(s),:] = src[.,.,s,:])
+ *   P         number of shards, 1 <= P <= N, N % P == 0.
+ *   d         row length in elements (any value >= 1; use d = 1 for lse or
+ *             position ids).
+ * The result is a pure byte permutation (bit-exact).  RA_CONTIGUOUS is the
+ * identity and is performed as a copy.
+ */
+ra_status ra_partition(const void* src, void* dst, int64_t B, int64_t H, int64_t N, int64_t d,
+                       int P, int layout, int inverse, int dtype, void* stream);
+
+/*
+ * ra_attn_fwd -- exact blockwise attention forward over P virtual shards.
+ *
+ * Computes, per (b, h), O = Softmax(Q K^T * scale + C) V and
+ * lse[i] = ln sum_t exp(Q_i . K_t * scale + C_it) (natural log), where C is
+ * -inf where the key's ORIGINAL token index exceeds the query's (causal != 0)
+ * and 0 otherwise (Striped review 核心公式; Ring explainer ステップ3).  The
+ * shard loop follows the ring: shard j's query tiles meet key block
+ * (j - r) mod P in round r, folded in with online softmax; tiles that the
+ * layout's GetMask hides completely are not computed.
+ *
+ *   q, k, v  device, [B, H, N, d] bf16, rows already in LAYOUT order (see
+ *            ra_partition), 16-byte aligned.
+ *   o        device, [B, H, N, d] bf16 output, layout order, 16-byte aligned.
+ *            Must not overlap q, k, v.
+ *   lse      device, [B, H, N] float32 output, layout order, 16-byte aligned.
+ *   d        64 or 128.
+ *   N, P     1 <= P, N % P == 0, c = N / P <= 2^30 / 128; any c (a ragged
+ *            last tile of a shard is masked).  B*H*N < 2^31.
+ *   layout   RA_CONTIGUOUS or RA_STRIPED, optionally | RA_SCHED_FREE.
+ *   causal   0: no mask (the layout then only permutes rows); else causal in
+ *            original token order.
+ *   scale    > 0 and finite; 1/sqrt(d) is the usual value.
+ * Arithmetic: bf16 operands, fp32 accumulation of Q K^T and P V on the
+ * tensor cores, fp32 softmax statistics, probabilities rounded to bf16 for
+ * the P V product, O rounded to bf16 once at the end.
+ */
+ra_status ra_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                      int64_t B, int64_t H, int64_t N, int64_t d, int P, int layout,
+                      int causal, float scale, void* stream);
+
+/*
+ * ra_lse_merge -- merge two partial attention results over disjoint key sets.
+ *
+ * From the split of the softmax denominator into per-node partial sums
+ * (1cademy, "Computing Attention Weights in Sequence Parallelism"):
+ *   lse = ln(e^lse_a + e^lse_b);  o = e^(lse_a - lse) o_a + e^(lse_b - lse) o_b
+ * A side with lse = -inf contributes nothing; both -inf gives o = 0,
+ * lse = -inf.
+ *
+ *   o_a, o_b, o_out      device, [rows, d] bf16, 16-byte aligned.
+ *   lse_a, lse_b, lse_out device, [rows] float32.
+ *   o_out may alias o_a (and lse_out lse_a): each element is read before it
+ *   is written by the same thread.
+ *   rows >= 0 (0 is a no-op), 1 <= d, d % 8 == 0.
+ * Arithmetic in fp32, o_out rounded to bf16.
+ */
+ra_status ra_lse_merge(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,
+                       void* o_out, float* lse_out, int64_t rows, int64_t d, void* stream);
+
+/*
+ * ra_tile_census -- count, on the device, what ra_attn_fwd's schedule does.
+ *
+ * For every query shard j and round r (key block (j - r) mod P), counts with
+ * the attention kernel's own tile classifier and per-row mask limits:
+ *   out[(j*P + r)*4 + 0]  tiles skipped
+ *   out[(j*P + r)*4 + 1]  tiles computed without a mask
+ *   out[(j*P + r)*4 + 2]  tiles computed with a per-element mask
+ *   out[(j*P + r)*4 + 3]  visible (query, key) pairs = the round's work
+ * for one (b, h) (every head has the same schedule).  Tiles are 128 x 128.
+ * The visible-pair counts are the per-device, per-round work of the Striped
+ * review (Ring Attention 工作负载 / Striped Attention 工作负载).
+ *
+ *   out   device, int64[P * P * 4], 8-byte aligned; overwritten.
+ *   N, P  as for ra_attn_fwd (d plays no role).
+ */
+ra_status ra_tile_census(int64_t N, int P, int layout, int causal, int64_t* out, void* stream);
+
+/*
+ * ra_device_fault -- read and clear the library's device fault word.
+ *
+ * Every wait inside the library's kernels is bounded.  A kernel that gives up
+ * a wait records a non-zero code here, releases what it holds and returns
+ * early (its outputs are then incomplete).  This call synchronises the
+ * current device, stores the word in *code (0 = no fault) and clears it.
+ * Returns RA_ERR_DEVICE_FAULT if the word was non-zero, RA_OK otherwise.
+ */
+ra_status ra_device_fault(int* code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RINGATTN_H_ */

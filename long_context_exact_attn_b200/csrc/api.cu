@@ -1,0 +1,191 @@
+// C-ABI entry points of libringattn.so: host-side validation, then a launch
+// on the caller's stream.  Declarations and contracts: include/ringattn.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "ra_internal.h"
+
+namespace ra {
+
+PFN_encodeTiled get_encode_tiled() {
+  static PFN_encodeTiled fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_encodeTiled>(p);
+  });
+  return fn;
+}
+
+namespace {
+
+struct DevInfo {
+  int ok;
+  int num_sms;
+};
+
+// Current device, checked to be sm_100 (B200 class); SM count cached.
+ra_status current_device(int* dev, DevInfo* info) {
+  static DevInfo cache[64];
+  static int cached[64] = {0};
+  static std::mutex mu;
+  if (cudaGetDevice(dev) != cudaSuccess) return RA_ERR_CUDA;
+  if (*dev < 0 || *dev >= 64) return RA_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cached[*dev]) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, *dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, *dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, *dev) != cudaSuccess)
+      return RA_ERR_CUDA;
+    cache[*dev].ok = (major == 10 && minor == 0);
+    cache[*dev].num_sms = sms;
+    cached[*dev] = 1;
+  }
+  *info = cache[*dev];
+  return info->ok ? RA_OK : RA_ERR_DEVICE;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool overlap(const void* a, int64_t na, const void* b, int64_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + (uintptr_t)nb && y < x + (uintptr_t)na;
+}
+
+}  // namespace
+}  // namespace ra
+
+using namespace ra;
+
+extern "C" {
+
+const char* ra_status_string(ra_status s) {
+  switch (s) {
+    case RA_OK: return "ok";
+    case RA_ERR_NULL: return "a required pointer is NULL";
+    case RA_ERR_ALIGN: return "a pointer is not suitably aligned (16 bytes)";
+    case RA_ERR_SHAPE: return "sizes out of range or N not a multiple of P";
+    case RA_ERR_HEADDIM: return "head dimension must be 64 or 128";
+    case RA_ERR_LAYOUT: return "unknown layout or flag bits";
+    case RA_ERR_SCALE: return "scale must be finite and > 0";
+    case RA_ERR_DTYPE: return "unknown dtype code";
+    case RA_ERR_ALIAS: return "input and output buffers overlap";
+    case RA_ERR_CUDA: return "a CUDA runtime/driver call failed";
+    case RA_ERR_DEVICE: return "current device is not an sm_100 GPU";
+    case RA_ERR_DEVICE_FAULT: return "a kernel gave up a bounded wait; outputs incomplete";
+    default: return "unknown status";
+  }
+}
+
+int ra_version(void) { return 100; }
+
+ra_status ra_partition(const void* src, void* dst, int64_t B, int64_t H, int64_t N, int64_t d,
+                       int P, int layout, int inverse, int dtype, void* stream) {
+  if (!src || !dst) return RA_ERR_NULL;
+  if (layout != RA_CONTIGUOUS && layout != RA_STRIPED) return RA_ERR_LAYOUT;
+  int64_t esz;
+  switch (dtype) {
+    case RA_BF16: esz = 2; break;
+    case RA_F32: case RA_I32: esz = 4; break;
+    default: return RA_ERR_DTYPE;
+  }
+  if (B < 1 || H < 1 || N < 1 || d < 1 || P < 1 || N % P != 0) return RA_ERR_SHAPE;
+  if (B * H * N >= ((int64_t)1 << 31) || d * esz >= ((int64_t)1 << 30)) return RA_ERR_SHAPE;
+  const int64_t row_bytes = d * esz;
+  const uintptr_t need = (row_bytes % 16 == 0) ? 16 : (esz == 2 ? 2 : 4);
+  if (!aligned(src, need) || !aligned(dst, need)) return RA_ERR_ALIGN;
+  const int64_t bytes = B * H * N * row_bytes;
+  if (overlap(src, bytes, dst, bytes)) return RA_ERR_ALIAS;
+  int dev;
+  DevInfo info;
+  ra_status st = current_device(&dev, &info);
+  if (st) return st;
+  return partition_launch(src, dst, B * H, N, P, row_bytes, layout == RA_STRIPED, inverse != 0,
+                          stream);
+}
+
+ra_status ra_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                      int64_t B, int64_t H, int64_t N, int64_t d, int P, int layout, int causal,
+                      float scale, void* stream) {
+  if (!q || !k || !v || !o || !lse) return RA_ERR_NULL;
+  if (layout & ~(0xff | RA_SCHED_FREE)) return RA_ERR_LAYOUT;
+  const int base = layout & 0xff;
+  if (base != RA_CONTIGUOUS && base != RA_STRIPED) return RA_ERR_LAYOUT;
+  if (d != 64 && d != 128) return RA_ERR_HEADDIM;
+  if (B < 1 || H < 1 || N < 1 || P < 1 || N % P != 0) return RA_ERR_SHAPE;
+  if (B * H * N >= ((int64_t)1 << 31) || B * H >= ((int64_t)1 << 31)) return RA_ERR_SHAPE;
+  if (N / P > ((int64_t)1 << 30) / 128) return RA_ERR_SHAPE;
+  if (!(scale > 0.f) || !isfinite(scale)) return RA_ERR_SCALE;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(lse, 16))
+    return RA_ERR_ALIGN;
+  const int64_t tb = B * H * N * d * 2, lb = B * H * N * 4;
+  if (overlap(o, tb, q, tb) || overlap(o, tb, k, tb) || overlap(o, tb, v, tb) ||
+      overlap(lse, lb, q, tb) || overlap(lse, lb, k, tb) || overlap(lse, lb, v, tb) ||
+      overlap(lse, lb, o, tb))
+    return RA_ERR_ALIAS;
+  int dev;
+  DevInfo info;
+  ra_status st = current_device(&dev, &info);
+  if (st) return st;
+  AttnLaunch a;
+  a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
+  a.BH = B * H; a.N = N; a.d = d; a.P = P;
+  a.striped = base == RA_STRIPED;
+  a.causal = causal != 0;
+  a.sched_free = (layout & RA_SCHED_FREE) != 0;
+  a.scale = scale;
+  a.device = dev;
+  a.num_sms = info.num_sms;
+  a.stream = stream;
+  return attn_fwd_launch(a);
+}
+
+ra_status ra_lse_merge(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,
+                       void* o_out, float* lse_out, int64_t rows, int64_t d, void* stream) {
+  if (!o_a || !lse_a || !o_b || !lse_b || !o_out || !lse_out) return RA_ERR_NULL;
+  if (rows < 0 || d < 1 || d % 8 != 0 || d > (1 << 20)) return RA_ERR_SHAPE;
+  if (rows >= ((int64_t)1 << 40)) return RA_ERR_SHAPE;
+  if (!aligned(o_a, 16) || !aligned(o_b, 16) || !aligned(o_out, 16) || !aligned(lse_a, 4) ||
+      !aligned(lse_b, 4) || !aligned(lse_out, 4))
+    return RA_ERR_ALIGN;
+  const int64_t ob = rows * d * 2, lb = rows * 4;
+  // o_out may coincide with o_a exactly; any other overlap is refused.
+  if ((o_out != o_a && overlap(o_out, ob, o_a, ob)) || overlap(o_out, ob, o_b, ob) ||
+      (lse_out != lse_a && overlap(lse_out, lb, lse_a, lb)) ||
+      (lse_out != lse_b && overlap(lse_out, lb, lse_b, lb)) || overlap(o_out, ob, lse_out, lb))
+    return RA_ERR_ALIAS;
+  int dev;
+  DevInfo info;
+  ra_status st = current_device(&dev, &info);
+  if (st) return st;
+  return lse_merge_launch(o_a, lse_a, o_b, lse_b, o_out, lse_out, rows, d, info.num_sms, stream);
+}
+
+ra_status ra_tile_census(int64_t N, int P, int layout, int causal, int64_t* out, void* stream) {
+  if (!out) return RA_ERR_NULL;
+  if (layout != RA_CONTIGUOUS && layout != RA_STRIPED) return RA_ERR_LAYOUT;
+  if (N < 1 || P < 1 || N % P != 0 || N >= ((int64_t)1 << 31) || P > 65536) return RA_ERR_SHAPE;
+  if (!aligned(out, 8)) return RA_ERR_ALIGN;
+  int dev;
+  DevInfo info;
+  ra_status st = current_device(&dev, &info);
+  if (st) return st;
+  return tile_census_launch(N, P, layout == RA_STRIPED, causal != 0, out, stream);
+}
+
+ra_status ra_device_fault(int* code) {
+  if (!code) return RA_ERR_NULL;
+  return read_device_fault(code);
+}
+
+}  // extern "C"

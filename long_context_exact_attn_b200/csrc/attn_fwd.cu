@@ -1,0 +1,569 @@
+// Exact blockwise ring/striped attention forward for sm_100a (B200).
+//
+// What is computed (Ring Attention explainer "ICLR 2024論文解説: Ring
+// Attention", ステップ2/ステップ3 and 実装例; Striped Attention review,
+// 核心公式 / GetMask 函数 / 分块与分瓦片): for each virtual shard j, its query
+// tiles stay resident while the key/value blocks arrive in ring order
+// (round r brings block (j - r) mod P); each key tile is folded into the
+// running row max m, row sum l and unnormalised output O by online softmax,
+// and O is divided by l once at the end.  Tiles that the block's causal
+// mask hides completely are never loaded or computed.
+//
+// Kernel organisation (one persistent CTA per SM, 320 threads):
+//   warps 0-3  softmax warpgroup for query tile 0 of the CTA's tile pair
+//   warps 4-7  softmax warpgroup for query tile 1
+//   warp  8    TMA producer: Q tile pair once per work item, then K and V
+//              tiles into a ring of shared-memory slots
+//   warp  9    tcgen05 issuer (one thread) + TMEM owner
+// Tensor memory (512 columns x 128 lanes x 32 bit):
+//   [0,128)  S0 = Q0 K^T (fp32), later overwritten in place by P0 (bf16x2,
+//            columns [0,64)) which is the A operand of P0 V
+//   [128,256) S1 / P1
+//   [256,256+D) O0 accumulator (fp32),  [256+D, 256+2D) O1
+// With the 32x32b TMEM access pattern thread i of a softmax warpgroup owns
+// query row i: the row max and row sum are plain per-thread reductions.
+//
+// The two query tiles are ping-ponged on the tensor core: while warpgroup 0
+// turns S0 into P0, the tensor core runs P1 V and the next Q1 K^T, and vice
+// versa.  Every wait is bounded (see mbar_wait); on a timeout the kernel
+// raises an abort flag, drains its own MMAs and TMA loads, frees TMEM and
+// returns, recording the fault in the library's device fault word.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ra_internal.h"
+#include "ra_ptx.cuh"
+#include "ra_tiles.cuh"
+
+namespace ra {
+
+__device__ unsigned int g_device_fault = 0;
+
+struct AttnParams {
+  __nv_bfloat16* o;
+  float* lse;
+  int BH;             // B * H
+  int N;              // sequence length
+  int c;              // shard length N / P
+  int P;              // shards
+  int npairs;         // query-tile pairs per shard = ceil(ceil(c/128) / 2)
+  int striped;        // layout
+  int causal;
+  int groups;         // shard groups (owner schedule) or 1 (free schedule)
+  int ctas_per_group;
+  float c2;           // scale * log2(e)
+  unsigned long long timeout_ns;
+};
+
+template <int D>
+struct Cfg {
+  static constexpr int kTileBytes = kBM * D * 2;           // one Q, K or V tile
+  static constexpr int kChunks = D / 64;                   // 128-byte swizzle chunks per row
+  static constexpr int kSlots = (D == 128) ? 5 : 10;       // K/V ring slots
+  static constexpr int kQOff = 0;
+  static constexpr int kRingOff = 2 * kTileBytes;
+  static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
+  // barriers: q_full, q_empty, full[kSlots], empty[kSlots], s_full[2],
+  // p_full[2], o_full[2], o_free[2], drain
+  static constexpr int kNumBars = 2 + 2 * kSlots + 8 + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
+  static constexpr int kThreads = 320;
+};
+
+// ------------------------------------------------------------ work items
+struct Item {
+  int bh, j, pair;
+};
+
+// Items of a shard group, in non-increasing order of work: causal striped
+// (and non-causal) work grows with the pair's local index; causal
+// contiguous work grows with the shard index first.
+__device__ __forceinline__ bool item_at(const AttnParams& p, int g, int u, Item& it) {
+  const int n_sh = (p.P - g + p.groups - 1) / p.groups;   // shards g, g+groups, ...
+  const int per_shard = p.npairs * p.BH;
+  if (u >= n_sh * per_shard) return false;
+  if (p.causal && !p.striped) {
+    const int sh_rank = u / per_shard;
+    const int rem = u - sh_rank * per_shard;
+    it.j = g + (n_sh - 1 - sh_rank) * p.groups;
+    it.pair = p.npairs - 1 - rem / p.BH;
+    it.bh = rem % p.BH;
+  } else {
+    const int per_pair = n_sh * p.BH;
+    const int pr = u / per_pair;
+    const int rem = u - pr * per_pair;
+    it.pair = p.npairs - 1 - pr;
+    it.j = g + (rem / p.BH) * p.groups;
+    it.bh = rem % p.BH;
+  }
+  return true;
+}
+
+// k-th item of this CTA: snake order over the group's members.
+__device__ __forceinline__ bool cta_item(const AttnParams& p, int k, Item& it) {
+  const int g = blockIdx.x / p.ctas_per_group;
+  const int m = blockIdx.x % p.ctas_per_group;
+  if (g >= p.groups) return false;
+  const int G = p.ctas_per_group;
+  const int u = k * G + ((k & 1) ? (G - 1 - m) : m);
+  return item_at(p, g, u, it);
+}
+
+// The key tiles met by a query-tile pair, in ring order.
+struct TileSeq {
+  int j, P, c, striped, causal;
+  int x0, x_last;           // first row of tile 0, last valid row of the pair
+  int r, kt, kend;
+  BlockMask bm;
+  int kb;
+
+  __device__ __forceinline__ void init(const AttnParams& p, const Item& it) {
+    j = it.j; P = p.P; c = p.c; striped = p.striped; causal = p.causal;
+    x0 = it.pair * 2 * kBM;
+    const int rows = tile_rows(x0, c) + tile_rows(x0 + kBM, c);
+    x_last = x0 + rows - 1;
+    r = -1; kt = 0; kend = 0;
+  }
+  // Next tile; false at the end.  Fills block index, key start and the kind
+  // of the tile for each of the two query tiles.
+  __device__ __forceinline__ bool next(int& kb_out, int& y0, int& k0, int& k1, BlockMask& m) {
+    while (true) {
+      if (kt >= kend) {
+        if (++r >= P) return false;
+        kb = key_block(j, r, P);
+        bm = block_mask(j, kb, striped, causal);
+        kend = key_tile_end(bm, x_last, c);
+        kt = 0;
+        continue;
+      }
+      const int y = kt * kBN;
+      ++kt;
+      const int a = tile_kind(bm, x0, y, c);
+      const int b = tile_kind(bm, x0 + kBM, y, c);
+      if (a == TILE_SKIP && b == TILE_SKIP) continue;
+      kb_out = kb; y0 = y; k0 = a; k1 = b; m = bm;
+      return true;
+    }
+  }
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase + C::kQOff;
+  const uint32_t sRing = sbase + C::kRingOff;
+  const uint32_t bars = sbase + C::kBarOff;
+  const uint32_t bar_q_full = bars + 0 * 8;
+  const uint32_t bar_q_empty = bars + 1 * 8;
+  auto bar_full = [&](int s) { return bars + (2 + s) * 8; };
+  auto bar_empty = [&](int s) { return bars + (2 + C::kSlots + s) * 8; };
+  const uint32_t bar_s_full = bars + (2 + 2 * C::kSlots) * 8;   // [2]
+  const uint32_t bar_p_full = bar_s_full + 16;                  // [2]
+  const uint32_t bar_o_full = bar_p_full + 16;                  // [2]
+  const uint32_t bar_o_free = bar_o_full + 16;                  // [2]
+  const uint32_t bar_drain = bar_o_free + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q_full, 1);
+    mbar_init(bar_q_empty, 1);
+    for (int s = 0; s < C::kSlots; ++s) {
+      mbar_init(bar_full(s), 1);
+      mbar_init(bar_empty(s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar_s_full + 8 * t, 1);
+      mbar_init(bar_p_full + 8 * t, 128);
+      mbar_init(bar_o_full + 8 * t, 1);
+      mbar_init(bar_o_free + 8 * t, 128);
+    }
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t n_loads = 0;
+      Item it;
+      bool ok = true;
+      for (int k = 0; ok && cta_item(p, k, it); ++k) {
+        if (!mbar_wait(bar_q_empty, (k & 1) ^ 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+        mbar_arrive_expect_tx(bar_q_full, 2 * C::kTileBytes);
+        const int x0 = it.pair * 2 * kBM;
+        for (int t = 0; t < 2; ++t)
+          for (int ch = 0; ch < C::kChunks; ++ch)
+            tma_load_4d(sQ + t * C::kTileBytes + ch * 16384, &tmQ, bar_q_full, ch * 64,
+                        x0 + t * kBM, it.j, it.bh);
+        TileSeq seq;
+        seq.init(p, it);
+        int kb, y0, k0, k1;
+        BlockMask bm;
+        while (seq.next(kb, y0, k0, k1, bm)) {
+          for (int kv = 0; kv < 2; ++kv) {
+            const int s = n_loads % C::kSlots;
+            const uint32_t ph = (n_loads / C::kSlots) & 1;
+            if (!mbar_wait(bar_empty(s), ph ^ 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+            mbar_arrive_expect_tx(bar_full(s), C::kTileBytes);
+            const CUtensorMap* tm = kv ? &tmV : &tmK;
+            for (int ch = 0; ch < C::kChunks; ++ch)
+              tma_load_4d(sRing + s * C::kTileBytes + ch * 16384, tm, bar_full(s), ch * 64, y0,
+                          kb, it.bh);
+            ++n_loads;
+          }
+          if (!ok) break;
+        }
+      }
+      // Every load this thread issued must have landed before the CTA exits.
+      volatile int no_abort = 0;
+      const uint32_t first = n_loads > (uint32_t)C::kSlots ? n_loads - C::kSlots : 0;
+      for (uint32_t n = first; n < n_loads; ++n)
+        mbar_wait(bar_full(n % C::kSlots), (n / C::kSlots) & 1, &no_abort, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, 0, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, 0, 1);
+      const uint32_t tS[2] = {tmem + C::kColS0, tmem + C::kColS1};
+      const uint32_t tO[2] = {tmem + C::kColO0, tmem + C::kColO1};
+      uint32_t n_loads = 0;   // K/V tiles consumed, in producer order
+      uint32_t p_cnt[2] = {0, 0};
+      Item it;
+      bool ok = true;
+
+      auto issue_qk = [&](int t, uint32_t kslot) {
+        const uint32_t qa = sQ + t * C::kTileBytes;
+        const uint32_t ka = sRing + kslot * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
+          mma_ss(tS[t], smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024),
+                 idesc_qk, kk > 0);
+        }
+        mma_commit(bar_s_full + 8 * t);
+      };
+      auto issue_pv = [&](int t, uint32_t vslot, uint32_t acc) {
+        const uint32_t va = sRing + vslot * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          mma_ts(tO[t], tS[t] + kk * 8, smem_desc_sw128(va + kk * 2048, 16384, 1024), idesc_pv,
+                 (acc | (uint32_t)kk) != 0);
+      };
+
+      for (int k = 0; ok && cta_item(p, k, it); ++k) {
+        if (!mbar_wait(bar_q_full, k & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+        tc_fence_after();
+        TileSeq seq;
+        seq.init(p, it);
+        int kb, y0, c0, c1, nkb, ny0, n0, n1;
+        BlockMask bm;
+        uint32_t acc[2] = {0, 0};
+        bool have = seq.next(kb, y0, c0, c1, bm);
+        // prologue: Q K^T of the first tile
+        uint32_t kslot = n_loads % C::kSlots;
+        if (!mbar_wait(bar_full(kslot), (n_loads / C::kSlots) & 1, abort_flag, p.timeout_ns)) {
+          ok = false; break;
+        }
+        tc_fence_after();
+        if (c0 != TILE_SKIP) issue_qk(0, kslot);
+        if (c1 != TILE_SKIP) issue_qk(1, kslot);
+        mma_commit(bar_empty(kslot));
+        ++n_loads;
+        while (have) {
+          const bool more = seq.next(nkb, ny0, n0, n1, bm);
+          const uint32_t vslot = n_loads % C::kSlots;
+          const uint32_t vph = (n_loads / C::kSlots) & 1;
+          ++n_loads;
+          uint32_t nkslot = 0;
+          if (more) {
+            nkslot = n_loads % C::kSlots;
+            if (!mbar_wait(bar_full(nkslot), (n_loads / C::kSlots) & 1, abort_flag,
+                           p.timeout_ns)) { ok = false; break; }
+            ++n_loads;
+          }
+          if (!mbar_wait(bar_full(vslot), vph, abort_flag, p.timeout_ns)) { ok = false; break; }
+          tc_fence_after();
+          const int cur[2] = {c0, c1};
+          const int nxt[2] = {n0, n1};
+          for (int t = 0; t < 2; ++t) {
+            if (cur[t] != TILE_SKIP) {
+              if (acc[t] == 0 && k > 0) {
+                if (!mbar_wait(bar_o_free + 8 * t, (k - 1) & 1, abort_flag, p.timeout_ns)) {
+                  ok = false; break;
+                }
+              }
+              if (!mbar_wait(bar_p_full + 8 * t, p_cnt[t] & 1, abort_flag, p.timeout_ns)) {
+                ok = false; break;
+              }
+              ++p_cnt[t];
+              tc_fence_after();
+              issue_pv(t, vslot, acc[t]);
+              acc[t] = 1;
+            }
+            if (t == 1) mma_commit(bar_empty(vslot));
+            if (more && nxt[t] != TILE_SKIP) issue_qk(t, nkslot);
+          }
+          if (!ok) break;
+          if (more) mma_commit(bar_empty(nkslot));
+          have = more;
+          c0 = n0; c1 = n1;
+        }
+        if (!ok) break;
+        mma_commit(bar_o_full + 0);
+        mma_commit(bar_o_full + 8);
+        mma_commit(bar_q_empty);
+      }
+      // All MMAs issued by this thread must be complete before TMEM is freed.
+      mma_commit(bar_drain);
+      volatile int no_abort = 0;
+      mbar_wait(bar_drain, 0, &no_abort, p.timeout_ns);
+    }
+    __syncwarp();
+  } else {
+    // ----------------------------------------------------- softmax warpgroups
+    const int t = warp / 4;                 // query tile of the pair
+    const int wq = warp % 4;                // TMEM lane quarter
+    const int row = wq * 32 + lane;         // row within the query tile
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + (t ? C::kColS1 : C::kColS0) + lane_off;
+    const uint32_t tO = tmem + (t ? C::kColO1 : C::kColO0) + lane_off;
+    const uint32_t my_s_full = bar_s_full + 8 * t;
+    const uint32_t my_p_full = bar_p_full + 8 * t;
+    const uint32_t my_o_full = bar_o_full + 8 * t;
+    const uint32_t my_o_free = bar_o_free + 8 * t;
+    const float c2 = p.c2;
+    uint32_t s_cnt = 0;
+    Item it;
+    bool ok = true;
+    for (int k = 0; ok && cta_item(p, k, it); ++k) {
+      TileSeq seq;
+      seq.init(p, it);
+      const int x = it.pair * 2 * kBM + t * kBM + row;   // local query row in shard
+      float m2 = -INFINITY;   // running max, in units of log2 (scores * c2)
+      float l = 0.f;
+      bool acc = false;
+      int kb, y0, k0, k1;
+      BlockMask bm;
+      while (seq.next(kb, y0, k0, k1, bm)) {
+        const int kind = t ? k1 : k0;
+        if (kind == TILE_SKIP) continue;
+        if (!mbar_wait(my_s_full, s_cnt & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+        ++s_cnt;
+        tc_fence_after();
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, sr[q]);
+        tmem_wait_ld();
+        float s[128];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[q * 32 + i] = __uint_as_float(sr[q][i]);
+        if (kind == TILE_PARTIAL) {
+          const int lim = row_limit(bm, x, y0, p.c);
+#pragma unroll
+          for (int i = 0; i < 128; ++i)
+            if (i >= lim) s[i] = -INFINITY;
+        }
+        float mx = s[0];
+#pragma unroll
+        for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
+        const float m_cand = fmaxf(m2, mx * c2);
+        const bool need = m_cand > m2 + 8.0f;
+        if (__any_sync(0xffffffffu, need)) {
+          const float alpha = (m_cand == -INFINITY) ? 1.f : ex2(m2 - m_cand);
+          if (acc) {
+#pragma unroll 1
+            for (int q = 0; q < D / 32; ++q) {
+              uint32_t orow[32];
+              tmem_ld32(tO + q * 32, orow);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                orow[i] = __float_as_uint(__uint_as_float(orow[i]) * alpha);
+              tmem_st32(tO + q * 32, orow);
+            }
+          }
+          l *= alpha;
+          m2 = m_cand;
+        }
+        const float msub = (m2 == -INFINITY) ? 0.f : m2;
+        uint32_t pk[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const float p0 = ex2(fmaf(s[2 * i], c2, -msub));
+          const float p1 = ex2(fmaf(s[2 * i + 1], c2, -msub));
+          l += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+        tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(my_p_full);
+        acc = true;
+      }
+      if (!ok) break;
+      // --------------------------------------------------------- epilogue
+      if (!mbar_wait(my_o_full, k & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+      tc_fence_after();
+      const bool valid = x < p.c;
+      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      const size_t grow = (size_t)it.bh * p.N + (size_t)it.j * p.c + (size_t)(valid ? x : 0);
+      __nv_bfloat16* orow_g = p.o + grow * D;
+#pragma unroll 1
+      for (int q = 0; q < D / 32; ++q) {
+        uint32_t orow[32];
+        tmem_ld32(tO + q * 32, orow);
+        tmem_wait_ld();
+        if (valid) {
+          uint4 v[4];
+          uint32_t* w = reinterpret_cast<uint32_t*>(v);
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            w[i] = pack_bf16x2(__uint_as_float(orow[2 * i]) * inv_l,
+                               __uint_as_float(orow[2 * i + 1]) * inv_l);
+          uint4* dst = reinterpret_cast<uint4*>(orow_g + q * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = v[i];
+        }
+      }
+      if (valid) p.lse[grow] = (m2 + __log2f(l)) * 0.69314718055994530942f;
+      tc_fence_before();
+      mbar_arrive(my_o_free);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) atomicOr(&g_device_fault, 1u);
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ host
+static bool encode_qkv_map(CUtensorMap* map, const void* base, int64_t BH, int64_t N, int64_t c,
+                           int P, int d) {
+  PFN_encodeTiled enc = get_encode_tiled();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)c, (cuuint64_t)P, (cuuint64_t)BH};
+  cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)c * d * 2, (cuuint64_t)N * d * 2};
+  cuuint32_t box[4] = {64, (cuuint32_t)kBM, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D>
+static ra_status launch(const AttnLaunch& a) {
+  using C = Cfg<D>;
+  CUtensorMap tq, tk, tv;
+  const int64_t c = a.N / a.P;
+  if (!encode_qkv_map(&tq, a.q, a.BH, a.N, c, a.P, D) ||
+      !encode_qkv_map(&tk, a.k, a.BH, a.N, c, a.P, D) ||
+      !encode_qkv_map(&tv, a.v, a.BH, a.N, c, a.P, D))
+    return RA_ERR_CUDA;
+  static int attr_set[64] = {0};
+  if (a.device < 64 && !attr_set[a.device]) {
+    if (cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes) != cudaSuccess)
+      return RA_ERR_CUDA;
+    attr_set[a.device] = 1;
+  }
+  AttnParams p;
+  p.o = reinterpret_cast<__nv_bfloat16*>(a.o);
+  p.lse = a.lse;
+  p.BH = (int)a.BH;
+  p.N = (int)a.N;
+  p.c = (int)c;
+  p.P = a.P;
+  const int T = (int)((c + kBM - 1) / kBM);
+  p.npairs = (T + 1) / 2;
+  p.striped = a.striped;
+  p.causal = a.causal;
+  p.c2 = (float)((double)a.scale * 1.4426950408889634074);
+  p.timeout_ns = 2000000000ull;
+  const long long items_total = (long long)p.npairs * a.P * a.BH;
+  int grid;
+  if (a.sched_free) {
+    p.groups = 1;
+    grid = (int)(items_total < a.num_sms ? items_total : a.num_sms);
+    p.ctas_per_group = grid;
+  } else {
+    p.groups = a.P < a.num_sms ? a.P : a.num_sms;
+    int G = a.num_sms / p.groups;
+    const long long per_group =
+        (long long)p.npairs * a.BH * ((a.P + p.groups - 1) / p.groups);
+    if (per_group < G) G = (int)per_group;
+    p.ctas_per_group = G;
+    grid = G * p.groups;
+  }
+  attn_fwd_kernel<D><<<grid, C::kThreads, C::kSmemBytes, (cudaStream_t)a.stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
+ra_status attn_fwd_launch(const AttnLaunch& a) {
+  if (a.d == 128) return launch<128>(a);
+  if (a.d == 64) return launch<64>(a);
+  return RA_ERR_HEADDIM;
+}
+
+ra_status read_device_fault(int* code) {
+  unsigned int v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return RA_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&v, g_device_fault, sizeof(v)) != cudaSuccess) return RA_ERR_CUDA;
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbol(g_device_fault, &zero, sizeof(zero)) != cudaSuccess) return RA_ERR_CUDA;
+  *code = (int)v;
+  return v ? RA_ERR_DEVICE_FAULT : RA_OK;
+}
+
+}  // namespace ra

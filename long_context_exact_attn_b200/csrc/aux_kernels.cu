@@ -1,0 +1,195 @@
+// Memory-bound helpers of the ring: layout permutation (ra_partition), the
+// (O, lse) merge (ra_lse_merge) and the tile census (ra_tile_census).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ra_internal.h"
+#include "ra_tiles.cuh"
+
+namespace ra {
+
+// ------------------------------------------------------------- partition
+// Row n of the destination (within one (b, h)) comes from source row
+//   forward (token -> layout): slot n holds token (n % c) * P + n / c
+//   inverse (layout -> token): token n sits in slot (n % P) * c + n / P
+// (striped placement of the Striped Attention review, 分区策略对比).
+template <typename U>
+__global__ void partition_kernel(const U* __restrict__ src, U* __restrict__ dst, int rows_total,
+                                 int N, int P, int c, int upr, int rows_per_block, int inverse) {
+  const int row0 = blockIdx.x * rows_per_block;
+  int nrows = rows_total - row0;
+  if (nrows > rows_per_block) nrows = rows_per_block;
+  const int units = nrows * upr;
+  for (int u = threadIdx.x; u < units; u += blockDim.x) {
+    const int rl = u / upr;
+    const int e = u - rl * upr;
+    const int row = row0 + rl;
+    const int bh = row / N;
+    const int n = row - bh * N;
+    int sn;
+    if (inverse) {
+      const int sh = n % P;
+      sn = sh * c + n / P;
+    } else {
+      const int sh = n / c;
+      sn = (n - sh * c) * P + sh;
+    }
+    dst[(size_t)row * upr + e] = src[((size_t)bh * N + sn) * upr + e];
+  }
+}
+
+template <typename U>
+static ra_status launch_partition_t(const void* src, void* dst, int rows_total, int N, int P,
+                                    int64_t row_bytes, int inverse, void* stream) {
+  const int upr = (int)(row_bytes / (int64_t)sizeof(U));
+  int rpb = 2048 / upr;
+  if (rpb < 1) rpb = 1;
+  const int blocks = (rows_total + rpb - 1) / rpb;
+  partition_kernel<U><<<blocks, 256, 0, (cudaStream_t)stream>>>(
+      reinterpret_cast<const U*>(src), reinterpret_cast<U*>(dst), rows_total, N, P, N / P, upr,
+      rpb, inverse);
+  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
+ra_status partition_launch(const void* src, void* dst, int64_t rows_outer, int64_t N, int64_t P,
+                           int64_t row_bytes, int striped, int inverse, void* stream) {
+  const int64_t total_bytes = rows_outer * N * row_bytes;
+  if (total_bytes == 0) return RA_OK;
+  if (!striped) {
+    // the contiguous placement is the identity
+    return cudaMemcpyAsync(dst, src, (size_t)total_bytes, cudaMemcpyDeviceToDevice,
+                           (cudaStream_t)stream) == cudaSuccess
+               ? RA_OK
+               : RA_ERR_CUDA;
+  }
+  const int rows_total = (int)(rows_outer * N);
+  const uintptr_t al = reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst);
+  if (row_bytes % 16 == 0 && al % 16 == 0)
+    return launch_partition_t<uint4>(src, dst, rows_total, (int)N, (int)P, row_bytes, inverse,
+                                     stream);
+  if (row_bytes % 8 == 0 && al % 8 == 0)
+    return launch_partition_t<uint2>(src, dst, rows_total, (int)N, (int)P, row_bytes, inverse,
+                                     stream);
+  if (row_bytes % 4 == 0 && al % 4 == 0)
+    return launch_partition_t<uint32_t>(src, dst, rows_total, (int)N, (int)P, row_bytes,
+                                        inverse, stream);
+  if (row_bytes % 2 == 0 && al % 2 == 0)
+    return launch_partition_t<uint16_t>(src, dst, rows_total, (int)N, (int)P, row_bytes,
+                                        inverse, stream);
+  return launch_partition_t<uint8_t>(src, dst, rows_total, (int)N, (int)P, row_bytes, inverse,
+                                     stream);
+}
+
+// -------------------------------------------------------------- lse merge
+// One warp per row: every lane reads both lse values before lane 0 writes
+// lse_out (which may alias lse_a); each 8-element chunk of o is read and
+// written by the same lane (o_out may alias o_a).
+__global__ void lse_merge_kernel(const uint4* oa, const float* lse_a,
+                                 const uint4* __restrict__ ob, const float* lse_b, uint4* oo,
+                                 float* lse_o, long long rows, int chunks) {
+  const int lane = threadIdx.x & 31;
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long r = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows;
+       r += warps) {
+    const float la = lse_a[r];
+    const float lb = lse_b[r];
+    const float mx = fmaxf(la, lb);
+    float wa = 0.f, wb = 0.f, lse = -INFINITY;
+    if (mx != -INFINITY) {
+      const float ea = __expf(la - mx);
+      const float eb = __expf(lb - mx);
+      const float s = ea + eb;
+      wa = ea / s;
+      wb = eb / s;
+      lse = mx + __logf(s);
+    }
+    __syncwarp();
+    for (int ch = lane; ch < chunks; ch += 32) {
+      const size_t idx = (size_t)r * chunks + ch;
+      const uint4 a = oa[idx];
+      const uint4 b = ob[idx];
+      const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+      uint4 out;
+      __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(&out);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 fa = __bfloat1622float2(a2[i]);
+        const float2 fb = __bfloat1622float2(b2[i]);
+        o2[i] = __floats2bfloat162_rn(wa * fa.x + wb * fb.x, wa * fa.y + wb * fb.y);
+      }
+      oo[idx] = out;
+    }
+    if (lane == 0) lse_o[r] = lse;
+    __syncwarp();
+  }
+}
+
+ra_status lse_merge_launch(const void* o_a, const float* lse_a, const void* o_b,
+                           const float* lse_b, void* o_out, float* lse_out, int64_t rows,
+                           int64_t d, int num_sms, void* stream) {
+  if (rows == 0) return RA_OK;
+  const int chunks = (int)(d / 8);
+  long long blocks = (rows + 7) / 8;
+  const long long cap = (long long)num_sms * 16;
+  if (blocks > cap) blocks = cap;
+  lse_merge_kernel<<<(int)blocks, 256, 0, (cudaStream_t)stream>>>(
+      reinterpret_cast<const uint4*>(o_a), lse_a, reinterpret_cast<const uint4*>(o_b), lse_b,
+      reinterpret_cast<uint4*>(o_out), lse_out, (long long)rows, chunks);
+  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------ tile census
+// One thread per (query shard j, round r, query tile qt); classification and
+// per-row limits are the attention kernel's own (ra_tiles.cuh).
+__global__ void tile_census_kernel(int c, int P, int T, int striped, int causal,
+                                   unsigned long long* out) {
+  const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (tid >= (long long)P * P * T) return;
+  const int qt = (int)(tid % T);
+  const int jr = (int)(tid / T);
+  const int j = jr / P;
+  const int r = jr % P;
+  const int kb = key_block(j, r, P);
+  const BlockMask bm = block_mask(j, kb, striped, causal);
+  const int x0 = qt * kBM;
+  const int rows = tile_rows(x0, c);
+  unsigned long long cnt[3] = {0, 0, 0};
+  unsigned long long pairs = 0;
+  for (int kt = 0; kt < T; ++kt) {
+    const int y0 = kt * kBN;
+    const int kind = tile_kind(bm, x0, y0, c);
+    ++cnt[kind];
+    if (kind == TILE_FULL) {
+      pairs += (unsigned long long)rows * kBN;
+    } else if (kind == TILE_PARTIAL) {
+      for (int i = 0; i < rows; ++i) {
+        int lim = row_limit(bm, x0 + i, y0, c);
+        lim = lim < 0 ? 0 : (lim > kBN ? kBN : lim);
+        pairs += (unsigned long long)lim;
+      }
+    }
+  }
+  unsigned long long* o = out + (size_t)(j * P + r) * 4;
+  atomicAdd(o + 0, cnt[0]);
+  atomicAdd(o + 1, cnt[1]);
+  atomicAdd(o + 2, cnt[2]);
+  atomicAdd(o + 3, pairs);
+}
+
+ra_status tile_census_launch(int64_t N, int P, int striped, int causal, int64_t* out,
+                             void* stream) {
+  const int c = (int)(N / P);
+  const int T = (c + kBM - 1) / kBM;
+  if (cudaMemsetAsync(out, 0, sizeof(int64_t) * 4 * (size_t)P * P, (cudaStream_t)stream) !=
+      cudaSuccess)
+    return RA_ERR_CUDA;
+  const long long threads = (long long)P * P * T;
+  const int blocks = (int)((threads + 127) / 128);
+  tile_census_kernel<<<blocks, 128, 0, (cudaStream_t)stream>>>(
+      c, P, T, striped, causal, reinterpret_cast<unsigned long long*>(out));
+  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
+}  // namespace ra

@@ -1,0 +1,47 @@
+// Internal interfaces between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <stdint.h>
+
+#include "../../include/ringattn.h"
+
+namespace ra {
+
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                    const cuuint32_t*, CUtensorMapInterleave,
+                                    CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                    CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled from the driver, looked up once (NULL on failure).
+PFN_encodeTiled get_encode_tiled();
+
+struct AttnLaunch {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  float* lse;
+  int64_t BH, N, d;
+  int P;
+  int striped, causal, sched_free;
+  float scale;
+  int device, num_sms;
+  void* stream;
+};
+
+ra_status attn_fwd_launch(const AttnLaunch& a);
+ra_status read_device_fault(int* code);
+
+ra_status partition_launch(const void* src, void* dst, int64_t rows_outer, int64_t N, int64_t P,
+                           int64_t row_bytes, int striped, int inverse, void* stream);
+
+ra_status lse_merge_launch(const void* o_a, const float* lse_a, const void* o_b,
+                           const float* lse_b, void* o_out, float* lse_out, int64_t rows,
+                           int64_t d, int num_sms, void* stream);
+
+ra_status tile_census_launch(int64_t N, int P, int striped, int causal, int64_t* out,
+                             void* stream);
+
+}  // namespace ra

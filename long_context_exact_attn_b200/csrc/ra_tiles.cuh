@@ -1,0 +1,120 @@
+// Tile schedule and causal masks of the virtual-shard ring, shared by the
+// attention kernel and the tile-census kernel (host and device).
+//
+// Geometry.  The sequence of N tokens is stored in LAYOUT order: P shards of
+// c = N / P rows each, shard after shard.  Shard j holds
+//   contiguous ("Ring"):  tokens j*c + x          (Ring Attention explainer,
+//                         ステップ1: シーケンスの分割)
+//   striped:              tokens x*P + j          (Striped Attention review,
+//                         分区策略对比: token t on device t mod P)
+// for local index x in [0, c).
+//
+// Causal mask over ORIGINAL positions (Striped review, 核心公式, matrix C):
+// key (shard kb, local y) is visible to query (shard j, local x) iff its
+// token index is <= the query's.  That reduces, per block pair, to
+//   contiguous: kb < j all visible; kb > j none; kb == j  y <= x
+//   striped:    kb <= j  y <= x;                 kb >  j  y <  x
+// i.e. the two GetMask procedures of the Striped review (GetMask 函数), read
+// with MASK indexed [key, query].  Both are "y < x + e" with e = 1 or 0, so
+// a tile needs one integer limit per query row.
+//
+// Rounds (Ring Attention explainer, ステップ2): in round r the device that
+// owns shard j holds key block kb = (j - r) mod P.
+//
+// Tiles are BM query rows x BN keys inside one (query shard, key block)
+// pair; a ragged last tile of a shard (c not a multiple of the tile) has
+// its out-of-shard rows/columns masked.  A tile is SKIP (nothing visible,
+// never computed), FULL (everything visible, no per-element mask) or
+// PARTIAL (per-element mask) -- the tile skipping of the Striped review,
+// 实现细节 / 分块与分瓦片.
+#pragma once
+
+#include <stdint.h>
+
+#if defined(__CUDACC__)
+#define RA_HD __host__ __device__ __forceinline__
+#else
+#define RA_HD inline
+#endif
+
+namespace ra {
+
+constexpr int kBM = 128;   // query rows per Q tile (one TMEM lane per row)
+constexpr int kBN = 128;   // keys per K/V tile
+
+enum TileKind : int { TILE_SKIP = 0, TILE_FULL = 1, TILE_PARTIAL = 2 };
+
+constexpr int kNoLimit = 0x3fffffff;
+
+// Per (query shard j, key block kb) mask parameters.
+struct BlockMask {
+  int all_hidden;   // whole block masked (contiguous causal, kb > j)
+  int use_diag;     // causal comparison needed (y < x + e)
+  int e;            // 1: key may equal query local index; 0: strictly before
+};
+
+RA_HD BlockMask block_mask(int j, int kb, int layout_striped, int causal) {
+  BlockMask m{0, 0, 1};
+  if (!causal) return m;
+  if (layout_striped) {
+    m.use_diag = 1;
+    m.e = (kb <= j) ? 1 : 0;
+  } else {
+    if (kb > j) {
+      m.all_hidden = 1;
+    } else if (kb == j) {
+      m.use_diag = 1;
+      m.e = 1;
+    }
+  }
+  return m;
+}
+
+// Number of valid query rows in the Q tile starting at local row x0.
+RA_HD int tile_rows(int x0, int c) {
+  int r = c - x0;
+  return r < 0 ? 0 : (r > kBM ? kBM : r);
+}
+
+// Classify the tile (query rows [x0, x0+BM), keys [y0, y0+BN)) of block
+// pair (j, kb).
+RA_HD int tile_kind(const BlockMask& m, int x0, int y0, int c) {
+  const int rows = tile_rows(x0, c);
+  if (rows == 0 || m.all_hidden || y0 >= c) return TILE_SKIP;
+  const int x_last = x0 + rows - 1;
+  if (m.use_diag && y0 >= x_last + m.e) return TILE_SKIP;
+  const bool ragged = (y0 + kBN > c);
+  if (!ragged && (!m.use_diag || y0 + kBN <= x0 + m.e)) return TILE_FULL;
+  return TILE_PARTIAL;
+}
+
+// For a PARTIAL tile: keys with column index col < limit are visible to the
+// query at local row x (col = key local index - y0).  Result may be <= 0
+// (row sees nothing in this tile) or >= BN (row sees the whole tile).
+RA_HD int row_limit(const BlockMask& m, int x, int y0, int c) {
+  int lim = c - y0;
+  if (m.use_diag) {
+    const int d = x + m.e - y0;
+    lim = d < lim ? d : lim;
+  }
+  return lim;
+}
+
+// Number of key tiles of block kb that can hold a visible key for any query
+// of the Q-tile pair whose last valid local row is x_last; tiles at or past
+// this index are skipped for the whole pair.
+RA_HD int key_tile_end(const BlockMask& m, int x_last, int c) {
+  const int T = (c + kBN - 1) / kBN;
+  if (m.all_hidden) return 0;
+  if (!m.use_diag) return T;
+  const int lim = x_last + m.e;             // visible keys: y < lim
+  const int end = (lim + kBN - 1) / kBN;
+  return end < T ? end : T;
+}
+
+RA_HD int key_block(int j, int r, int P) {
+  int kb = j - r;
+  return kb < 0 ? kb + P : kb;
+}
+
+}  // namespace ra

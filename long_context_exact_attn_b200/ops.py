@@ -1,0 +1,181 @@
+"""Python binding of libringattn.so (argument marshalling only).
+
+Every function here validates nothing beyond what is needed to build the
+call, hands raw device pointers, sizes and the current CUDA stream to the
+C ABI (include/ringattn.h), and raises ``RingAttnError`` on a non-zero
+status.  There is no fallback: if the library is missing or the device is
+not an sm_100 GPU, calls fail loudly.
+"""
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libringattn.so")
+
+CONTIGUOUS = 0
+STRIPED = 1
+SCHED_FREE = 0x100
+
+BF16 = 0
+F32 = 1
+I32 = 2
+
+_DTYPE_CODE = {torch.bfloat16: BF16, torch.float32: F32, torch.int32: I32}
+
+_lib = None
+
+
+class RingAttnError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f"{where}: status {status} ({status_string(status)})")
+
+
+def lib():
+    """The loaded C library (loaded on first use; raises if it is missing)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m long_context_exact_attn_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        i64, vp, i32, f32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        L.ra_status_string.restype = ctypes.c_char_p
+        L.ra_status_string.argtypes = [i32]
+        L.ra_version.restype = i32
+        L.ra_version.argtypes = []
+        L.ra_partition.restype = i32
+        L.ra_partition.argtypes = [vp, vp, i64, i64, i64, i64, i32, i32, i32, i32, vp]
+        L.ra_attn_fwd.restype = i32
+        L.ra_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, i32, i32, f32, vp]
+        L.ra_lse_merge.restype = i32
+        L.ra_lse_merge.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, vp]
+        L.ra_tile_census.restype = i32
+        L.ra_tile_census.argtypes = [i64, i32, i32, i32, vp, vp]
+        L.ra_device_fault.restype = i32
+        L.ra_device_fault.argtypes = [ctypes.POINTER(ctypes.c_int)]
+        _lib = L
+    return _lib
+
+
+def status_string(status):
+    return lib().ra_status_string(int(status)).decode()
+
+
+def _check(status, where):
+    if status != 0:
+        raise RingAttnError(status, where)
+
+
+def _stream(t):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _cuda_contig(t, name):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def partition(x, P, layout, inverse=False, out=None):
+    """Token order -> layout order (or back, ``inverse=True``) along dim -2 of
+    a [B, H, N, d] tensor, or along the only dim of an [N] tensor (position
+    ids).  bf16, float32 or int32."""
+    _cuda_contig(x, "x")
+    if x.dtype not in _DTYPE_CODE:
+        raise ValueError(f"unsupported dtype {x.dtype}")
+    if x.dim() == 1:
+        B, H, N, d = 1, 1, x.shape[0], 1
+    elif x.dim() == 4:
+        B, H, N, d = x.shape
+    elif x.dim() == 3:           # [B, H, N] (e.g. lse)
+        B, H, N = x.shape
+        d = 1
+    else:
+        raise ValueError("expected [N], [B, H, N] or [B, H, N, d]")
+    if out is None:
+        out = torch.empty_like(x)
+    if out.shape != x.shape or out.dtype != x.dtype:
+        raise ValueError("out must match x in shape and dtype")
+    _cuda_contig(out, "out")
+    _check(lib().ra_partition(_ptr(x), _ptr(out), B, H, N, d, int(P), int(layout), int(bool(inverse)),
+                              _DTYPE_CODE[x.dtype], _stream(x)), "ra_partition")
+    return out
+
+
+def attn_fwd(q, k, v, P, layout, causal=True, scale=None, sched_free=False, out=None, lse=None):
+    """Exact blockwise attention forward; q, k, v: [B, H, N, d] bf16 CUDA
+    tensors in LAYOUT order.  Returns (o [B, H, N, d] bf16, lse [B, H, N]
+    float32), both in layout order."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _cuda_contig(t, n)
+        if t.dtype != torch.bfloat16:
+            raise ValueError(f"{n} must be bfloat16")
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must all be [B, H, N, d] of the same shape")
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = d ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if out.shape != q.shape or out.dtype != torch.bfloat16:
+        raise ValueError("out must be bf16 of q's shape")
+    if lse.shape != (B, H, N) or lse.dtype != torch.float32:
+        raise ValueError("lse must be float32 [B, H, N]")
+    _cuda_contig(out, "out")
+    _cuda_contig(lse, "lse")
+    lay = int(layout) | (SCHED_FREE if sched_free else 0)
+    _check(lib().ra_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, d, int(P),
+                             lay, int(bool(causal)), float(scale), _stream(q)), "ra_attn_fwd")
+    return out, lse
+
+
+def lse_merge(o_a, lse_a, o_b, lse_b, out=None, lse_out=None):
+    """Merge two partial (o, lse) results over disjoint key sets; o: [..., d]
+    bf16, lse: [...] float32."""
+    if o_b.shape != o_a.shape or lse_a.shape != o_a.shape[:-1] or lse_b.shape != lse_a.shape:
+        raise ValueError("o_a, o_b must match and lse_* must be o's shape without the last dim")
+    if o_a.dtype != torch.bfloat16 or o_b.dtype != torch.bfloat16:
+        raise ValueError("o_a, o_b must be bfloat16")
+    if lse_a.dtype != torch.float32 or lse_b.dtype != torch.float32:
+        raise ValueError("lse_a, lse_b must be float32")
+    d = o_a.shape[-1]
+    rows = o_a.numel() // d
+    if out is None:
+        out = torch.empty_like(o_a)
+    if lse_out is None:
+        lse_out = torch.empty_like(lse_a)
+    for n, t in (("o_a", o_a), ("lse_a", lse_a), ("o_b", o_b), ("lse_b", lse_b), ("out", out),
+                 ("lse_out", lse_out)):
+        _cuda_contig(t, n)
+    _check(lib().ra_lse_merge(_ptr(o_a), _ptr(lse_a), _ptr(o_b), _ptr(lse_b), _ptr(out),
+                              _ptr(lse_out), rows, d, _stream(o_a)), "ra_lse_merge")
+    return out, lse_out
+
+
+def tile_census(N, P, layout, causal, device="cuda"):
+    """int64 [P, P, 4]: per (query shard j, round r): skipped / full /
+    masked tiles and visible pairs, from the attention kernel's classifier."""
+    out = torch.empty((P, P, 4), dtype=torch.int64, device=device)
+    _check(lib().ra_tile_census(int(N), int(P), int(layout), int(bool(causal)), _ptr(out),
+                                _stream(out)), "ra_tile_census")
+    return out
+
+
+def device_fault():
+    """Read and clear the device fault word (synchronises the device)."""
+    code = ctypes.c_int(0)
+    st = lib().ra_device_fault(ctypes.byref(code))
+    if st not in (0, 11):
+        raise RingAttnError(st, "ra_device_fault")
+    return code.value

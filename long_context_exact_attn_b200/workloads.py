@@ -71,19 +71,20 @@ BY_NAME = {w.name: w for w in ALL}
 
 
 def make_qkv(w: Workload, device="cpu"):
-    """q, k, v as bfloat16 [B, H, N, d] tensors, in token order."""
+    """q, k, v as bfloat16 [B, H, N, d] tensors, in token order.
+
+    Each tensor is rounded to bfloat16 right after it is drawn, so that the
+    float32 copies of the long workloads are never all alive at once."""
     g = torch.Generator("cpu").manual_seed(w.seed)
     shape = [w.B, w.H, w.N, w.d]
-    q = torch.randn(shape, generator=g, dtype=torch.float32)
-    k = torch.randn(shape, generator=g, dtype=torch.float32)
-    v = torch.randn(shape, generator=g, dtype=torch.float32)
-    if w.qk_scale_up != 1.0:
-        q = q * w.qk_scale_up
-        k = k * w.qk_scale_up
-    q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))
-    if device != "cpu":
-        q, k, v = (t.to(device) for t in (q, k, v))
-    return q, k, v
+    out = []
+    for i in range(3):
+        t = torch.randn(shape, generator=g, dtype=torch.float32)
+        if i < 2 and w.qk_scale_up != 1.0:
+            t.mul_(w.qk_scale_up)
+        t = t.to(torch.bfloat16)
+        out.append(t.to(device) if device != "cpu" else t)
+    return tuple(out)
 
 
 def make_qkv_head(w: Workload, b: int, h: int):

@@ -1,0 +1,106 @@
+"""The C ABI on the host (no GPU needed): the library loads, exports every
+symbol the header declares, and refuses invalid arguments before touching
+the device."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from long_context_exact_attn_b200 import build, ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ringattn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build(quiet=True)
+    return ops.lib()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ra_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for s in ("ra_partition", "ra_attn_fwd", "ra_lse_merge", "ra_status_string",
+              "ra_tile_census", "ra_device_fault", "ra_version"):
+        assert s in syms
+
+
+def test_library_exports_every_declared_symbol(L):
+    for s in declared_symbols():
+        assert hasattr(L, s), s
+
+
+def test_status_strings(L):
+    assert ops.status_string(0) == "ok"
+    for code in range(1, 12):
+        assert ops.status_string(code) not in ("", "unknown status")
+    assert ops.status_string(999) == "unknown status"
+    assert L.ra_version() >= 100
+
+
+# Fake, never-dereferenced device addresses: every call below must be refused
+# by host validation before any CUDA call.
+A = 1 << 40
+Bp = 2 << 40
+Cp = 3 << 40
+Op = 4 << 40
+Lp = 5 << 40
+vp = ctypes.c_void_p
+
+
+def attn(L, q=A, k=Bp, v=Cp, o=Op, lse=Lp, B=1, H=2, N=1024, d=128, P=4, layout=0, causal=1,
+         scale=0.088):
+    return L.ra_attn_fwd(vp(q), vp(k), vp(v), vp(o), vp(lse), B, H, N, d, P, layout, causal,
+                         scale, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=0), 1), (dict(lse=0), 1),
+    (dict(q=A + 8), 2), (dict(o=Op + 2), 2), (dict(lse=Lp + 4), 2),
+    (dict(N=1000, P=3), 3), (dict(P=0), 3), (dict(N=0), 3), (dict(B=0), 3),
+    (dict(d=96), 4), (dict(d=256), 4),
+    (dict(layout=2), 5), (dict(layout=0x400), 5),
+    (dict(scale=0.0), 6), (dict(scale=float("inf")), 6), (dict(scale=float("nan")), 6),
+    (dict(scale=-1.0), 6),
+    (dict(o=A), 8), (dict(lse=Op + 64), 8),
+])
+def test_attn_fwd_rejects_invalid_arguments(L, kw, code):
+    assert attn(L, **kw) == code
+
+
+def test_partition_rejects_invalid_arguments(L):
+    P = L.ra_partition
+    assert P(None, vp(Bp), 1, 1, 16, 4, 4, 1, 0, 0, None) == 1
+    assert P(vp(A), vp(Bp), 1, 1, 16, 4, 4, 7, 0, 0, None) == 5
+    assert P(vp(A), vp(Bp), 1, 1, 16, 4, 4, 1, 0, 9, None) == 7
+    assert P(vp(A), vp(Bp), 1, 1, 15, 4, 4, 1, 0, 0, None) == 3
+    assert P(vp(A + 2), vp(Bp), 1, 1, 16, 8, 4, 1, 0, 0, None) == 2    # 16-byte rows
+    assert P(vp(A), vp(A + 64), 1, 1, 16, 8, 4, 1, 0, 0, None) == 8    # overlap
+
+
+def test_lse_merge_and_census_reject_invalid_arguments(L):
+    M = L.ra_lse_merge
+    assert M(None, vp(A), vp(Bp), vp(Cp), vp(Op), vp(Lp), 4, 8, None) == 1
+    assert M(vp(A), vp(A + 1024), vp(Bp), vp(Cp), vp(Op), vp(Lp), 4, 12, None) == 3
+    assert M(vp(A + 4), vp(A + 1024), vp(Bp), vp(Cp), vp(Op), vp(Lp), 4, 8, None) == 2
+    assert M(vp(A), vp(Lp), vp(Bp), vp(Cp), vp(A + 16), vp(Lp + 64), 4, 8, None) == 8
+    C = L.ra_tile_census
+    assert C(16, 4, 0, 1, None, None) == 1
+    assert C(16, 3, 0, 1, vp(A), None) == 3
+    assert C(16, 4, 3, 1, vp(A), None) == 5
+    assert L.ra_device_fault(None) == 1
+
+
+def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(ops, "_lib", None)
+    monkeypatch.setattr(ops, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        ops.lib()
