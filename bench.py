@@ -1,0 +1,419 @@
+"""Benchmark: causal ring/striped attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-compare] [--no-cpu-baseline]
+
+One step is the whole hot path over one batch of synthetic input: partition
+Q, K, V into the layout order, the attention forward (all rounds of all
+virtual shards), and un-partition O and lse back to token order.
+
+Metric: useful causal attention TFLOP/s (4*d FLOPs per unmasked query-key
+pair, all heads), with tokens/s and the fraction of the measured dense-BF16
+tensor peak alongside.  The default workload is the stress configuration
+(B=1, H=16, N=262144, d=128, P=16 striped, q/k scaled x3).  Inputs (3 GiB)
+are far larger than L2 (126 MB), so no L2 flush is needed between steps.
+
+With --gpus N > 1 (launched under torchrun) every rank runs its own replica
+of the workload: the work has no exchange step on one GPU, so scaling is
+weak and value = all ranks' useful FLOPs / slowest rank's time.
+
+--impl reference times the CPU oracle (fp64 NumPy, plain definition) on a
+bounded row sample of the same workload, on this machine's host cores.
+"""
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from long_context_exact_attn_b200 import workloads as W  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+SPEC_BF16_TFLOPS = 2250.0
+METRIC = "causal attn fwd useful TFLOP/s & % BF16 tensor peak; tokens/s (1×B200)"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "long_context_exact_attn_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload_name):
+    """DRAM bytes per attention launch from the committed ncu summary, if it
+    was taken on the current kernel sources for this workload (else None)."""
+    path = os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = d.get(workload_name)
+    if not e or e.get("kernel_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # NVML missing: clocks unknown
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            self._stop.wait(0.1)
+
+    def start(self):
+        if self.nv:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------- CPU oracle
+def oracle_head(w, h):
+    q, k, v = W.make_qkv_head(w, 0, h)
+    return h, q.double().numpy(), k.double().numpy(), v.double().numpy()
+
+
+def cpu_oracle_rate(w, budget_s, seed=0, head=None):
+    """Run the oracle's plain definition row by row on a bounded sample of
+    the workload; returns (useful TFLOP/s, description, threads)."""
+    from threadpoolctl import threadpool_info
+
+    from oracle import attention as OA
+
+    rng = np.random.default_rng(seed)
+    h, qn, kn, vn = head if head is not None else oracle_head(w, int(rng.integers(0, w.H)))
+    rows = np.sort(rng.choice(w.N, size=min(w.N, 4096), replace=False))
+    done, flops = 0, 0
+    t0 = time.perf_counter()
+    for i in rows:
+        OA.attention_rows(qn, kn, vn, w.scale, w.causal, [int(i)])
+        flops += 4 * w.d * ((int(i) + 1) if w.causal else w.N)
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    desc = (f"{done} query rows of head {h} (uniform random over the sequence) of {w.name}, "
+            f"each against all its visible keys; fp64 NumPy oracle; {dt:.1f} s")
+    return flops / dt / 1e12, desc, threads
+
+
+def run_reference(args, w, rank):
+    if rank != 0:
+        return
+    vals = []
+    desc = threads = None
+    head = oracle_head(w, w.H - 1)
+    for i in range(args.warmup + args.steps):
+        rate, desc, threads = cpu_oracle_rate(w, args.ref_budget, seed=i, head=head)
+        if i >= args.warmup:
+            vals.append(rate)
+    val = statistics.mean(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": w.useful_flops() / (val * 1e12) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N,
+                                        "d": w.d, "P": w.P, "layout": w.layout_name},
+        "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU path
+class Path:
+    """Device buffers and the step of the hot path for one workload."""
+
+    def __init__(self, ops, w, q, k, v, sched_free=False, layout=None):
+        self.ops, self.w = ops, w
+        self.layout = w.layout if layout is None else layout
+        self.sched_free = sched_free
+        dev = torch.device("cuda", torch.cuda.current_device())
+        self.q, self.k, self.v = (t.to(dev) for t in (q, k, v))
+        self.qp, self.kp, self.vp = (torch.empty_like(t) for t in (self.q, self.k, self.v))
+        self.op = torch.empty_like(self.q)
+        self.o = torch.empty_like(self.q)
+        self.lsep = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+        self.lse = torch.empty_like(self.lsep)
+        self.ev_attn = []
+        self.launches_per_step = 6 if self.layout == W.STRIPED else 1
+
+    def step(self, time_attn=False):
+        ops, w, P, lay = self.ops, self.w, self.w.P, self.layout
+        if lay == W.STRIPED:
+            for src, dst in ((self.q, self.qp), (self.k, self.kp), (self.v, self.vp)):
+                ops.partition(src, P, lay, out=dst)
+            qq, kk, vv = self.qp, self.kp, self.vp
+        else:
+            qq, kk, vv = self.q, self.k, self.v
+        if time_attn:
+            s = torch.cuda.current_stream()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+        ops.attn_fwd(qq, kk, vv, P, lay, w.causal, sched_free=self.sched_free,
+                     out=self.op if lay == W.STRIPED else self.o,
+                     lse=self.lsep if lay == W.STRIPED else self.lse)
+        if time_attn:
+            e1.record(s)
+            self.ev_attn.append((e0, e1))
+        if lay == W.STRIPED:
+            ops.partition(self.op, P, lay, inverse=True, out=self.o)
+            ops.partition(self.lsep, P, lay, inverse=True, out=self.lse)
+
+    def attn_ms(self):
+        torch.cuda.synchronize()
+        ts = [a.elapsed_time(b) for a, b in self.ev_attn]
+        self.ev_attn = []
+        return ts
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def timed(fn, steps, world):
+    barrier(world)
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(steps):
+        fn()
+    e1.record(s)
+    torch.cuda.synchronize()
+    barrier(world)
+    return max_over_ranks(e0.elapsed_time(e1) / steps, world)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=W.STRESS_256K.name, choices=sorted(W.BY_NAME))
+    ap.add_argument("--sched", default="owner", choices=["owner", "free"])
+    ap.add_argument("--no-compare", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--ref-budget", type=float, default=15.0,
+                    help="seconds of CPU work per reference step")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = W.BY_NAME[args.workload]
+
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        return
+
+    from long_context_exact_attn_b200 import ops
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    ops.lib()
+    peaks, peaks_src = load_peaks()
+
+    q, k, v = W.make_qkv(w)
+    path = Path(ops, w, q, k, v, sched_free=(args.sched == "free"))
+
+    for _ in range(args.warmup):
+        path.step()
+    torch.cuda.synchronize()
+    if ops.device_fault():
+        raise RuntimeError("device fault during warm-up")
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    ms = timed(lambda: path.step(time_attn=True), args.steps, world)
+    clocks = sampler.stop()
+    attn_ts = path.attn_ms()
+    if ops.device_fault():
+        raise RuntimeError("device fault during the timed steps")
+    attn_ms = statistics.mean(attn_ts)
+    attn_ms = max_over_ranks(attn_ms, world)
+
+    flops = w.useful_flops()
+    value = flops * world / (ms * 1e-3) / 1e12
+    tokens_s = w.B * w.N * world / (ms * 1e-3)
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (t.pin_memory() for t in (q, k, v))
+        ho = torch.empty(path.o.shape, dtype=path.o.dtype).pin_memory()
+        hl = torch.empty(path.lse.shape, dtype=path.lse.dtype).pin_memory()
+
+        def e2e_step():
+            path.q.copy_(hq, non_blocking=True)
+            path.k.copy_(hk, non_blocking=True)
+            path.v.copy_(hv, non_blocking=True)
+            path.step()
+            ho.copy_(path.o, non_blocking=True)
+            hl.copy_(path.lse, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        e2e_ms = timed(e2e_step, max(1, min(args.steps, 5)), world)
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+        d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+        e2e = {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    # ---- the layout/schedule comparison at equal shapes (attention only)
+    compare = None
+    if not args.no_compare:
+        compare = {}
+        for lay in (W.STRIPED, W.CONTIGUOUS):
+            for sched in ("owner", "free"):
+                pth = path if (lay == w.layout and sched == args.sched) else None
+                if pth is None:
+                    pth = Path(ops, w, q, k, v, sched_free=(sched == "free"), layout=lay)
+                    pth.step()
+                    torch.cuda.synchronize()
+                n = 3
+                for _ in range(n):
+                    pth.step(time_attn=True)
+                t = statistics.median(pth.attn_ms())
+                t = max_over_ranks(t, world)
+                compare[f"{W.LAYOUT_NAMES[lay]}_{sched}"] = {
+                    "attn_ms": round(t, 3), "useful_tflops": round(flops / (t * 1e-3) / 1e12, 1)}
+                if pth is not path:
+                    del pth
+                    torch.cuda.empty_cache()
+        so, co = compare["striped_owner"]["attn_ms"], compare["contiguous_owner"]["attn_ms"]
+        compare["contiguous_over_striped_owner"] = round(co / so, 3)
+        if ops.device_fault():
+            raise RuntimeError("device fault during the layout comparison")
+
+    # ---- CPU oracle baseline (rank 0, one GPU only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, desc, threads = cpu_oracle_rate(w, 15.0)
+        cpu = {"value": rate, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": desc}
+
+    peak_key = "bf16_tflops_sustained"
+    peak = float(peaks.get(peak_key, FALLBACK_PEAKS[peak_key]))
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    traffic = recorded_traffic(w.name)
+    roofline = {"bound": "tensor", "kernel": "attn_fwd_kernel<128>", "achieved": achieved,
+                "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                "peak_source": f"{peaks_src} {peak_key}",
+                "frac_of_burst_peak": achieved / float(peaks.get("bf16_tflops",
+                                                                 FALLBACK_PEAKS["bf16_tflops"])),
+                "frac_of_spec_2250": achieved / SPEC_BF16_TFLOPS,
+                "attn_ms_per_launch": attn_ms,
+                "useful_flops_per_launch": flops}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16; q,k x3 for the stress workload)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "P": w.P,
+                   "layout": w.layout_name, "causal": w.causal, "schedule": args.sched,
+                   "step": "partition q,k,v -> attention -> unpartition o,lse",
+                   "l2": "inputs (3 GiB) larger than L2; no flush",
+                   "parallelism": f"replicas x{world}"},
+        "tokens_per_s": tokens_s,
+        "frac_of_peak": value / world / peak,
+        "gpu_launches": path.launches_per_step * args.steps,
+        "clocks": clocks,
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "layout_compare": compare,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

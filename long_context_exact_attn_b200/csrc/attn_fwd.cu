@@ -436,8 +436,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (int i = 0; i < 64; ++i) {
           const float p0 = ex2(fmaf(s[2 * i], c2, -msub));
           const float p1 = ex2(fmaf(s[2 * i + 1], c2, -msub));
-          l += p0 + p1;
           pk[i] = pack_bf16x2(p0, p1);
+          // The row sum takes the bf16-rounded probabilities that P V uses, so
+          // the weights applied to V are normalised by their own sum.
+          l += __uint_as_float(pk[i] << 16) + __uint_as_float(pk[i] & 0xffff0000u);
         }
         tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
         tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
