@@ -164,6 +164,32 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Packed pairs of fp32 (sm_100 f32x2 arithmetic: one instruction, two lanes).
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unf2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 template <int D>
 __global__ void __launch_bounds__(320, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -328,6 +354,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           tc_fence_after();
           const int cur[2] = {c0, c1};
           const int nxt[2] = {n0, n1};
+#pragma unroll
           for (int t = 0; t < 2; ++t) {
             if (cur[t] != TILE_SKIP) {
               if (acc[t] == 0 && k > 0) {
@@ -383,7 +410,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       seq.init(p, it);
       const int x = it.pair * 2 * kBM + t * kBM + row;   // local query row in shard
       float m2 = -INFINITY;   // running max, in units of log2 (scores * c2)
-      float l = 0.f;
+      float l = 0.f;    // row sum of the probabilities (exact fp32) -> lse
+      float lr = 0.f;   // row sum of the bf16-rounded probabilities P V uses -> O
       bool acc = false;
       int kb, y0, k0, k1;
       BlockMask bm;
@@ -408,9 +436,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           for (int i = 0; i < 128; ++i)
             if (i >= lim) s[i] = -INFINITY;
         }
-        float mx = s[0];
+        // Row max: eight independent chains of 3-input max.
+        float mx8[8];
 #pragma unroll
-        for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
+        for (int a = 0; a < 8; ++a) {
+          float acc = fmax3(s[a], s[a + 8], s[a + 16]);
+#pragma unroll
+          for (int kq = 3; kq < 15; kq += 2) acc = fmax3(acc, s[a + 8 * kq], s[a + 8 * kq + 8]);
+          mx8[a] = fmaxf(acc, s[a + 120]);
+        }
+        const float mx = fmaxf(fmax3(mx8[0], mx8[1], mx8[2]),
+                               fmaxf(fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const float m_cand = fmaxf(m2, mx * c2);
         const bool need = m_cand > m2 + 8.0f;
         if (__any_sync(0xffffffffu, need)) {
@@ -428,21 +464,38 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             }
           }
           l *= alpha;
+          lr *= alpha;
           m2 = m_cand;
         }
         const float msub = (m2 == -INFINITY) ? 0.f : m2;
-        uint32_t pk[64];
+        const uint64_t c2x2 = f2(c2, c2);
+        const uint64_t nm2 = f2(-msub, -msub);
+        uint64_t sum_e[4] = {0, 0, 0, 0};   // exact probabilities (for lse)
+        uint64_t sum_r[4] = {0, 0, 0, 0};   // bf16-rounded probabilities (for O)
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float p0 = ex2(fmaf(s[2 * i], c2, -msub));
-          const float p1 = ex2(fmaf(s[2 * i + 1], c2, -msub));
-          pk[i] = pack_bf16x2(p0, p1);
-          // The row sum takes the bf16-rounded probabilities that P V uses, so
-          // the weights applied to V are normalised by their own sum.
-          l += __uint_as_float(pk[i] << 16) + __uint_as_float(pk[i] & 0xffff0000u);
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int e = ch * 32 + 2 * i;
+            float a0, a1;
+            unf2(ffma2(f2(s[e], s[e + 1]), c2x2, nm2), a0, a1);
+            const float p0 = ex2(a0);
+            const float p1 = ex2(a1);
+            pk[i] = pack_bf16x2(p0, p1);
+            sum_e[i & 3] = fadd2(sum_e[i & 3], f2(p0, p1));
+            sum_r[i & 3] = fadd2(sum_r[i & 3], f2(__uint_as_float(pk[i] << 16),
+                                                  __uint_as_float(pk[i] & 0xffff0000u)));
+          }
+          tmem_st16(tS + ch * 16, pk);
         }
-        tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-        tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+        {
+          float a, b, c_, d_;
+          unf2(fadd2(fadd2(sum_e[0], sum_e[1]), fadd2(sum_e[2], sum_e[3])), a, b);
+          unf2(fadd2(fadd2(sum_r[0], sum_r[1]), fadd2(sum_r[2], sum_r[3])), c_, d_);
+          l += a + b;
+          lr += c_ + d_;
+        }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(my_p_full);
@@ -453,7 +506,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (!mbar_wait(my_o_full, k & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
       tc_fence_after();
       const bool valid = x < p.c;
-      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      // O is normalised by the sum of the rounded weights it was built from;
+      // lse uses the exact sum.
+      const float inv_l = (lr > 0.f) ? 1.f / lr : 0.f;
       const size_t grow = (size_t)it.bh * p.N + (size_t)it.j * p.c + (size_t)(valid ? x : 0);
       __nv_bfloat16* orow_g = p.o + grow * D;
 #pragma unroll 1

@@ -130,7 +130,7 @@ def test_parity_8k_workloads(w):
         assert_close(o[0, h], lse[0, h], o_ref, lse_ref, f"{w.name} head {h}")
     for h in range(1, w.H - 1):   # sampled rows elsewhere
         rows = sample_rows(w, 16, h)
-        o_ref, lse_ref = OA.attention_rows(q[0, h].numpy(), k[0, h].numpy(), v[0, h].numpy(),
+        o_ref, lse_ref = OA.attention_rows(q[0, h].float().numpy(), k[0, h].float().numpy(), v[0, h].float().numpy(),
                                            w.scale, True, rows)
         assert_close(o[0, h, rows], lse[0, h, rows], o_ref, lse_ref, f"{w.name} head {h}")
     # causal row 0 sees only key 0: O row 0 is v_0 exactly
@@ -171,7 +171,7 @@ def test_parity_long_workloads_sampled(w, sched_free):
     o, lse = run_path(q, k, v, w.P, w.layout, w.causal, sched_free)
     for h in (0, w.H // 2, w.H - 1):
         rows = sample_rows(w, 24, h)
-        o_ref, lse_ref = OA.attention_rows(q[0, h].numpy(), k[0, h].numpy(), v[0, h].numpy(),
+        o_ref, lse_ref = OA.attention_rows(q[0, h].float().numpy(), k[0, h].float().numpy(), v[0, h].float().numpy(),
                                            w.scale, True, rows)
         assert_close(o[0, h, rows], lse[0, h, rows], o_ref, lse_ref, f"{w.name} head {h}")
     assert np.array_equal(o[0, :, 0], v[0, :, 0].float().numpy())
