@@ -33,6 +33,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "exp2_poly.h"
 #include "ra_internal.h"
 #include "ra_ptx.cuh"
 #include "ra_tiles.cuh"
@@ -188,6 +189,41 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
+}
+
+// acc += bf16 value (mixed-precision add: bf16 operand, fp32 accumulator).
+__device__ __forceinline__ float add_bf16(float acc, unsigned short h) {
+  asm("add.rn.f32.bf16 %0, %1, %0;" : "+f"(acc) : "h"(h));
+  return acc;
+}
+__device__ __forceinline__ void split_bf16x2(uint32_t v, unsigned short& lo, unsigned short& hi) {
+  asm("mov.b32 {%0, %1}, %2;" : "=h"(lo), "=h"(hi) : "r"(v));
+}
+
+// 2^x for a pair of fp32 values on the FMA/ALU pipes instead of the MUFU:
+// x = j + f with j = round(x) (added to the exponent field) and f in
+// [-1/2, 1/2] (minimax polynomial of exp2_poly.h).  x is clamped below at
+// -125 so that the exponent field stays normal; 2^-125 in place of 0 for a
+// masked score changes no sum at fp32 resolution.
+__device__ __forceinline__ void exp2_poly2(uint64_t x2, float& r0, float& r1) {
+  float x0, x1;
+  unf2(x2, x0, x1);
+  x0 = fmaxf(x0, -125.f);
+  x1 = fmaxf(x1, -125.f);
+  const uint64_t magic = f2(12582912.f, 12582912.f);        // 1.5 * 2^23
+  const uint64_t t = fadd2(f2(x0, x1), magic);               // round to nearest integer
+  const uint64_t j = fadd2(t, f2(-12582912.f, -12582912.f));
+  float j0, j1;
+  unf2(j, j0, j1);
+  const uint64_t fr = fadd2(f2(x0, x1), f2(-j0, -j1));
+  uint64_t p = ffma2(fr, f2(RA_EXP2_C3, RA_EXP2_C3), f2(RA_EXP2_C2, RA_EXP2_C2));
+  p = ffma2(p, fr, f2(RA_EXP2_C1, RA_EXP2_C1));
+  p = ffma2(p, fr, f2(1.f, 1.f));
+  float p0, p1, t0, t1;
+  unf2(p, p0, p1);
+  unf2(t, t0, t1);
+  r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
 template <int D>
@@ -471,28 +507,36 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const uint64_t c2x2 = f2(c2, c2);
         const uint64_t nm2 = f2(-msub, -msub);
         uint64_t sum_e[4] = {0, 0, 0, 0};   // exact probabilities (for lse)
-        uint64_t sum_r[4] = {0, 0, 0, 0};   // bf16-rounded probabilities (for O)
+        float sum_r[4] = {0.f, 0.f, 0.f, 0.f};   // bf16-rounded ones (for O)
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int e = ch * 32 + 2 * i;
-            float a0, a1;
-            unf2(ffma2(f2(s[e], s[e + 1]), c2x2, nm2), a0, a1);
-            const float p0 = ex2(a0);
-            const float p1 = ex2(a1);
+            const uint64_t x2 = ffma2(f2(s[e], s[e + 1]), c2x2, nm2);
+            float p0, p1;
+            if ((i & 3) == 3) {
+              exp2_poly2(x2, p0, p1);          // a quarter of the exps off the MUFU
+            } else {
+              float a0, a1;
+              unf2(x2, a0, a1);
+              p0 = ex2(a0);
+              p1 = ex2(a1);
+            }
             pk[i] = pack_bf16x2(p0, p1);
             sum_e[i & 3] = fadd2(sum_e[i & 3], f2(p0, p1));
-            sum_r[i & 3] = fadd2(sum_r[i & 3], f2(__uint_as_float(pk[i] << 16),
-                                                  __uint_as_float(pk[i] & 0xffff0000u)));
+            unsigned short h0, h1;
+            split_bf16x2(pk[i], h0, h1);
+            sum_r[i & 3] = add_bf16(add_bf16(sum_r[i & 3], h0), h1);
           }
           tmem_st16(tS + ch * 16, pk);
         }
         {
           float a, b, c_, d_;
           unf2(fadd2(fadd2(sum_e[0], sum_e[1]), fadd2(sum_e[2], sum_e[3])), a, b);
-          unf2(fadd2(fadd2(sum_r[0], sum_r[1]), fadd2(sum_r[2], sum_r[3])), c_, d_);
+          c_ = sum_r[0] + sum_r[1];
+          d_ = sum_r[2] + sum_r[3];
           l += a + b;
           lr += c_ + d_;
         }

@@ -20,7 +20,10 @@ Tile census: a block of c x c pairs is cut into tiles of bm x bn (Striped
 review, 实现细节 / 分块与分瓦片: a fully masked tile is skipped).  A tile is
 "skip" if every pair in it is masked, "full" if none is, "partial"
 otherwise.  The ragged tail (c not a multiple of the tile) is counted with
-the tile's out-of-range rows and columns ignored.
+the tile's out-of-range rows ignored.  Reading for a tile cut by the end of
+the key block (y0 + bn > c): its columns past the block hold no key of this
+block, so computing the tile needs a per-element mask even when every
+in-block pair is visible -- it counts as "partial" unless it is skipped.
 """
 
 import numpy as np
@@ -74,7 +77,7 @@ def tile_census_brute_force(j, r, N, P, layout, causal, bm, bn):
             n_blocked = np.count_nonzero(t)
             if n_blocked == t.size:
                 skip += 1
-            elif n_blocked == 0:
+            elif n_blocked == 0 and y0 + bn <= c:
                 full += 1
             else:
                 partial += 1
