@@ -81,26 +81,25 @@ struct Item {
   int bh, j, pair;
 };
 
-// Items of a shard group, in non-increasing order of work: causal striped
-// (and non-causal) work grows with the pair's local index; causal
-// contiguous work grows with the shard index first.
+// Items of a shard group.  Head-major, so that the CTAs running at the same
+// time share one head's K/V blocks in L2; inside a head, work is
+// non-increasing (causal striped and non-causal work grows with the pair's
+// local index, causal contiguous work with the shard index first), so each
+// head's list ends with its lightest items.
 __device__ __forceinline__ bool item_at(const AttnParams& p, int g, int u, Item& it) {
   const int n_sh = (p.P - g + p.groups - 1) / p.groups;   // shards g, g+groups, ...
-  const int per_shard = p.npairs * p.BH;
-  if (u >= n_sh * per_shard) return false;
+  const int per_head = p.npairs * n_sh;
+  if (u >= per_head * p.BH) return false;
+  it.bh = u / per_head;
+  const int rem = u - it.bh * per_head;
   if (p.causal && !p.striped) {
-    const int sh_rank = u / per_shard;
-    const int rem = u - sh_rank * per_shard;
+    const int sh_rank = rem / p.npairs;
     it.j = g + (n_sh - 1 - sh_rank) * p.groups;
-    it.pair = p.npairs - 1 - rem / p.BH;
-    it.bh = rem % p.BH;
+    it.pair = p.npairs - 1 - (rem - sh_rank * p.npairs);
   } else {
-    const int per_pair = n_sh * p.BH;
-    const int pr = u / per_pair;
-    const int rem = u - pr * per_pair;
+    const int pr = rem / n_sh;
     it.pair = p.npairs - 1 - pr;
-    it.j = g + (rem / p.BH) * p.groups;
-    it.bh = rem % p.BH;
+    it.j = g + (rem - pr * n_sh) * p.groups;
   }
   return true;
 }
@@ -226,6 +225,31 @@ __device__ __forceinline__ void exp2_poly2(uint64_t x2, float& r0, float& r1) {
   r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
+// S (TMEM, fp32 128 x 128) = Q tile (smem) x K tile (smem)^T; both K-major
+// with 128-byte swizzle, d/16 MMAs of K = 16.
+template <int D>
+__device__ __forceinline__ void mma_qk(uint32_t s_tmem, uint32_t qa, uint32_t ka) {
+  constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN, 0, 0);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
+    mma_ss(s_tmem, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), idesc,
+           kk > 0);
+  }
+}
+
+// O (TMEM, fp32 128 x D) (+)= P (TMEM, bf16 128 x 128) x V tile (smem, 128
+// keys x D, D contiguous = MN-major, 128-byte swizzle): 8 MMAs of K = 16 keys.
+template <int D>
+__device__ __forceinline__ void mma_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t va,
+                                       uint32_t acc) {
+  constexpr uint32_t idesc = idesc_bf16_f32(kBM, D, 0, 1);
+#pragma unroll
+  for (int kk = 0; kk < kBN / 16; ++kk)
+    mma_ts(o_tmem, p_tmem + kk * 8, smem_desc_sw128(va + kk * 2048, 16384, 1024), idesc,
+           (acc | (uint32_t)kk) != 0);
+}
+
 template <int D>
 __global__ void __launch_bounds__(320, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -326,93 +350,80 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     __syncwarp();
   } else if (warp == 9) {
     // ---------------------------------------------------------- MMA issuer
+    // All state lives in scalars (no arrays indexed at run time, no
+    // by-reference captures): this thread is on the tensor core's critical
+    // path, and anything it keeps in local memory costs a round trip per use.
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, 0, 0);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, 0, 1);
-      const uint32_t tS[2] = {tmem + C::kColS0, tmem + C::kColS1};
-      const uint32_t tO[2] = {tmem + C::kColO0, tmem + C::kColO1};
-      uint32_t n_loads = 0;   // K/V tiles consumed, in producer order
-      uint32_t p_cnt[2] = {0, 0};
+      const uint32_t tS0 = tmem + C::kColS0, tS1 = tmem + C::kColS1;
+      const uint32_t tO0 = tmem + C::kColO0, tO1 = tmem + C::kColO1;
+      const uint32_t sQ0 = sQ, sQ1 = sQ + C::kTileBytes;
+      const uint32_t s_full0 = bar_s_full, s_full1 = bar_s_full + 8;
+      const uint32_t p_full0 = bar_p_full, p_full1 = bar_p_full + 8;
+      const uint32_t o_free0 = bar_o_free, o_free1 = bar_o_free + 8;
+      const uint32_t full0 = bars + 2 * 8, empty0 = bars + (2 + C::kSlots) * 8;
+      uint32_t slot = 0, phase = 0;       // next K/V tile to consume, in producer order
+      uint32_t pc0 = 0, pc1 = 0;          // p_full phases consumed per query tile
       Item it;
       bool ok = true;
-
-      auto issue_qk = [&](int t, uint32_t kslot) {
-        const uint32_t qa = sQ + t * C::kTileBytes;
-        const uint32_t ka = sRing + kslot * C::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
-          mma_ss(tS[t], smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024),
-                 idesc_qk, kk > 0);
-        }
-        mma_commit(bar_s_full + 8 * t);
-      };
-      auto issue_pv = [&](int t, uint32_t vslot, uint32_t acc) {
-        const uint32_t va = sRing + vslot * C::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_ts(tO[t], tS[t] + kk * 8, smem_desc_sw128(va + kk * 2048, 16384, 1024), idesc_pv,
-                 (acc | (uint32_t)kk) != 0);
-      };
-
       for (int k = 0; ok && cta_item(p, k, it); ++k) {
         if (!mbar_wait(bar_q_full, k & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
-        tc_fence_after();
         TileSeq seq;
         seq.init(p, it);
-        int kb, y0, c0, c1, nkb, ny0, n0, n1;
+        int kb, y0, c0, c1, n0 = TILE_SKIP, n1 = TILE_SKIP;
         BlockMask bm;
-        uint32_t acc[2] = {0, 0};
+        uint32_t acc0 = 0, acc1 = 0;
         bool have = seq.next(kb, y0, c0, c1, bm);
         // prologue: Q K^T of the first tile
-        uint32_t kslot = n_loads % C::kSlots;
-        if (!mbar_wait(bar_full(kslot), (n_loads / C::kSlots) & 1, abort_flag, p.timeout_ns)) {
-          ok = false; break;
-        }
+        uint32_t kslot = slot;
+        if (!mbar_wait(full0 + 8 * kslot, phase, abort_flag, p.timeout_ns)) { ok = false; break; }
         tc_fence_after();
-        if (c0 != TILE_SKIP) issue_qk(0, kslot);
-        if (c1 != TILE_SKIP) issue_qk(1, kslot);
-        mma_commit(bar_empty(kslot));
-        ++n_loads;
+        const uint32_t ka0 = sRing + kslot * C::kTileBytes;
+        if (c0 != TILE_SKIP) { mma_qk<D>(tS0, sQ0, ka0); mma_commit(s_full0); }
+        if (c1 != TILE_SKIP) { mma_qk<D>(tS1, sQ1, ka0); mma_commit(s_full1); }
+        mma_commit(empty0 + 8 * kslot);
+        if (++slot == C::kSlots) { slot = 0; phase ^= 1; }
         while (have) {
-          const bool more = seq.next(nkb, ny0, n0, n1, bm);
-          const uint32_t vslot = n_loads % C::kSlots;
-          const uint32_t vph = (n_loads / C::kSlots) & 1;
-          ++n_loads;
+          const bool more = seq.next(kb, y0, n0, n1, bm);
+          const uint32_t vslot = slot, vph = phase;
+          if (++slot == C::kSlots) { slot = 0; phase ^= 1; }
           uint32_t nkslot = 0;
           if (more) {
-            nkslot = n_loads % C::kSlots;
-            if (!mbar_wait(bar_full(nkslot), (n_loads / C::kSlots) & 1, abort_flag,
-                           p.timeout_ns)) { ok = false; break; }
-            ++n_loads;
+            nkslot = slot;
+            if (!mbar_wait(full0 + 8 * nkslot, phase, abort_flag, p.timeout_ns)) { ok = false; break; }
+            if (++slot == C::kSlots) { slot = 0; phase ^= 1; }
           }
-          if (!mbar_wait(bar_full(vslot), vph, abort_flag, p.timeout_ns)) { ok = false; break; }
-          tc_fence_after();
-          const int cur[2] = {c0, c1};
-          const int nxt[2] = {n0, n1};
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            if (cur[t] != TILE_SKIP) {
-              if (acc[t] == 0 && k > 0) {
-                if (!mbar_wait(bar_o_free + 8 * t, (k - 1) & 1, abort_flag, p.timeout_ns)) {
-                  ok = false; break;
-                }
-              }
-              if (!mbar_wait(bar_p_full + 8 * t, p_cnt[t] & 1, abort_flag, p.timeout_ns)) {
-                ok = false; break;
-              }
-              ++p_cnt[t];
-              tc_fence_after();
-              issue_pv(t, vslot, acc[t]);
-              acc[t] = 1;
+          if (!mbar_wait(full0 + 8 * vslot, vph, abort_flag, p.timeout_ns)) { ok = false; break; }
+          const uint32_t va = sRing + vslot * C::kTileBytes;
+          const uint32_t nka = sRing + nkslot * C::kTileBytes;
+          // query tile 0: P0 V, then the next Q0 K^T into the freed S0/P0 columns
+          if (c0 != TILE_SKIP) {
+            if (acc0 == 0 && k > 0 && !mbar_wait(o_free0, (k - 1) & 1, abort_flag, p.timeout_ns)) {
+              ok = false; break;
             }
-            if (t == 1) mma_commit(bar_empty(vslot));
-            if (more && nxt[t] != TILE_SKIP) issue_qk(t, nkslot);
+            if (!mbar_wait(p_full0, pc0 & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+            ++pc0;
+            tc_fence_after();
+            mma_pv<D>(tO0, tS0, va, acc0);
+            acc0 = 1;
           }
-          if (!ok) break;
-          if (more) mma_commit(bar_empty(nkslot));
+          if (more && n0 != TILE_SKIP) { tc_fence_after(); mma_qk<D>(tS0, sQ0, nka); mma_commit(s_full0); }
+          // query tile 1
+          if (c1 != TILE_SKIP) {
+            if (acc1 == 0 && k > 0 && !mbar_wait(o_free1, (k - 1) & 1, abort_flag, p.timeout_ns)) {
+              ok = false; break;
+            }
+            if (!mbar_wait(p_full1, pc1 & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+            ++pc1;
+            tc_fence_after();
+            mma_pv<D>(tO1, tS1, va, acc1);
+            acc1 = 1;
+          }
+          mma_commit(empty0 + 8 * vslot);
+          if (more && n1 != TILE_SKIP) { tc_fence_after(); mma_qk<D>(tS1, sQ1, nka); mma_commit(s_full1); }
+          if (more) mma_commit(empty0 + 8 * nkslot);
           have = more;
-          c0 = n0; c1 = n1;
+          c0 = n0;
+          c1 = n1;
         }
         if (!ok) break;
         mma_commit(bar_o_full + 0);
@@ -561,15 +572,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tmem_ld32(tO + q * 32, orow);
         tmem_wait_ld();
         if (valid) {
-          uint4 v[4];
-          uint32_t* w = reinterpret_cast<uint32_t*>(v);
+          uint32_t w[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             w[i] = pack_bf16x2(__uint_as_float(orow[2 * i]) * inv_l,
                                __uint_as_float(orow[2 * i + 1]) * inv_l);
           uint4* dst = reinterpret_cast<uint4*>(orow_g + q * 32);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = v[i];
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
         }
       }
       if (valid) p.lse[grow] = (m2 + __log2f(l)) * 0.69314718055994530942f;
