@@ -250,6 +250,13 @@ __device__ __forceinline__ void mma_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_
            (acc | (uint32_t)kk) != 0);
 }
 
+// One pair in kPolyEvery of each row's exps goes to the FMA-pipe polynomial
+// (0: all on the MUFU).
+#ifndef RA_POLY_EVERY
+#define RA_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = RA_POLY_EVERY;
+
 template <int D>
 __global__ void __launch_bounds__(320, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -457,8 +464,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       seq.init(p, it);
       const int x = it.pair * 2 * kBM + t * kBM + row;   // local query row in shard
       float m2 = -INFINITY;   // running max, in units of log2 (scores * c2)
-      float l = 0.f;    // row sum of the probabilities (exact fp32) -> lse
-      float lr = 0.f;   // row sum of the bf16-rounded probabilities P V uses -> O
+      float l = 0.f;    // row sum of the probabilities (fp32)
       bool acc = false;
       int kb, y0, k0, k1;
       BlockMask bm;
@@ -495,7 +501,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const float mx = fmaxf(fmax3(mx8[0], mx8[1], mx8[2]),
                                fmaxf(fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const float m_cand = fmaxf(m2, mx * c2);
-        const bool need = m_cand > m2 + 8.0f;
+        // Rescale whenever the running max grows: the largest probability of
+        // the row is then exactly 1, so its bf16 rounding in P V costs
+        // nothing (a lazy threshold lets it reach 2^t with an uncovered
+        // rounding error of up to 2^-8 of the dominant term).
+        const bool need = m_cand > m2;
         if (__any_sync(0xffffffffu, need)) {
           const float alpha = (m_cand == -INFINITY) ? 1.f : ex2(m2 - m_cand);
           if (acc) {
@@ -511,14 +521,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             }
           }
           l *= alpha;
-          lr *= alpha;
           m2 = m_cand;
         }
         const float msub = (m2 == -INFINITY) ? 0.f : m2;
         const uint64_t c2x2 = f2(c2, c2);
         const uint64_t nm2 = f2(-msub, -msub);
-        uint64_t sum_e[4] = {0, 0, 0, 0};   // exact probabilities (for lse)
-        float sum_r[4] = {0.f, 0.f, 0.f, 0.f};   // bf16-rounded ones (for O)
+        uint64_t sum_e[4] = {0, 0, 0, 0};   // row sum of the probabilities
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
           uint32_t pk[16];
@@ -527,8 +535,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             const int e = ch * 32 + 2 * i;
             const uint64_t x2 = ffma2(f2(s[e], s[e + 1]), c2x2, nm2);
             float p0, p1;
-            if ((i & 3) == 3) {
-              exp2_poly2(x2, p0, p1);          // a quarter of the exps off the MUFU
+            if (kPolyEvery && (i % kPolyEvery) == kPolyEvery - 1) {
+              exp2_poly2(x2, p0, p1);          // a share of the exps off the MUFU
             } else {
               float a0, a1;
               unf2(x2, a0, a1);
@@ -537,19 +545,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             }
             pk[i] = pack_bf16x2(p0, p1);
             sum_e[i & 3] = fadd2(sum_e[i & 3], f2(p0, p1));
-            unsigned short h0, h1;
-            split_bf16x2(pk[i], h0, h1);
-            sum_r[i & 3] = add_bf16(add_bf16(sum_r[i & 3], h0), h1);
+
           }
           tmem_st16(tS + ch * 16, pk);
         }
         {
-          float a, b, c_, d_;
+          float a, b;
           unf2(fadd2(fadd2(sum_e[0], sum_e[1]), fadd2(sum_e[2], sum_e[3])), a, b);
-          c_ = sum_r[0] + sum_r[1];
-          d_ = sum_r[2] + sum_r[3];
           l += a + b;
-          lr += c_ + d_;
         }
         tmem_wait_st();
         tc_fence_before();
@@ -561,9 +564,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (!mbar_wait(my_o_full, k & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
       tc_fence_after();
       const bool valid = x < p.c;
-      // O is normalised by the sum of the rounded weights it was built from;
-      // lse uses the exact sum.
-      const float inv_l = (lr > 0.f) ? 1.f / lr : 0.f;
+      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
       const size_t grow = (size_t)it.bh * p.N + (size_t)it.j * p.c + (size_t)(valid ? x : 0);
       __nv_bfloat16* orow_g = p.o + grow * D;
 #pragma unroll 1
