@@ -237,12 +237,19 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """Max of a per-rank number over all ranks (nccl: on the device; gloo: host)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_value(flops_per_rank, ms_max, world):
+    """Whole-job useful TFLOP/s: every rank's work over the slowest rank's time."""
+    return flops_per_rank * world / (ms_max * 1e-3) / 1e12
 
 
 def timed(fn, steps, world):
@@ -317,7 +324,7 @@ def main():
     attn_ms = max_over_ranks(attn_ms, world)
 
     flops = w.useful_flops()
-    value = flops * world / (ms * 1e-3) / 1e12
+    value = job_value(flops, ms, world)
     tokens_s = w.B * w.N * world / (ms * 1e-3)
 
     # ---- end to end through the public API with host buffers
