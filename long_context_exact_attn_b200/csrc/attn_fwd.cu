@@ -199,6 +199,19 @@ __device__ __forceinline__ void split_bf16x2(uint32_t v, unsigned short& lo, uns
   asm("mov.b32 {%0, %1}, %2;" : "=h"(lo), "=h"(hi) : "r"(v));
 }
 
+// r[i] *= alpha for 32 fp32 values held as raw bits (packed f32x2 multiplies).
+__device__ __forceinline__ void scale_row32(uint32_t (&r)[32], uint64_t a2) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    uint64_t v = f2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+    asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(v) : "l"(a2));
+    float lo, hi;
+    unf2(v, lo, hi);
+    r[2 * i] = __float_as_uint(lo);
+    r[2 * i + 1] = __float_as_uint(hi);
+  }
+}
+
 // 2^x for a pair of fp32 values on the FMA/ALU pipes instead of the MUFU:
 // x = j + f with j = round(x) (added to the exponent field) and f in
 // [-1/2, 1/2] (minimax polynomial of exp2_poly.h).  x is clamped below at
@@ -506,20 +519,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         // nothing (a lazy threshold lets it reach 2^t with an uncovered
         // rounding error of up to 2^-8 of the dominant term).
         const bool need = m_cand > m2;
-        if (__any_sync(0xffffffffu, need)) {
-          const float alpha = (m_cand == -INFINITY) ? 1.f : ex2(m2 - m_cand);
-          if (acc) {
-#pragma unroll 1
-            for (int q = 0; q < D / 32; ++q) {
-              uint32_t orow[32];
-              tmem_ld32(tO + q * 32, orow);
-              tmem_wait_ld();
-#pragma unroll
-              for (int i = 0; i < 32; ++i)
-                orow[i] = __float_as_uint(__uint_as_float(orow[i]) * alpha);
-              tmem_st32(tO + q * 32, orow);
-            }
-          }
+        // The O rescale itself is deferred until after the exps: it only has
+        // to land before this tile's P V, and by then the scores are dead, so
+        // the whole O row can be loaded at once.
+        const bool rescale = __any_sync(0xffffffffu, need);
+        float alpha = 1.f;
+        if (rescale) {
+          alpha = (m_cand == -INFINITY) ? 1.f : ex2(m2 - m_cand);
           l *= alpha;
           m2 = m_cand;
         }
@@ -553,6 +559,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           float a, b;
           unf2(fadd2(fadd2(sum_e[0], sum_e[1]), fadd2(sum_e[2], sum_e[3])), a, b);
           l += a + b;
+        }
+        if (rescale && acc) {
+          uint32_t o0[32], o1[32], o2[32], o3[32];
+          tmem_ld32(tO + 0, o0);
+          if (D > 32) tmem_ld32(tO + 32, o1);
+          if (D > 64) tmem_ld32(tO + 64, o2);
+          if (D > 96) tmem_ld32(tO + 96, o3);
+          tmem_wait_ld();
+          const uint64_t a2 = f2(alpha, alpha);
+          scale_row32(o0, a2);
+          tmem_st32(tO + 0, o0);
+          if (D > 32) { scale_row32(o1, a2); tmem_st32(tO + 32, o1); }
+          if (D > 64) { scale_row32(o2, a2); tmem_st32(tO + 64, o2); }
+          if (D > 96) { scale_row32(o3, a2); tmem_st32(tO + 96, o3); }
         }
         tmem_wait_st();
         tc_fence_before();
