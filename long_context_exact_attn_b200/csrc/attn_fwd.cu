@@ -306,9 +306,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar_s_full + 8 * t, 1);
-      mbar_init(bar_p_full + 8 * t, 128);
+      mbar_init(bar_p_full + 8 * t, 4);     // one arrival per softmax warp
       mbar_init(bar_o_full + 8 * t, 1);
-      mbar_init(bar_o_free + 8 * t, 128);
+      mbar_init(bar_o_free + 8 * t, 4);
     }
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
@@ -576,7 +576,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(my_p_full);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(my_p_full);
         acc = true;
       }
       if (!ok) break;
@@ -606,7 +607,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
       if (valid) p.lse[grow] = (m2 + __log2f(l)) * 0.69314718055994530942f;
       tc_fence_before();
-      mbar_arrive(my_o_free);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(my_o_free);
     }
   }
 
