@@ -114,41 +114,41 @@ __device__ __forceinline__ bool cta_item(const AttnParams& p, int k, Item& it) {
   return item_at(p, g, u, it);
 }
 
-// The key tiles met by a query-tile pair, in ring order.
+// The key tiles met by a query-tile pair, in ring order.  Per block the two
+// query tiles' FULL / PARTIAL / SKIP thresholds are computed once; per tile
+// the classification is two compares each.
 struct TileSeq {
   int j, P, c, striped, causal;
-  int x0, x_last;           // first row of tile 0, last valid row of the pair
+  int x0;                   // first row of query tile 0
   int r, kt, kend;
+  TileSpan s0, s1;
   BlockMask bm;
   int kb;
 
   __device__ __forceinline__ void init(const AttnParams& p, const Item& it) {
     j = it.j; P = p.P; c = p.c; striped = p.striped; causal = p.causal;
     x0 = it.pair * 2 * kBM;
-    const int rows = tile_rows(x0, c) + tile_rows(x0 + kBM, c);
-    x_last = x0 + rows - 1;
     r = -1; kt = 0; kend = 0;
   }
   // Next tile; false at the end.  Fills block index, key start and the kind
   // of the tile for each of the two query tiles.
   __device__ __forceinline__ bool next(int& kb_out, int& y0, int& k0, int& k1, BlockMask& m) {
-    while (true) {
-      if (kt >= kend) {
-        if (++r >= P) return false;
-        kb = key_block(j, r, P);
-        bm = block_mask(j, kb, striped, causal);
-        kend = key_tile_end(bm, x_last, c);
-        kt = 0;
-        continue;
-      }
-      const int y = kt * kBN;
-      ++kt;
-      const int a = tile_kind(bm, x0, y, c);
-      const int b = tile_kind(bm, x0 + kBM, y, c);
-      if (a == TILE_SKIP && b == TILE_SKIP) continue;
-      kb_out = kb; y0 = y; k0 = a; k1 = b; m = bm;
-      return true;
+    while (kt >= kend) {
+      if (++r >= P) return false;
+      kb = key_block(j, r, P);
+      bm = block_mask(j, kb, striped, causal);
+      s0 = tile_span(bm, x0, c);
+      s1 = tile_span(bm, x0 + kBM, c);
+      kend = s0.part_end > s1.part_end ? s0.part_end : s1.part_end;
+      kt = 0;
     }
+    kb_out = kb;
+    y0 = kt * kBN;
+    k0 = tile_kind_at(s0, kt);
+    k1 = tile_kind_at(s1, kt);
+    m = bm;
+    ++kt;
+    return true;
   }
 };
 

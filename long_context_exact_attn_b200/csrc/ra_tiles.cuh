@@ -44,8 +44,6 @@ constexpr int kBN = 128;   // keys per K/V tile
 
 enum TileKind : int { TILE_SKIP = 0, TILE_FULL = 1, TILE_PARTIAL = 2 };
 
-constexpr int kNoLimit = 0x3fffffff;
-
 // Per (query shard j, key block kb) mask parameters.
 struct BlockMask {
   int all_hidden;   // whole block masked (contiguous causal, kb > j)
@@ -76,16 +74,41 @@ RA_HD int tile_rows(int x0, int c) {
   return r < 0 ? 0 : (r > kBM ? kBM : r);
 }
 
-// Classify the tile (query rows [x0, x0+BM), keys [y0, y0+BN)) of block
-// pair (j, kb).
-RA_HD int tile_kind(const BlockMask& m, int x0, int y0, int c) {
+// Along the key tiles of one block, the tiles of a query tile are FULL for
+// kt < full_end, PARTIAL for full_end <= kt < part_end and SKIP from part_end
+// on (visibility y < min(x + e, c) is monotone in y): one pair of thresholds
+// per (block, query tile) classifies every tile.
+struct TileSpan {
+  int full_end, part_end;
+};
+
+RA_HD TileSpan tile_span(const BlockMask& m, int x0, int c) {
   const int rows = tile_rows(x0, c);
-  if (rows == 0 || m.all_hidden || y0 >= c) return TILE_SKIP;
-  const int x_last = x0 + rows - 1;
-  if (m.use_diag && y0 >= x_last + m.e) return TILE_SKIP;
-  const bool ragged = (y0 + kBN > c);
-  if (!ragged && (!m.use_diag || y0 + kBN <= x0 + m.e)) return TILE_FULL;
-  return TILE_PARTIAL;
+  const int T = (c + kBN - 1) / kBN;
+  TileSpan s{0, 0};
+  if (rows == 0 || m.all_hidden) return s;
+  int part_end = T, full_lim = c;
+  if (m.use_diag) {
+    const int v = x0 + rows - 1 + m.e;      // the last row sees keys y < v
+    const int pe = (v + kBN - 1) / kBN;
+    part_end = pe < T ? pe : T;
+    const int f = x0 + m.e;                 // the first row sees keys y < f
+    full_lim = f < c ? f : c;
+  }
+  int full_end = full_lim / kBN;            // tiles entirely below full_lim
+  s.full_end = full_end < part_end ? full_end : part_end;
+  s.part_end = part_end;
+  return s;
+}
+
+RA_HD int tile_kind_at(const TileSpan& s, int kt) {
+  return kt < s.full_end ? TILE_FULL : (kt < s.part_end ? TILE_PARTIAL : TILE_SKIP);
+}
+
+// Classify the tile (query rows [x0, x0+BM), keys [y0, y0+BN)) of block
+// pair (j, kb); y0 is a multiple of BN.
+RA_HD int tile_kind(const BlockMask& m, int x0, int y0, int c) {
+  return tile_kind_at(tile_span(m, x0, c), y0 / kBN);
 }
 
 // For a PARTIAL tile: keys with column index col < limit are visible to the
@@ -98,18 +121,6 @@ RA_HD int row_limit(const BlockMask& m, int x, int y0, int c) {
     lim = d < lim ? d : lim;
   }
   return lim;
-}
-
-// Number of key tiles of block kb that can hold a visible key for any query
-// of the Q-tile pair whose last valid local row is x_last; tiles at or past
-// this index are skipped for the whole pair.
-RA_HD int key_tile_end(const BlockMask& m, int x_last, int c) {
-  const int T = (c + kBN - 1) / kBN;
-  if (m.all_hidden) return 0;
-  if (!m.use_diag) return T;
-  const int lim = x_last + m.e;             // visible keys: y < lim
-  const int end = (lim + kBN - 1) / kBN;
-  return end < T ? end : T;
 }
 
 RA_HD int key_block(int j, int r, int P) {
