@@ -152,6 +152,14 @@ struct TileSeq {
   }
 };
 
+// mbar_wait for a whole warp: the result is the same in every lane (a lane
+// that gave up makes the warp give up).
+__device__ __forceinline__ bool wmbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+                                           uint64_t limit_ns) {
+  const bool ok = mbar_wait(bar, parity, abort, limit_ns);
+  return __all_sync(0xffffffffu, ok);
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -246,8 +254,8 @@ __device__ __forceinline__ void mma_qk(uint32_t s_tmem, uint32_t qa, uint32_t ka
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
-    mma_ss(s_tmem, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), idesc,
-           kk > 0);
+    mma_ss_w(s_tmem, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024),
+             idesc, kk > 0);
   }
 }
 
@@ -259,8 +267,8 @@ __device__ __forceinline__ void mma_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_
   constexpr uint32_t idesc = idesc_bf16_f32(kBM, D, 0, 1);
 #pragma unroll
   for (int kk = 0; kk < kBN / 16; ++kk)
-    mma_ts(o_tmem, p_tmem + kk * 8, smem_desc_sw128(va + kk * 2048, 16384, 1024), idesc,
-           (acc | (uint32_t)kk) != 0);
+    mma_ts_w(o_tmem, p_tmem + kk * 8, smem_desc_sw128(va + kk * 2048, 16384, 1024), idesc,
+             (acc | (uint32_t)kk) != 0);
 }
 
 // One pair in kPolyEvery of each row's exps goes to the FMA-pipe polynomial
@@ -370,10 +378,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     __syncwarp();
   } else if (warp == 9) {
     // ---------------------------------------------------------- MMA issuer
-    // All state lives in scalars (no arrays indexed at run time, no
-    // by-reference captures): this thread is on the tensor core's critical
-    // path, and anything it keeps in local memory costs a round trip per use.
-    if (lane == 0) {
+    // The whole warp runs this loop with identical values (warp-uniform, so
+    // addresses and descriptors stay in uniform registers); each MMA and
+    // commit is issued by one elected lane.  The issue rate of this warp is
+    // on the tensor core's critical path.
+    {
       const uint32_t tS0 = tmem + C::kColS0, tS1 = tmem + C::kColS1;
       const uint32_t tO0 = tmem + C::kColO0, tO1 = tmem + C::kColO1;
       const uint32_t sQ0 = sQ, sQ1 = sQ + C::kTileBytes;
@@ -386,7 +395,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       Item it;
       bool ok = true;
       for (int k = 0; ok && cta_item(p, k, it); ++k) {
-        if (!mbar_wait(bar_q_full, k & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+        if (!wmbar_wait(bar_q_full, k & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
         TileSeq seq;
         seq.init(p, it);
         int kb, y0, c0, c1, n0 = TILE_SKIP, n1 = TILE_SKIP;
@@ -395,12 +404,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         bool have = seq.next(kb, y0, c0, c1, bm);
         // prologue: Q K^T of the first tile
         uint32_t kslot = slot;
-        if (!mbar_wait(full0 + 8 * kslot, phase, abort_flag, p.timeout_ns)) { ok = false; break; }
+        if (!wmbar_wait(full0 + 8 * kslot, phase, abort_flag, p.timeout_ns)) { ok = false; break; }
         tc_fence_after();
         const uint32_t ka0 = sRing + kslot * C::kTileBytes;
-        if (c0 != TILE_SKIP) { mma_qk<D>(tS0, sQ0, ka0); mma_commit(s_full0); }
-        if (c1 != TILE_SKIP) { mma_qk<D>(tS1, sQ1, ka0); mma_commit(s_full1); }
-        mma_commit(empty0 + 8 * kslot);
+        if (c0 != TILE_SKIP) { mma_qk<D>(tS0, sQ0, ka0); mma_commit_w(s_full0); }
+        if (c1 != TILE_SKIP) { mma_qk<D>(tS1, sQ1, ka0); mma_commit_w(s_full1); }
+        mma_commit_w(empty0 + 8 * kslot);
         if (++slot == C::kSlots) { slot = 0; phase ^= 1; }
         while (have) {
           const bool more = seq.next(kb, y0, n0, n1, bm);
@@ -409,51 +418,51 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           uint32_t nkslot = 0;
           if (more) {
             nkslot = slot;
-            if (!mbar_wait(full0 + 8 * nkslot, phase, abort_flag, p.timeout_ns)) { ok = false; break; }
+            if (!wmbar_wait(full0 + 8 * nkslot, phase, abort_flag, p.timeout_ns)) { ok = false; break; }
             if (++slot == C::kSlots) { slot = 0; phase ^= 1; }
           }
-          if (!mbar_wait(full0 + 8 * vslot, vph, abort_flag, p.timeout_ns)) { ok = false; break; }
+          if (!wmbar_wait(full0 + 8 * vslot, vph, abort_flag, p.timeout_ns)) { ok = false; break; }
           const uint32_t va = sRing + vslot * C::kTileBytes;
           const uint32_t nka = sRing + nkslot * C::kTileBytes;
           // query tile 0: P0 V, then the next Q0 K^T into the freed S0/P0 columns
           if (c0 != TILE_SKIP) {
-            if (acc0 == 0 && k > 0 && !mbar_wait(o_free0, (k - 1) & 1, abort_flag, p.timeout_ns)) {
+            if (acc0 == 0 && k > 0 && !wmbar_wait(o_free0, (k - 1) & 1, abort_flag, p.timeout_ns)) {
               ok = false; break;
             }
-            if (!mbar_wait(p_full0, pc0 & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+            if (!wmbar_wait(p_full0, pc0 & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
             ++pc0;
             tc_fence_after();
             mma_pv<D>(tO0, tS0, va, acc0);
             acc0 = 1;
           }
-          if (more && n0 != TILE_SKIP) { tc_fence_after(); mma_qk<D>(tS0, sQ0, nka); mma_commit(s_full0); }
+          if (more && n0 != TILE_SKIP) { tc_fence_after(); mma_qk<D>(tS0, sQ0, nka); mma_commit_w(s_full0); }
           // query tile 1
           if (c1 != TILE_SKIP) {
-            if (acc1 == 0 && k > 0 && !mbar_wait(o_free1, (k - 1) & 1, abort_flag, p.timeout_ns)) {
+            if (acc1 == 0 && k > 0 && !wmbar_wait(o_free1, (k - 1) & 1, abort_flag, p.timeout_ns)) {
               ok = false; break;
             }
-            if (!mbar_wait(p_full1, pc1 & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+            if (!wmbar_wait(p_full1, pc1 & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
             ++pc1;
             tc_fence_after();
             mma_pv<D>(tO1, tS1, va, acc1);
             acc1 = 1;
           }
-          mma_commit(empty0 + 8 * vslot);
-          if (more && n1 != TILE_SKIP) { tc_fence_after(); mma_qk<D>(tS1, sQ1, nka); mma_commit(s_full1); }
-          if (more) mma_commit(empty0 + 8 * nkslot);
+          mma_commit_w(empty0 + 8 * vslot);
+          if (more && n1 != TILE_SKIP) { tc_fence_after(); mma_qk<D>(tS1, sQ1, nka); mma_commit_w(s_full1); }
+          if (more) mma_commit_w(empty0 + 8 * nkslot);
           have = more;
           c0 = n0;
           c1 = n1;
         }
         if (!ok) break;
-        mma_commit(bar_o_full + 0);
-        mma_commit(bar_o_full + 8);
-        mma_commit(bar_q_empty);
+        mma_commit_w(bar_o_full + 0);
+        mma_commit_w(bar_o_full + 8);
+        mma_commit_w(bar_q_empty);
       }
       // All MMAs issued by this thread must be complete before TMEM is freed.
-      mma_commit(bar_drain);
+      mma_commit_w(bar_drain);
       volatile int no_abort = 0;
-      mbar_wait(bar_drain, 0, &no_abort, p.timeout_ns);
+      wmbar_wait(bar_drain, 0, &no_abort, p.timeout_ns);
     }
     __syncwarp();
   } else {
