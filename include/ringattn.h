@@ -189,6 +189,20 @@ ra_status ra_tile_census(int64_t N, int P, int layout, int causal, int64_t* out,
  */
 ra_status ra_device_fault(int* code);
 
+/*
+ * ra_wait_selftest -- exercise the bounded-wait and fault-reporting path.
+ *
+ * Not an operation of the pages: a diagnostic for the library's failure
+ * detection.  Launches one warp that waits, through the same bounded wait
+ * the attention kernel uses, on a barrier that nothing ever completes.  The
+ * wait gives up after limit_ns nanoseconds of wall time; the kernel then
+ * records fault code 2 in the device fault word and returns, leaving the
+ * CUDA context usable.  Read the code with ra_device_fault().
+ *
+ *   limit_ns  1000 <= limit_ns <= 1e10, else RA_ERR_SHAPE.
+ */
+ra_status ra_wait_selftest(int64_t limit_ns, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -183,6 +183,15 @@ ra_status ra_tile_census(int64_t N, int P, int layout, int causal, int64_t* out,
   return tile_census_launch(N, P, layout == RA_STRIPED, causal != 0, out, stream);
 }
 
+ra_status ra_wait_selftest(int64_t limit_ns, void* stream) {
+  if (limit_ns < 1000 || limit_ns > 10000000000LL) return RA_ERR_SHAPE;
+  int dev;
+  DevInfo info;
+  ra_status st = current_device(&dev, &info);
+  if (st) return st;
+  return wait_selftest_launch(limit_ns, stream);
+}
+
 ra_status ra_device_fault(int* code) {
   if (!code) return RA_ERR_NULL;
   return read_device_fault(code);

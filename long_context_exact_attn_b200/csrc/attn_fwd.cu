@@ -700,6 +700,29 @@ ra_status attn_fwd_launch(const AttnLaunch& a) {
   return RA_ERR_HEADDIM;
 }
 
+// Bounded-wait self-test: one warp initialises an mbarrier that nothing ever
+// arrives on and waits for it through the same bounded wait the attention
+// kernel uses.  The wait gives up after `limit_ns`, the abort path records
+// fault code 2 in the device fault word, and the kernel returns normally.
+__global__ void wait_selftest_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncwarp();
+  const bool ok = mbar_wait(smem_u32(&bar), 0, &abort_flag, limit_ns);
+  __syncwarp();
+  if (threadIdx.x == 0 && (!ok || abort_flag)) atomicOr(&g_device_fault, 2u);
+}
+
+ra_status wait_selftest_launch(int64_t limit_ns, void* stream) {
+  wait_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>((unsigned long long)limit_ns);
+  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
 ra_status read_device_fault(int* code) {
   unsigned int v = 0;
   if (cudaDeviceSynchronize() != cudaSuccess) return RA_ERR_CUDA;

@@ -33,6 +33,7 @@ struct AttnLaunch {
 
 ra_status attn_fwd_launch(const AttnLaunch& a);
 ra_status read_device_fault(int* code);
+ra_status wait_selftest_launch(int64_t limit_ns, void* stream);
 
 ra_status partition_launch(const void* src, void* dst, int64_t rows_outer, int64_t N, int64_t P,
                            int64_t row_bytes, int striped, int inverse, void* stream);

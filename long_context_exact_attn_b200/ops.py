@@ -55,6 +55,8 @@ def lib():
         L.ra_lse_merge.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, vp]
         L.ra_tile_census.restype = i32
         L.ra_tile_census.argtypes = [i64, i32, i32, i32, vp, vp]
+        L.ra_wait_selftest.restype = i32
+        L.ra_wait_selftest.argtypes = [i64, vp]
         L.ra_device_fault.restype = i32
         L.ra_device_fault.argtypes = [ctypes.POINTER(ctypes.c_int)]
         _lib = L
@@ -170,6 +172,13 @@ def tile_census(N, P, layout, causal, device="cuda"):
     _check(lib().ra_tile_census(int(N), int(P), int(layout), int(bool(causal)), _ptr(out),
                                 _stream(out)), "ra_tile_census")
     return out
+
+
+def wait_selftest(limit_ns=100_000_000, device="cuda"):
+    """Launch the bounded-wait self-test (a wait that nothing completes)."""
+    dev = torch.device(device)
+    stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    _check(lib().ra_wait_selftest(int(limit_ns), stream), "ra_wait_selftest")
 
 
 def device_fault():

@@ -29,7 +29,7 @@ def declared_symbols():
 def test_header_declares_the_boundary():
     syms = declared_symbols()
     for s in ("ra_partition", "ra_attn_fwd", "ra_lse_merge", "ra_status_string",
-              "ra_tile_census", "ra_device_fault", "ra_version"):
+              "ra_tile_census", "ra_device_fault", "ra_version", "ra_wait_selftest"):
         assert s in syms
 
 
@@ -97,6 +97,8 @@ def test_lse_merge_and_census_reject_invalid_arguments(L):
     assert C(16, 3, 0, 1, vp(A), None) == 3
     assert C(16, 4, 3, 1, vp(A), None) == 5
     assert L.ra_device_fault(None) == 1
+    assert L.ra_wait_selftest(10, None) == 3
+    assert L.ra_wait_selftest(2 * 10**10, None) == 3
 
 
 def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
