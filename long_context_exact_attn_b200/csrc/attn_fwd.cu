@@ -67,8 +67,9 @@ struct Cfg {
   static constexpr int kRingOff = 2 * kTileBytes;
   static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
   // barriers: q_full, q_empty, full[kSlots], empty[kSlots], s_full[2],
-  // p_full[2], o_full[2], o_free[2], drain
-  static constexpr int kNumBars = 2 + 2 * kSlots + 8 + 1;
+  // p_full[2] (P columns of keys 0-63 ready), p_full2[2] (keys 64-127),
+  // o_full[2], o_free[2], drain
+  static constexpr int kNumBars = 2 + 2 * kSlots + 10 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
   static constexpr uint32_t kTmemCols = 512;
@@ -261,12 +262,12 @@ __device__ __forceinline__ void mma_qk(uint32_t s_tmem, uint32_t qa, uint32_t ka
 
 // O (TMEM, fp32 128 x D) (+)= P (TMEM, bf16 128 x 128) x V tile (smem, 128
 // keys x D, D contiguous = MN-major, 128-byte swizzle): 8 MMAs of K = 16 keys.
-template <int D>
+template <int D, int KK0 = 0, int KK1 = kBN / 16>
 __device__ __forceinline__ void mma_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t va,
                                        uint32_t acc) {
   constexpr uint32_t idesc = idesc_bf16_f32(kBM, D, 0, 1);
 #pragma unroll
-  for (int kk = 0; kk < kBN / 16; ++kk)
+  for (int kk = KK0; kk < KK1; ++kk)
     mma_ts_w(o_tmem, p_tmem + kk * 8, smem_desc_sw128(va + kk * 2048, 16384, 1024), idesc,
              (acc | (uint32_t)kk) != 0);
 }
@@ -296,7 +297,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   auto bar_empty = [&](int s) { return bars + (2 + C::kSlots + s) * 8; };
   const uint32_t bar_s_full = bars + (2 + 2 * C::kSlots) * 8;   // [2]
   const uint32_t bar_p_full = bar_s_full + 16;                  // [2]
-  const uint32_t bar_o_full = bar_p_full + 16;                  // [2]
+  const uint32_t bar_p_full2 = bar_p_full + 16;                 // [2]
+  const uint32_t bar_o_full = bar_p_full2 + 16;                 // [2]
   const uint32_t bar_o_free = bar_o_full + 16;                  // [2]
   const uint32_t bar_drain = bar_o_free + 16;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
@@ -315,6 +317,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar_s_full + 8 * t, 1);
       mbar_init(bar_p_full + 8 * t, 4);     // one arrival per softmax warp
+      mbar_init(bar_p_full2 + 8 * t, 4);
       mbar_init(bar_o_full + 8 * t, 1);
       mbar_init(bar_o_free + 8 * t, 4);
     }
@@ -388,6 +391,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const uint32_t sQ0 = sQ, sQ1 = sQ + C::kTileBytes;
       const uint32_t s_full0 = bar_s_full, s_full1 = bar_s_full + 8;
       const uint32_t p_full0 = bar_p_full, p_full1 = bar_p_full + 8;
+      const uint32_t p_full2_0 = bar_p_full2, p_full2_1 = bar_p_full2 + 8;
       const uint32_t o_free0 = bar_o_free, o_free1 = bar_o_free + 8;
       const uint32_t full0 = bars + 2 * 8, empty0 = bars + (2 + C::kSlots) * 8;
       uint32_t slot = 0, phase = 0;       // next K/V tile to consume, in producer order
@@ -429,10 +433,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             if (acc0 == 0 && k > 0 && !wmbar_wait(o_free0, (k - 1) & 1, abort_flag, p.timeout_ns)) {
               ok = false; break;
             }
+            // P in two halves: the first 4 k-steps (keys 0-63) start while the
+            // softmax is still producing keys 64-127.
             if (!wmbar_wait(p_full0, pc0 & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+            tc_fence_after();
+            mma_pv<D, 0, 4>(tO0, tS0, va, acc0);
+            if (!wmbar_wait(p_full2_0, pc0 & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
             ++pc0;
             tc_fence_after();
-            mma_pv<D>(tO0, tS0, va, acc0);
+            mma_pv<D, 4, 8>(tO0, tS0, va, 1);
             acc0 = 1;
           }
           if (more && n0 != TILE_SKIP) { tc_fence_after(); mma_qk<D>(tS0, sQ0, nka); mma_commit_w(s_full0); }
@@ -441,10 +450,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             if (acc1 == 0 && k > 0 && !wmbar_wait(o_free1, (k - 1) & 1, abort_flag, p.timeout_ns)) {
               ok = false; break;
             }
+            // P in two halves: the first 4 k-steps (keys 0-63) start while the
+            // softmax is still producing keys 64-127.
             if (!wmbar_wait(p_full1, pc1 & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+            tc_fence_after();
+            mma_pv<D, 0, 4>(tO1, tS1, va, acc1);
+            if (!wmbar_wait(p_full2_1, pc1 & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
             ++pc1;
             tc_fence_after();
-            mma_pv<D>(tO1, tS1, va, acc1);
+            mma_pv<D, 4, 8>(tO1, tS1, va, 1);
             acc1 = 1;
           }
           mma_commit_w(empty0 + 8 * vslot);
@@ -475,6 +489,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const uint32_t tO = tmem + (t ? C::kColO1 : C::kColO0) + lane_off;
     const uint32_t my_s_full = bar_s_full + 8 * t;
     const uint32_t my_p_full = bar_p_full + 8 * t;
+    const uint32_t my_p_full2 = bar_p_full2 + 8 * t;
     const uint32_t my_o_full = bar_o_full + 8 * t;
     const uint32_t my_o_free = bar_o_free + 8 * t;
     const float c2 = p.c2;
@@ -563,6 +578,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
           }
           tmem_st16(tS + ch * 16, pk);
+          if (ch == 1 && !(rescale && acc)) {
+            // keys 0-63 of P are in TMEM: let P V start on them
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(my_p_full);
+          }
         }
         {
           float a, b;
@@ -586,7 +608,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(my_p_full);
+        if (lane == 0) {
+          if (rescale && acc) mbar_arrive(my_p_full);   // O had to be rescaled first
+          mbar_arrive(my_p_full2);
+        }
         acc = true;
       }
       if (!ok) break;
