@@ -82,6 +82,8 @@ SMALL = [
     (1, 1, 1, 128, 1, W.CONTIGUOUS, True, 1.0),
     (1, 4, 4096, 128, 16, W.STRIPED, True, 3.0),
     (1, 2, 2048, 64, 2, W.STRIPED, False, 1.0),
+    (3, 1, 384, 128, 3, W.STRIPED, True, 1.0),        # c = 128: one tile per shard
+    (1, 1, 1000, 128, 5, W.STRIPED, True, 3.0),       # c = 200, P not a power of two
 ]
 
 
@@ -121,9 +123,10 @@ def sample_rows(w, n_random, seed):
 
 
 @pytest.mark.parametrize("w", [W.RING_8K, W.STRIPED_8K], ids=lambda w: w.name)
-def test_parity_8k_workloads(w):
+@pytest.mark.parametrize("sched_free", [False, True])
+def test_parity_8k_workloads(w, sched_free):
     q, k, v = W.make_qkv(w)
-    o, lse = run_path(q, k, v, w.P, w.layout, w.causal)
+    o, lse = run_path(q, k, v, w.P, w.layout, w.causal, sched_free)
     for h in (0, w.H - 1):        # whole heads, element by element
         o_ref, lse_ref = OA.attention(q[0, h].double().numpy(), k[0, h].double().numpy(),
                                       v[0, h].double().numpy(), w.scale, True)
@@ -176,6 +179,48 @@ def test_parity_long_workloads_sampled(w, sched_free):
         assert_close(o[0, h, rows], lse[0, h, rows], o_ref, lse_ref, f"{w.name} head {h}")
     assert np.array_equal(o[0, :, 0], v[0, :, 0].float().numpy())
     assert np.isfinite(o).all() and np.isfinite(lse).all()
+
+
+def test_parity_d64_batched_striped():
+    """d = 64 at scale, B > 1, striped causal: two heads element by element,
+    sampled rows elsewhere."""
+    w = W.Workload("d64", 2, 4, 8192, 64, 8, W.STRIPED, True, 21, qk_scale_up=3.0)
+    q, k, v = W.make_qkv(w)
+    o, lse = run_path(q, k, v, w.P, w.layout, True)
+    for b, h in ((0, 0), (1, 3)):
+        o_ref, lse_ref = OA.attention(q[b, h].double().numpy(), k[b, h].double().numpy(),
+                                      v[b, h].double().numpy(), w.scale, True)
+        assert_close(o[b, h], lse[b, h], o_ref, lse_ref, f"d64 b{b} h{h}")
+    for b, h in ((0, 2), (1, 1)):
+        rows = sample_rows(w, 16, b * 7 + h)
+        o_ref, lse_ref = OA.attention_rows(q[b, h].float().numpy(), k[b, h].float().numpy(),
+                                           v[b, h].float().numpy(), w.scale, True, rows)
+        assert_close(o[b, h, rows], lse[b, h, rows], o_ref, lse_ref, f"d64 b{b} h{h} rows")
+
+
+def test_parity_noncausal_long_sampled():
+    """Non-causal striped, N = 32768: every row attends to every key."""
+    w = W.Workload("noncausal32k", 1, 2, 32768, 128, 8, W.STRIPED, False, 22)
+    q, k, v = W.make_qkv(w)
+    o, lse = run_path(q, k, v, w.P, w.layout, False)
+    for h in range(2):
+        rows = sample_rows(w, 24, h)
+        o_ref, lse_ref = OA.attention_rows(q[0, h].float().numpy(), k[0, h].float().numpy(),
+                                           v[0, h].float().numpy(), w.scale, False, rows)
+        assert_close(o[0, h, rows], lse[0, h, rows], o_ref, lse_ref, f"noncausal h{h}")
+
+
+def test_parity_long_contiguous_sampled():
+    """The contiguous (ring) layout at the 128K size, as the benchmark's
+    layout comparison runs it."""
+    w = W.LONG_128K.with_(layout=W.CONTIGUOUS)
+    q, k, v = W.make_qkv(w)
+    o, lse = run_path(q, k, v, w.P, w.layout, True)
+    for h in (0, w.H - 1):
+        rows = sample_rows(w, 24, h)
+        o_ref, lse_ref = OA.attention_rows(q[0, h].float().numpy(), k[0, h].float().numpy(),
+                                           v[0, h].float().numpy(), w.scale, True, rows)
+        assert_close(o[0, h, rows], lse[0, h, rows], o_ref, lse_ref, f"contiguous 128K h{h}")
 
 
 # ------------------------------------------------------------ integer parity
