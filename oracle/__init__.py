@@ -21,6 +21,8 @@ source pages:
   Attention explainer ステップ2/ステップ3 and its 実装例).
 * ``work``         -- the per-device/per-round work formulas (Striped review,
   Ring Attention 工作负载 / Striped Attention 工作负载) and brute-force counts.
+* ``backward``     -- gradients dQ, dK, dV of the definition (the pages give
+  no backward; the textbook softmax derivative of 核心公式).
 * ``merge``        -- merging two partial (O, lse) results by splitting the
   softmax denominator into per-node partial sums (1cademy page "Computing
   Attention Weights in Sequence Parallelism").
@@ -32,4 +34,4 @@ Functions with no such pin say "parity unpinned" in their docstring; there are
 none at present.
 """
 
-from . import attention, merge, masks, partition, ring, work  # noqa: F401
+from . import attention, backward, merge, masks, partition, ring, work  # noqa: F401

@@ -140,3 +140,33 @@ def test_merge_mutant_fails_split_pin(monkeypatch):
     monkeypatch.setattr(merge, "lse_merge", wrong)
     with pytest.raises(AssertionError):
         TA.test_lse_merge_of_key_halves_equals_full(7)
+
+
+def _backward_mutant(kind):
+    def f(q, k, v, do, scale, causal, q_pos=None, k_pos=None):
+        q, k, v, do = (np.asarray(a, dtype=np.float64) for a in (q, k, v, do))
+        o, lse = att.attention(q, k, v, scale, causal)
+        n = q.shape[0]
+        s = (q @ k.T) * scale
+        if causal:
+            s = np.where(np.triu(np.ones((n, n), bool), 1), -np.inf, s)
+        p = np.exp(s - lse[:, None])
+        dv = p.T @ do
+        dp = do @ v.T
+        d_row = np.sum(do * o, axis=1)
+        ds = p * dp if kind == "no_D" else p * (dp - d_row[:, None])
+        dq = (ds @ k) * scale
+        dk = (ds @ q) * scale if kind == "dk_untransposed" else (ds.T @ q) * scale
+        if kind == "dv_no_transpose":
+            dv = p @ do
+        return dq, dk, dv, d_row
+    return f
+
+
+@pytest.mark.parametrize("kind", ["no_D", "dk_untransposed", "dv_no_transpose"])
+def test_backward_mutants_fail_autograd_pin(monkeypatch, kind):
+    import tests.test_oracle_backward as TB
+    from oracle import backward as OB
+    monkeypatch.setattr(OB, "attention_backward", _backward_mutant(kind))
+    with pytest.raises(AssertionError):
+        TB.test_backward_equals_torch_autograd(True, 9, 8)
