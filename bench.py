@@ -277,6 +277,8 @@ def main():
     ap.add_argument("--no-compare", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="also time the backward pass (dQ, dK, dV) on the same workload")
     ap.add_argument("--ref-budget", type=float, default=15.0,
                     help="seconds of CPU work per reference step")
     args = ap.parse_args()
@@ -376,6 +378,31 @@ def main():
         if ops.device_fault():
             raise RuntimeError("device fault during the layout comparison")
 
+    # ---- backward pass (optional): 10 d FLOP per visible pair (5 GEMMs)
+    backward = None
+    if args.backward:
+        lay = path.layout
+        qq, kk, vv = (path.qp, path.kp, path.vp) if lay == W.STRIPED else (path.q, path.k, path.v)
+        oo = path.op if lay == W.STRIPED else path.o
+        ll = path.lsep if lay == W.STRIPED else path.lse
+        path.step()
+        dout = torch.randn(qq.shape, device=qq.device,
+                           generator=torch.Generator(device=qq.device).manual_seed(1)).to(qq.dtype)
+        ws = torch.empty(qq.numel() // qq.shape[-1], dtype=torch.float32, device=qq.device)
+        grads = [torch.empty_like(qq) for _ in range(3)]
+
+        def bwd_step():
+            ops.attn_bwd(qq, kk, vv, oo, dout, ll, w.P, lay, w.causal, workspace=ws,
+                         dq=grads[0], dk=grads[1], dv=grads[2])
+
+        bwd_step()
+        torch.cuda.synchronize()
+        bms = timed(bwd_step, max(1, min(args.steps, 3)), world)
+        if ops.device_fault():
+            raise RuntimeError("device fault during the backward pass")
+        backward = {"ms": bms, "useful_tflops": 2.5 * flops / (bms * 1e-3) / 1e12,
+                    "flop_convention": "10 d per visible pair (QK^T, dO V^T, dV, dK, dQ)"}
+
     # ---- CPU oracle baseline (rank 0, one GPU only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -414,6 +441,7 @@ def main():
         "cpu_baseline": cpu,
         "e2e": e2e,
         "layout_compare": compare,
+        "backward": backward,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -24,8 +24,9 @@
  *
  * Conventions for every entry point:
  *   - All pointers marked "device" are CUDA device pointers on the current
- *     device; the caller allocates and owns every buffer.  The library never
- *     allocates device memory and keeps no pointer after a call returns.
+ *     device; the caller allocates and owns every buffer (including the
+ *     backward's workspace).  The library never allocates device memory and
+ *     keeps no pointer after a call returns.
  *   - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL =
  *     the legacy default stream).  A return of RA_OK means the work was
  *     validated and enqueued, not that it finished.
@@ -140,6 +141,32 @@ ra_status ra_partition(const void* src, void* dst, int64_t B, int64_t H, int64_t
 ra_status ra_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                       int64_t B, int64_t H, int64_t N, int64_t d, int P, int layout,
                       int causal, float scale, void* stream);
+
+/*
+ * ra_attn_bwd -- gradients of ra_attn_fwd: dQ, dK, dV.
+ *
+ * The pages give no backward algorithm (the Striped review measures training
+ * speedups, 五 核心结果); this is the derivative of the forward's definition
+ * (Striped review 核心公式) over the same shards, masks and skipped tiles:
+ *   P = exp(Q K^T * scale + C - lse),  D = rowsum(dO o O),
+ *   dS = P o (dO V^T - D),  dV = P^T dO,  dK = dS^T Q * scale,  dQ = dS K * scale.
+ *
+ *   q, k, v, o, dout  device, [B, H, N, d] bf16, layout order (o and lse as
+ *                     returned by ra_attn_fwd on the same q, k, v).
+ *   lse               device, [B, H, N] float32, layout order.
+ *   dq, dk, dv        device, [B, H, N, d] bf16 outputs, layout order; must
+ *                     not overlap each other or any input.
+ *   workspace         device, float32[B * H * N] scratch the call overwrites
+ *                     (holds D); owned by the caller, no overlap with others.
+ *   All pointers 16-byte aligned.  d, N, P, layout (no scheduling flag),
+ *   causal and scale as for ra_attn_fwd.
+ * Arithmetic: bf16 operands, fp32 accumulation on the tensor cores, P and dS
+ * rounded to bf16 for their products, outputs rounded to bf16 once.
+ */
+ra_status ra_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                      const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                      float* workspace, int64_t B, int64_t H, int64_t N, int64_t d, int P,
+                      int layout, int causal, float scale, void* stream);
 
 /*
  * ra_lse_merge -- merge two partial attention results over disjoint key sets.

@@ -16,7 +16,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libringattn.so")
-SOURCES = ["api.cu", "attn_fwd.cu", "aux_kernels.cu"]
+SOURCES = ["api.cu", "attn_fwd.cu", "attn_bwd.cu", "aux_kernels.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -565,7 +565,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             const int e = ch * 32 + 2 * i;
             const uint64_t x2 = ffma2(f2(s[e], s[e + 1]), c2x2, nm2);
             float p0, p1;
-            if (kPolyEvery && (i % kPolyEvery) == kPolyEvery - 1) {
+            if (kPolyEvery > 0 && (i % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
               exp2_poly2(x2, p0, p1);          // a share of the exps off the MUFU
             } else {
               float a0, a1;
@@ -746,6 +746,21 @@ __global__ void wait_selftest_kernel(unsigned long long limit_ns) {
 ra_status wait_selftest_launch(int64_t limit_ns, void* stream) {
   wait_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>((unsigned long long)limit_ns);
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
+// Device address of the fault word on the current device, for kernels of
+// other translation units (device symbols are not shared across files
+// without relocatable device code).
+unsigned int* device_fault_word() {
+  static unsigned int* cache[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!cache[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_device_fault) != cudaSuccess) return nullptr;
+    cache[dev] = reinterpret_cast<unsigned int*>(ptr);
+  }
+  return cache[dev];
 }
 
 ra_status read_device_fault(int* code) {

@@ -32,7 +32,29 @@ struct AttnLaunch {
 };
 
 ra_status attn_fwd_launch(const AttnLaunch& a);
+
+struct BwdLaunch {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* o;
+  const void* dout;
+  const float* lse;
+  void* dq;
+  void* dk;
+  void* dv;
+  float* workspace;
+  int64_t BH, N, d;
+  int P;
+  int striped, causal;
+  float scale;
+  int device, num_sms;
+  void* stream;
+};
+
+ra_status attn_bwd_launch(const BwdLaunch& a);
 ra_status read_device_fault(int* code);
+unsigned int* device_fault_word();
 ra_status wait_selftest_launch(int64_t limit_ns, void* stream);
 
 ra_status partition_launch(const void* src, void* dst, int64_t rows_outer, int64_t N, int64_t P,

@@ -51,6 +51,9 @@ def lib():
         L.ra_partition.argtypes = [vp, vp, i64, i64, i64, i64, i32, i32, i32, i32, vp]
         L.ra_attn_fwd.restype = i32
         L.ra_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, i32, i32, f32, vp]
+        L.ra_attn_bwd.restype = i32
+        L.ra_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i32,
+                                  i32, i32, f32, vp]
         L.ra_lse_merge.restype = i32
         L.ra_lse_merge.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, vp]
         L.ra_tile_census.restype = i32
@@ -140,6 +143,38 @@ def attn_fwd(q, k, v, P, layout, causal=True, scale=None, sched_free=False, out=
     _check(lib().ra_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, d, int(P),
                              lay, int(bool(causal)), float(scale), _stream(q)), "ra_attn_fwd")
     return out, lse
+
+
+def attn_bwd(q, k, v, o, dout, lse, P, layout, causal=True, scale=None, workspace=None,
+             dq=None, dk=None, dv=None):
+    """Gradients (dq, dk, dv) of attn_fwd; all tensors in LAYOUT order, as
+    returned by attn_fwd on the same q, k, v.  ``workspace``: float32 with
+    B*H*N elements (allocated here if not given)."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _cuda_contig(t, n)
+        if t.dtype != torch.bfloat16 or t.shape != q.shape:
+            raise ValueError(f"{n} must be bfloat16 of q's shape")
+    if q.dim() != 4:
+        raise ValueError("expected [B, H, N, d]")
+    B, H, N, d = q.shape
+    _cuda_contig(lse, "lse")
+    if lse.shape != (B, H, N) or lse.dtype != torch.float32:
+        raise ValueError("lse must be float32 [B, H, N]")
+    if scale is None:
+        scale = d ** -0.5
+    if workspace is None:
+        workspace = torch.empty(B * H * N, dtype=torch.float32, device=q.device)
+    if workspace.numel() < B * H * N or workspace.dtype != torch.float32:
+        raise ValueError("workspace must hold B*H*N float32")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    for n, t in (("dq", dq), ("dk", dk), ("dv", dv), ("workspace", workspace)):
+        _cuda_contig(t, n)
+    _check(lib().ra_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
+                             _ptr(dk), _ptr(dv), _ptr(workspace), B, H, N, d, int(P), int(layout),
+                             int(bool(causal)), float(scale), _stream(q)), "ra_attn_bwd")
+    return dq, dk, dv
 
 
 def lse_merge(o_a, lse_a, o_b, lse_b, out=None, lse_out=None):

@@ -29,7 +29,8 @@ def declared_symbols():
 def test_header_declares_the_boundary():
     syms = declared_symbols()
     for s in ("ra_partition", "ra_attn_fwd", "ra_lse_merge", "ra_status_string",
-              "ra_tile_census", "ra_device_fault", "ra_version", "ra_wait_selftest"):
+              "ra_tile_census", "ra_device_fault", "ra_version", "ra_wait_selftest",
+              "ra_attn_bwd"):
         assert s in syms
 
 
@@ -106,3 +107,18 @@ def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
     monkeypatch.setattr(ops, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         ops.lib()
+
+
+def bwd(L, q=A, k=Bp, v=Cp, o=Op, do=6 << 40, lse=Lp, dq=7 << 40, dk=8 << 40, dv=9 << 40,
+        ws=10 << 40, B=1, H=2, N=1024, d=128, P=4, layout=1, causal=1, scale=0.088):
+    return L.ra_attn_bwd(vp(q), vp(k), vp(v), vp(o), vp(do), vp(lse), vp(dq), vp(dk), vp(dv),
+                         vp(ws), B, H, N, d, P, layout, causal, scale, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ws=0), 1), (dict(do=0), 1), (dict(dq=(7 << 40) + 8), 2), (dict(ws=(10 << 40) + 4), 2),
+    (dict(N=1000, P=3), 3), (dict(d=32), 4), (dict(layout=0x101), 5), (dict(scale=0.0), 6),
+    (dict(dq=A), 8), (dict(dk=7 << 40), 8), (dict(ws=Lp), 8),
+])
+def test_attn_bwd_rejects_invalid_arguments(L, kw, code):
+    assert bwd(L, **kw) == code
