@@ -62,6 +62,8 @@ typedef int ra_status;
 #define RA_ERR_CUDA 9        /* a CUDA runtime/driver call failed              */
 #define RA_ERR_DEVICE 10     /* current device is not sm_100 (B200)            */
 #define RA_ERR_DEVICE_FAULT 11 /* a kernel gave up a bounded wait (see below)  */
+#define RA_ERR_SCRATCH 12    /* problem larger than the built-in scratch of    */
+                             /* ra_attn_bwd_noalloc (B*H*N > 1048576)          */
 
 /* Layouts (low byte of `layout`). */
 #define RA_CONTIGUOUS 0      /* shard j = tokens [j*c, (j+1)*c)  (Ring)        */
@@ -167,6 +169,31 @@ ra_status ra_attn_bwd(const void* q, const void* k, const void* v, const void* o
                       const void* dout, const float* lse, void* dq, void* dk, void* dv,
                       float* workspace, int64_t B, int64_t H, int64_t N, int64_t d, int P,
                       int layout, int causal, float scale, void* stream);
+
+/*
+ * ra_attn_bwd_noalloc -- ra_attn_bwd for callers that cannot allocate.
+ *
+ * No counterpart in the paper: this is a library convenience.  Some callers
+ * are handed their input and output buffers by a host framework that owns
+ * all device memory (a plug-in, an embedded runtime, a serving process with
+ * a fixed memory budget) and may not allocate more, or cannot afford a
+ * device allocation that might block or fail in the middle of a step.  For
+ * them this entry point takes no workspace: the backward's scratch row
+ * vector (D, one float per query row) lives in a fixed array inside the
+ * library, 2^20 floats (4 MiB) reserved on every GPU that loads the library
+ * until the process exits.  It calls no allocator.
+ *
+ *   Arguments as for ra_attn_bwd, minus `workspace`.
+ *   B * H * N must be <= 1048576, else RA_ERR_SCRATCH (nothing launched).
+ *   The first call on a device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   All calls share the one array: calls whose kernels overlap on the GPU
+ *   race on it and give wrong results; order them on one stream.
+ */
+ra_status ra_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                              const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                              int64_t B, int64_t H, int64_t N, int64_t d, int P, int layout,
+                              int causal, float scale, void* stream);
 
 /*
  * ra_lse_merge -- merge two partial attention results over disjoint key sets.

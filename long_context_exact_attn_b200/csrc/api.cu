@@ -82,6 +82,9 @@ const char* ra_status_string(ra_status s) {
     case RA_ERR_CUDA: return "a CUDA runtime/driver call failed";
     case RA_ERR_DEVICE: return "current device is not an sm_100 GPU";
     case RA_ERR_DEVICE_FAULT: return "a kernel gave up a bounded wait; outputs incomplete";
+    case RA_ERR_SCRATCH:
+      return "B*H*N exceeds the built-in scratch of ra_attn_bwd_noalloc (1048576 rows); "
+             "use ra_attn_bwd with a workspace";
     default: return "unknown status";
   }
 }
@@ -192,6 +195,47 @@ ra_status ra_attn_bwd(const void* q, const void* k, const void* v, const void* o
   a.num_sms = info.num_sms;
   a.stream = stream;
   return attn_bwd_launch(a);
+}
+
+ra_status ra_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                              const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                              int64_t B, int64_t H, int64_t N, int64_t d, int P, int layout,
+                              int causal, float scale, void* stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return RA_ERR_NULL;
+  if (layout != RA_CONTIGUOUS && layout != RA_STRIPED) return RA_ERR_LAYOUT;
+  if (d != 64 && d != 128) return RA_ERR_HEADDIM;
+  if (B < 1 || H < 1 || N < 1 || P < 1 || N % P != 0) return RA_ERR_SHAPE;
+  if (B * H * N >= ((int64_t)1 << 31) || N / P > ((int64_t)1 << 30) / 128) return RA_ERR_SHAPE;
+  if (B * H * N > kNoAllocScratchFloats) return RA_ERR_SCRATCH;
+  if (!(scale > 0.f) || !isfinite(scale)) return RA_ERR_SCALE;
+  const void* all[] = {q, k, v, o, dout, lse, dq, dk, dv};
+  for (const void* ptr : all)
+    if (!aligned(ptr, 16)) return RA_ERR_ALIGN;
+  const int64_t tb = B * H * N * d * 2, lb = B * H * N * 4;
+  const void* ins[] = {q, k, v, o, dout};
+  void* outs[] = {dq, dk, dv};
+  for (void* out : outs) {
+    for (const void* in : ins)
+      if (overlap(out, tb, in, tb)) return RA_ERR_ALIAS;
+    if (overlap(out, tb, lse, lb)) return RA_ERR_ALIAS;
+  }
+  if (overlap(dq, tb, dk, tb) || overlap(dq, tb, dv, tb) || overlap(dk, tb, dv, tb))
+    return RA_ERR_ALIAS;
+  int dev;
+  DevInfo info;
+  ra_status st = current_device(&dev, &info);
+  if (st) return st;
+  BwdLaunch a;
+  a.q = q; a.k = k; a.v = v; a.o = o; a.dout = dout; a.lse = lse;
+  a.dq = dq; a.dk = dk; a.dv = dv; a.workspace = nullptr;
+  a.BH = B * H; a.N = N; a.d = d; a.P = P;
+  a.striped = layout == RA_STRIPED;
+  a.causal = causal != 0;
+  a.scale = scale;
+  a.device = dev;
+  a.num_sms = info.num_sms;
+  a.stream = stream;
+  return attn_bwd_noalloc_launch(a);
 }
 
 ra_status ra_lse_merge(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,

@@ -23,6 +23,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "ra_internal.h"
 #include "ra_ptx.cuh"
 #include "ra_tiles.cuh"
@@ -612,6 +614,34 @@ ra_status attn_bwd_launch(const BwdLaunch& a) {
   if (a.d == 128) return launch_bwd<128>(a);
   if (a.d == 64) return launch_bwd<64>(a);
   return RA_ERR_HEADDIM;
+}
+
+// ------------------------------------------- backward without allocation
+// For callers that must not allocate device memory themselves: the scratch
+// row vector D of the backward lives in this fixed device array instead of a
+// caller workspace.  Every GPU that loads the library reserves it until the
+// process exits.  All calls share it: two calls whose kernels overlap on the
+// GPU (different streams, or devices sharing nothing but this library) race
+// on it.  D is fully rewritten by every call, so nothing has to be cleared.
+static __device__ __align__(256) float g_bwd_scratch[kNoAllocScratchFloats];
+
+ra_status attn_bwd_noalloc_launch(BwdLaunch a) {
+  if (a.BH * a.N > kNoAllocScratchFloats) return RA_ERR_SCRATCH;
+  // In host code `g_bwd_scratch` names a host-side stand-in; the kernels need
+  // the device address, looked up once per device with that device current.
+  static float* addr[64] = {nullptr};
+  static std::mutex mu;
+  if (a.device < 0 || a.device >= 64) return RA_ERR_DEVICE;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[a.device]) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_bwd_scratch) != cudaSuccess || !ptr) return RA_ERR_CUDA;
+      addr[a.device] = reinterpret_cast<float*>(ptr);
+    }
+  }
+  a.workspace = addr[a.device];
+  return attn_bwd_launch(a);
 }
 
 }  // namespace ra

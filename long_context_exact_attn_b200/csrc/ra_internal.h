@@ -53,6 +53,10 @@ struct BwdLaunch {
 };
 
 ra_status attn_bwd_launch(const BwdLaunch& a);
+
+// Capacity (floats) of the fixed scratch used by ra_attn_bwd_noalloc.
+constexpr long long kNoAllocScratchFloats = 1LL << 20;
+ra_status attn_bwd_noalloc_launch(BwdLaunch a);
 ra_status read_device_fault(int* code);
 unsigned int* device_fault_word();
 ra_status wait_selftest_launch(int64_t limit_ns, void* stream);

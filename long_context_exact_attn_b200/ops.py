@@ -54,6 +54,9 @@ def lib():
         L.ra_attn_bwd.restype = i32
         L.ra_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i32,
                                   i32, i32, f32, vp]
+        L.ra_attn_bwd_noalloc.restype = i32
+        L.ra_attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64,
+                                          i32, i32, i32, f32, vp]
         L.ra_lse_merge.restype = i32
         L.ra_lse_merge.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, vp]
         L.ra_tile_census.restype = i32
@@ -174,6 +177,29 @@ def attn_bwd(q, k, v, o, dout, lse, P, layout, causal=True, scale=None, workspac
     _check(lib().ra_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
                              _ptr(dk), _ptr(dv), _ptr(workspace), B, H, N, d, int(P), int(layout),
                              int(bool(causal)), float(scale), _stream(q)), "ra_attn_bwd")
+    return dq, dk, dv
+
+
+def attn_bwd_noalloc(q, k, v, o, dout, lse, P, layout, causal, scale, dq, dk, dv):
+    """attn_bwd through ra_attn_bwd_noalloc: for callers that own all device
+    memory and cannot let the library (or this binding) allocate.  The outputs
+    dq, dk, dv must be passed in; the scratch is the library's fixed array
+    (B*H*N <= 1048576).  Calls overlapping on the GPU race on that array."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout),
+                 ("dq", dq), ("dk", dk), ("dv", dv)):
+        _cuda_contig(t, n)
+        if t.dtype != torch.bfloat16 or t.shape != q.shape:
+            raise ValueError(f"{n} must be bfloat16 of q's shape")
+    if q.dim() != 4:
+        raise ValueError("expected [B, H, N, d]")
+    B, H, N, d = q.shape
+    _cuda_contig(lse, "lse")
+    if lse.shape != (B, H, N) or lse.dtype != torch.float32:
+        raise ValueError("lse must be float32 [B, H, N]")
+    _check(lib().ra_attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                                     _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, int(P),
+                                     int(layout), int(bool(causal)), float(scale), _stream(q)),
+           "ra_attn_bwd_noalloc")
     return dq, dk, dv
 
 

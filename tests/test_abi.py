@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(L):
 
 def test_status_strings(L):
     assert ops.status_string(0) == "ok"
-    for code in range(1, 12):
+    for code in range(1, 13):
         assert ops.status_string(code) not in ("", "unknown status")
     assert ops.status_string(999) == "unknown status"
     assert L.ra_version() >= 100
@@ -122,3 +122,19 @@ def bwd(L, q=A, k=Bp, v=Cp, o=Op, do=6 << 40, lse=Lp, dq=7 << 40, dk=8 << 40, dv
 ])
 def test_attn_bwd_rejects_invalid_arguments(L, kw, code):
     assert bwd(L, **kw) == code
+
+
+def bwd_noalloc(L, q=A, k=Bp, v=Cp, o=Op, do=6 << 40, lse=Lp, dq=7 << 40, dk=8 << 40, dv=9 << 40,
+                B=1, H=2, N=1024, d=128, P=4, layout=1, causal=1, scale=0.088):
+    return L.ra_attn_bwd_noalloc(vp(q), vp(k), vp(v), vp(o), vp(do), vp(lse), vp(dq), vp(dk),
+                                 vp(dv), B, H, N, d, P, layout, causal, scale, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dv=0), 1), (dict(dq=(7 << 40) + 8), 2), (dict(N=1000, P=3), 3), (dict(d=32), 4),
+    (dict(layout=0x101), 5), (dict(scale=0.0), 6), (dict(dq=A), 8), (dict(dk=7 << 40), 8),
+    # one row past the built-in scratch (1048576 floats), and far past it
+    (dict(B=1, H=1, N=(1 << 20) + 128, P=1), 12), (dict(B=4, H=16, N=131072, P=8), 12),
+])
+def test_attn_bwd_noalloc_rejects_invalid_arguments(L, kw, code):
+    assert bwd_noalloc(L, **kw) == code
