@@ -13,11 +13,13 @@
 //   bwd_dkdv     one CTA per key tile: loops over the query tiles that can
 //                see it, S^T = K Q^T and dP^T = V dO^T on the tensor cores,
 //                P^T and dS^T in TMEM (bf16), dV += P^T dO, dK += dS^T Q
-//   bwd_dq       one CTA per query tile: loops over key tiles in ring order,
+//   bwd_dq       one CTA per query tile: loops over the key tiles it sees,
 //                S = Q K^T, dP = dO V^T, dS in TMEM, dQ += dS K
-// Each CTA is one warpgroup (thread i owns TMEM lane i); one elected thread
-// issues TMA loads and MMAs; the next query (resp. key/value) tile is loaded
-// into a second shared-memory buffer while the current one is computed.
+// Both tile kernels are warp-specialised like the forward: a TMA producer
+// warp (two shared-memory stages of the streamed tile pair), an MMA warp,
+// and two element-wise warpgroups (thread = TMEM lane, each warpgroup one
+// half of the 128 columns).  The MMA order overlaps the next tile's score
+// MMA with the exponentials of the current one.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -81,35 +83,67 @@ __device__ __forceinline__ float bex2(float x) {
   return y;
 }
 
-// Wait by the whole CTA; gives up (and flags the CTA) after the time limit.
-__device__ __forceinline__ bool cta_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                         uint64_t limit) {
-  const bool ok = mbar_wait(bar, parity, abort, limit);
-  return __syncthreads_and(ok) != 0;
+template <int D>
+struct BwdCfg {
+  static constexpr int kTile = kBM * D * 2;   // bytes of a 128 x D bf16 tile
+  // smem: the fixed tile pair (F0, F1), two stages of the streamed tile pair,
+  // a ring of four per-column vector slots ({lse2, D} x 128 fp32), barriers
+  static constexpr int kFixed0 = 0, kFixed1 = kTile;
+  static constexpr int kStream = 2 * kTile;            // + stage * 2 * kTile
+  static constexpr int kVec = 6 * kTile;
+  static constexpr int kVecSlots = 4;
+  static constexpr int kBar = kVec + kVecSlots * 2 * kBM * 4;
+  static constexpr int kSmem = kBar + 128 + 1024;
+  static constexpr int kThreads = 320;   // 8 element-wise warps, producer, MMA
+};
+
+// Barrier offsets from BwdCfg::kBar (8 bytes each); tmem slot and abort flag
+// after them.  A stage has two full barriers: kBarFull for its first tile
+// (the operand of the score MMA), kBarFull2 for its second.
+enum : uint32_t {
+  kBarFixed = 0, kBarFull = 8, kBarEmpty = 24, kBarS = 40, kBarDP = 48, kBarP = 56,
+  kBarDS = 64, kBarAcc = 72, kBarDrain = 80, kBarFull2 = 88, kTmemSlot = 112, kAbort = 116
+};
+
+// TMA: one 128 x D tile of a [BH, P, c, D] tensor at (shard, row0, bh).
+template <int D>
+__device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* tm, uint32_t bar,
+                                          int row0, int shard, int bh) {
+#pragma unroll
+  for (int ch = 0; ch < D / 64; ++ch) tma_load_4d(dst + ch * 16384, tm, bar, ch * 64, row0, shard, bh);
 }
 
-// S (TMEM) = A (smem, 128 x D, K-major) x B (smem, 128 x D, K-major)^T
+// Whole-warp bounded wait (same result in every lane).
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+                                          uint64_t limit) {
+  const bool ok = mbar_wait(bar, parity, abort, limit);
+  return __all_sync(0xffffffffu, ok) != 0;
+}
+
+// S (TMEM, 128 x 128) = A (smem 128 x D, K-major) x B (smem 128 x D, K-major)^T
 template <int D>
 __device__ __forceinline__ void bwd_mma_ss(uint32_t d_tmem, uint32_t a, uint32_t b) {
   constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN, 0, 0);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
-    mma_ss(d_tmem, smem_desc_sw128(a + off, 16, 1024), smem_desc_sw128(b + off, 16, 1024), idesc,
-           kk > 0);
+    mma_ss_w(d_tmem, smem_desc_sw128(a + off, 16, 1024), smem_desc_sw128(b + off, 16, 1024), idesc,
+             kk > 0);
   }
 }
 
 // D (TMEM, 128 x D) (+)= A (TMEM, bf16 128 x 128) x B (smem tile [128 x D],
-// D contiguous, read as MN-major K x N).
+// D contiguous, read as MN-major K x N).  A is kept as two halves written by
+// the two element-wise warpgroups: K columns 0-63 packed at a_tmem + 0..31,
+// K columns 64-127 packed at a_tmem + 64..95.
 template <int D>
 __device__ __forceinline__ void bwd_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b,
                                            uint32_t acc) {
   constexpr uint32_t idesc = idesc_bf16_f32(kBM, D, 0, 1);
 #pragma unroll
   for (int kk = 0; kk < kBN / 16; ++kk)
-    mma_ts(d_tmem, a_tmem + kk * 8, smem_desc_sw128(b + kk * 2048, 16384, 1024), idesc,
-           (acc | (uint32_t)kk) != 0);
+    mma_ts_w(d_tmem, a_tmem + (kk / 4) * 64 + (kk % 4) * 8,
+             smem_desc_sw128(b + kk * 2048, 16384, 1024), idesc, (acc | (uint32_t)kk) != 0);
 }
 
 // Store 32 fp32 TMEM values (one row chunk) as bf16, times `mul`.
@@ -124,33 +158,101 @@ __device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (
   for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
 }
 
+// Common set-up of both kernels: barriers, TMEM (512 columns), descriptor
+// prefetch.  Returns the TMEM base.
 template <int D>
-struct BwdCfg {
-  static constexpr int kTile = kBM * D * 2;   // bytes of a 128 x D bf16 tile
-  static constexpr int kChunks = D / 64;
-  // smem: fixed tile pair (A0, A1), two buffers of the streamed tile pair,
-  // per-column vectors (2 buffers x {lse2, D} x 128 fp32), barriers
-  static constexpr int kFixed0 = 0, kFixed1 = kTile;
-  static constexpr int kStream = 2 * kTile;            // + buf * 2 * kTile
-  static constexpr int kVec = 6 * kTile;
-  static constexpr int kBar = kVec + 2 * 2 * kBM * 4;
-  static constexpr int kSmem = kBar + 64 + 1024;
-};
+__device__ __forceinline__ uint32_t bwd_setup(uint8_t* smem, int warp, int lane,
+                                              uint32_t full_count, const CUtensorMap* m0,
+                                              const CUtensorMap* m1, const CUtensorMap* m2,
+                                              const CUtensorMap* m3) {
+  using C = BwdCfg<D>;
+  const uint32_t bar = smem_u32(smem) + C::kBar;
+  if (threadIdx.x == 0) {
+    mbar_init(bar + kBarFixed, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar + kBarFull + 8 * s, full_count);
+      mbar_init(bar + kBarFull2 + 8 * s, 1);
+      mbar_init(bar + kBarEmpty + 8 * s, 1);
+    }
+    mbar_init(bar + kBarS, 1);
+    mbar_init(bar + kBarDP, 1);
+    mbar_init(bar + kBarP, 8);     // one arrival per element-wise warp
+    mbar_init(bar + kBarDS, 8);
+    mbar_init(bar + kBarAcc, 1);
+    mbar_init(bar + kBarDrain, 1);
+    *reinterpret_cast<volatile int*>(smem + C::kBar + kAbort) = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(smem + C::kBar + kTmemSlot), 512);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(m0);
+    tma_prefetch_desc(m1);
+    tma_prefetch_desc(m2);
+    tma_prefetch_desc(m3);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  return *reinterpret_cast<volatile uint32_t*>(smem + C::kBar + kTmemSlot);
+}
 
-// TMA: one 128 x D tile of a [BH, P, c, D] tensor at (shard, row0, bh).
+// Common tear-down: every role has finished; record an abort, free TMEM.
 template <int D>
-__device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* tm, uint32_t bar,
-                                          int row0, int shard, int bh) {
-#pragma unroll
-  for (int ch = 0; ch < D / 64; ++ch) tma_load_4d(dst + ch * 16384, tm, bar, ch * 64, row0, shard, bh);
+__device__ __forceinline__ void bwd_teardown(uint8_t* smem, uint32_t tmem, int warp,
+                                             const BwdParams& p, unsigned int code) {
+  using C = BwdCfg<D>;
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && *reinterpret_cast<volatile int*>(smem + C::kBar + kAbort) && p.fault)
+    atomicOr(p.fault, code);
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
 }
 
 // ------------------------------------------------------------- dK, dV
 // Work item: key tile kt of block kb of (b, h).  Query tiles visiting it:
 // every (query shard j, tile qt) whose tile against this key tile is not
-// skipped, shards in the order kb, kb+1, ... (the reverse ring).
+// skipped; shards in ascending order, so that the CTAs running at the same
+// time stream the same query tiles through L2 (the gradient is a sum, its
+// order is free).
+struct QCursor {
+  int j, qt, P, T, c, kb, striped, causal, y0;
+  __device__ void init(const BwdParams& p, int kb_, int y0_) {
+    j = 0; qt = 0; P = p.P; T = p.T; c = p.c; kb = kb_; striped = p.striped; causal = p.causal;
+    y0 = y0_;
+  }
+  __device__ bool next(int& oj, int& oqt) {
+    while (j < P) {
+      if (qt >= T) { qt = 0; ++j; continue; }
+      const BlockMask m = block_mask(j, kb, striped, causal);
+      if (m.all_hidden) { qt = T; continue; }
+      const int k = tile_kind(m, qt * kBM, y0, c);
+      ++qt;
+      if (k != TILE_SKIP) { oj = j; oqt = qt - 1; return true; }
+    }
+    return false;
+  }
+};
+
+// Item order: longest first.  Causal striped / non-causal: key tile kt is
+// seen by about T - kt query tiles of every shard, so kt ascending; causal
+// contiguous: block kb is seen by shards kb..P-1, so kb ascending.  Heads
+// vary slowest, so the CTAs of one wave share one head's tiles in L2.
+__device__ __forceinline__ void dkdv_item(const BwdParams& p, int idx, int& bh, int& kb, int& kt) {
+  const int per_head = p.P * p.T;
+  bh = idx / per_head;
+  const int r = idx % per_head;
+  if (p.causal && !p.striped) { kb = r / p.T; kt = r % p.T; }
+  else { kt = r / p.P; kb = r % p.P; }
+}
+
 template <int D>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(320, 1)
 bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                 const BwdParams p) {
@@ -158,211 +260,282 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  const uint32_t sb = smem_u32(smem);
-  const uint32_t bar_fixed = sb + C::kBar, bar_ld0 = bar_fixed + 8, bar_mma = bar_fixed + 24;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + C::kBar + 40);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBar + 44);
-  float* vec = reinterpret_cast<float*>(smem + C::kVec);   // [buf][lse2|D][128]
-  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-
-  const int T = p.T;
-  const int kt = blockIdx.x % T;
-  const int kb = (blockIdx.x / T) % p.P;
-  const int bh = blockIdx.x / (T * p.P);
+  const uint32_t sb = smem_u32(smem), bar = sb + C::kBar;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBar + kAbort);
+  float* vec = reinterpret_cast<float*>(smem + C::kVec);   // [stage][lse2 | D][128]
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  int bh, kb, kt;
+  dkdv_item(p, blockIdx.x, bh, kb, kt);
   const int y0 = kt * kBN;
-  const int y = y0 + tid;                       // this thread's key (local in block kb)
 
-  if (tid == 0) {
-    mbar_init(bar_fixed, 1);
-    mbar_init(bar_ld0, 1);
-    mbar_init(bar_ld0 + 8, 1);
-    mbar_init(bar_mma, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 0) {
-    tmem_alloc(smem_u32(tslot), 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tslot;
+  // producer lanes all arrive on a stage after writing its vectors
+  const uint32_t tmem = bwd_setup<D>(smem, warp, lane, 32, &tmQ, &tmK, &tmV, &tmdO);
   const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 256 + D;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
 
-  // The query tiles of this key tile, in order; one cursor for loads (one
-  // ahead) and one for compute.
-  struct Cursor {
-    int j, qt, P, T, c, kb, striped, causal, y0, done;
-    __device__ bool next(int& oj, int& oqt, int& kind) {
-      while (!done) {
-        if (qt >= T) {
-          qt = 0;
-          if (++j >= P) { done = 1; return false; }
-        }
-        const int jj = (kb + j) % P;
-        const BlockMask m = block_mask(jj, kb, striped, causal);
-        const int k = tile_kind(m, qt * kBM, y0, c);
-        ++qt;
-        if (k != TILE_SKIP) { oj = jj; oqt = qt - 1; kind = k; return true; }
-      }
-      return false;
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar + kBarFixed, 2 * C::kTile);
+      load_tile<D>(sb + C::kFixed0, &tmK, bar + kBarFixed, y0, kb, bh);
+      load_tile<D>(sb + C::kFixed1, &tmV, bar + kBarFixed, y0, kb, bh);
     }
-  };
-  Cursor ld{0, 0, p.P, T, p.c, kb, p.striped, p.causal, y0, 0};
-  Cursor cm = ld;
-
-  bool ok = true;
-  uint32_t issued[2] = {0, 0}, consumed[2] = {0, 0};
-  if (tid == 0) {
-    mbar_arrive_expect_tx(bar_fixed, 2 * C::kTile);
-    load_tile<D>(sb + C::kFixed0, &tmK, bar_fixed, y0, kb, bh);
-    load_tile<D>(sb + C::kFixed1, &tmV, bar_fixed, y0, kb, bh);
-  }
-  // Query tile loads run one ahead of the compute cursor, alternating buffers.
-  int lj, lqt, lkind;
-  auto issue_load = [&](int buf, int j, int qt) {
-    const uint32_t dst = sb + C::kStream + buf * 2 * C::kTile;
-    if (tid == 0) {
-      mbar_arrive_expect_tx(bar_ld0 + 8 * buf, 2 * C::kTile);
-      load_tile<D>(dst, &tmQ, bar_ld0 + 8 * buf, qt * kBM, j, bh);
-      load_tile<D>(dst + C::kTile, &tmdO, bar_ld0 + 8 * buf, qt * kBM, j, bh);
-    }
-    ++issued[buf];
-    // per-column lse (log2 units) and D of this query tile
-    const int x = qt * kBM + tid;
-    float* v = vec + buf * 2 * kBM;
-    const size_t row = (size_t)bh * p.N + (size_t)j * p.c + (size_t)(x < p.c ? x : 0);
-    v[tid] = (x < p.c) ? p.lse[row] * 1.4426950408889634f : INFINITY;
-    v[kBM + tid] = (x < p.c) ? p.dvec[row] : 0.f;
-  };
-  if (ld.next(lj, lqt, lkind)) issue_load(0, lj, lqt);
-  bool fixed_done = cta_wait(bar_fixed, 0, abort_flag, p.timeout_ns);
-  if (!fixed_done) ok = false;
-  tc_fence_after();
-
-  uint32_t n = 0, mma_ph = 0, accum = 0;
-  int cj, cqt, ckind;
-  while (ok && cm.next(cj, cqt, ckind)) {
-    const int buf = n & 1;
-    // Next query tile into the other buffer; the MMAs that read it last
-    // completed at the end of the previous iteration.
-    __syncthreads();
-    if (ld.next(lj, lqt, lkind)) issue_load(buf ^ 1, lj, lqt);
-    if (!cta_wait(bar_ld0 + 8 * buf, consumed[buf] & 1, abort_flag, p.timeout_ns)) {
-      ok = false;
-      break;
-    }
-    ++consumed[buf];
-    tc_fence_after();
-    const uint32_t sq = sb + C::kStream + buf * 2 * C::kTile, sdo = sq + C::kTile;
-    if (warp == 0 && lane == 0) {
-      bwd_mma_ss<D>(tS, sb + C::kFixed0, sq);     // S^T = K Q^T
-      bwd_mma_ss<D>(tdP, sb + C::kFixed1, sdo);   // dP^T = V dO^T
-      mma_commit(bar_mma);
-    }
-    __syncwarp();
-    if (!cta_wait(bar_mma, mma_ph, abort_flag, p.timeout_ns)) { ok = false; break; }
-    mma_ph ^= 1;
-    tc_fence_after();
-    // P^T and dS^T for this thread's key row; column q = query qt*128 + q
-    const float* lse2 = vec + buf * 2 * kBM;
-    const float* dcol = lse2 + kBM;
-    const BlockMask bm = block_mask(cj, kb, p.striped, p.causal);
-    int lo = 0, hi = p.c - cqt * kBM;             // visible query columns [lo, hi)
-    if (bm.use_diag) {
-      const int l2 = y + 1 - bm.e - cqt * kBM;    // query x sees key y iff y < x + e
-      lo = l2 > 0 ? l2 : 0;
-    }
-    if (y >= p.c) hi = 0;
-#pragma unroll 1
-    for (int ch = 0; ch < 4; ++ch) {
-      uint32_t sv[32], dv[32];
-      tmem_ld32(tS + lane_off + ch * 32, sv);
-      tmem_ld32(tdP + lane_off + ch * 32, dv);
-      tmem_wait_ld();
-      uint32_t pk[16], dk[16];
+    QCursor cur;
+    cur.init(p, kb, y0);
+    uint32_t n = 0;
+    int j, qt;
+    while (cur.next(j, qt)) {
+      const int s = n & 1;
+      // Per-column lse (log2 units) and D of this query tile, into vector
+      // slot n mod 4 before the stage is free, so that their load latency
+      // is off the critical path.  Slot n mod 4 was last read for tile n-4,
+      // which finished before the stage wait of tile n-2 passed.
+      float* v = vec + (n % C::kVecSlots) * 2 * kBM;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float pr[2], ds[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int q = ch * 32 + 2 * i + u;
-          const bool vis = (q >= lo) && (q < hi);
-          const float pv = vis ? bex2(fmaf(__uint_as_float(sv[2 * i + u]), p.c2, -lse2[q])) : 0.f;
-          pr[u] = pv;
-          ds[u] = pv * (__uint_as_float(dv[2 * i + u]) - dcol[q]);
-        }
-        pk[i] = pack2(pr[0], pr[1]);
-        dk[i] = pack2(ds[0], ds[1]);
+      for (int u = 0; u < 4; ++u) {
+        const int q = lane + 32 * u, x = qt * kBM + q;
+        const bool valid = x < p.c;
+        const size_t row = (size_t)bh * p.N + (size_t)j * p.c + (size_t)(valid ? x : 0);
+        v[q] = valid ? p.lse[row] * 1.4426950408889634f : INFINITY;
+        v[kBM + q] = valid ? p.dvec[row] : 0.f;
       }
-      tmem_st16(tS + lane_off + ch * 16, pk);
-      tmem_st16(tdP + lane_off + ch * 16, dk);
-    }
-    tmem_wait_st();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (warp == 0 && lane == 0) {
-      bwd_mma_ts<D>(tdV, tS, sdo, accum);   // dV += P^T dO
-      bwd_mma_ts<D>(tdK, tdP, sq, accum);   // dK += dS^T Q
-      mma_commit(bar_mma);
-    }
-    __syncwarp();
-    accum = 1;
-    if (!cta_wait(bar_mma, mma_ph, abort_flag, p.timeout_ns)) { ok = false; break; }
-    mma_ph ^= 1;
-    tc_fence_after();
-    ++n;
-  }
-  // Epilogue: dK (times scale) and dV rows of this key tile.  TMEM loads are
-  // warp-collective; only the stores are guarded per row.
-  if (ok) {
-    const bool valid = y < p.c;
-    const size_t row = (size_t)bh * p.N + (size_t)kb * p.c + (size_t)(valid ? y : 0);
-#pragma unroll 1
-    for (int q = 0; q < D / 32; ++q) {
-      uint32_t r[32];
-      if (accum) {
-        tmem_ld32(tdK + lane_off + q * 32, r);
-        tmem_wait_ld();
+      if (n >= 2 && !warp_wait(bar + kBarEmpty + 8 * s, ((n >> 1) - 1) & 1, abort_flag, p.timeout_ns))
+        break;
+      const uint32_t dst = sb + C::kStream + s * 2 * C::kTile;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar + kBarFull + 8 * s, C::kTile);
+        load_tile<D>(dst, &tmQ, bar + kBarFull + 8 * s, qt * kBM, j, bh);
+        mbar_arrive_expect_tx(bar + kBarFull2 + 8 * s, C::kTile);
+        load_tile<D>(dst + C::kTile, &tmdO, bar + kBarFull2 + 8 * s, qt * kBM, j, bh);
       } else {
+        mbar_arrive(bar + kBarFull + 8 * s);
+      }
+      ++n;
+    }
+    // every issued load must have landed before the CTA exits
+    if (lane == 0) {
+      volatile int no_abort = 0;
+      mbar_wait(bar + kBarFixed, 0, &no_abort, p.timeout_ns);
+      for (uint32_t m = n > 2 ? n - 2 : 0; m < n; ++m) {
+        mbar_wait(bar + kBarFull + 8 * (m & 1), (m >> 1) & 1, &no_abort, p.timeout_ns);
+        mbar_wait(bar + kBarFull2 + 8 * (m & 1), (m >> 1) & 1, &no_abort, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ---------------------------------------------------------- MMA issuer
+    // Order per query tile i (stage s):  dV += P_i^T dO_i, S_{i+1} = K Q_{i+1}^T,
+    // dK += dS_i^T Q_i, dP_{i+1} = V dO_{i+1}^T.  S_{i+1} reuses the columns
+    // of P_i right after the MMA that reads them (tcgen05 MMAs of one CTA
+    // run in issue order), so the tensor core computes the next scores while
+    // the element-wise warps finish dS_i and start on P_{i+1}.
+    QCursor cur;
+    cur.init(p, kb, y0);
+    int j, qt;
+    bool ok = warp_wait(bar + kBarFixed, 0, abort_flag, p.timeout_ns);
+    bool have = cur.next(j, qt);
+    uint32_t i = 0;
+    if (ok && have) {
+      ok = warp_wait(bar + kBarFull, 0, abort_flag, p.timeout_ns);
+      if (ok) {
+        tc_fence_after();
+        bwd_mma_ss<D>(tS, sb + C::kFixed0, sb + C::kStream);
+        mma_commit_w(bar + kBarS);
+        ok = warp_wait(bar + kBarFull2, 0, abort_flag, p.timeout_ns);
+      }
+      if (ok) {
+        tc_fence_after();
+        bwd_mma_ss<D>(tdP, sb + C::kFixed1, sb + C::kStream + C::kTile);
+        mma_commit_w(bar + kBarDP);
+      }
+    }
+    while (ok && have) {
+      const int s = i & 1;
+      const uint32_t sq = sb + C::kStream + s * 2 * C::kTile, sdo = sq + C::kTile;
+      const uint32_t nq = sb + C::kStream + (s ^ 1) * 2 * C::kTile, ndo = nq + C::kTile;
+      const bool more = cur.next(j, qt);
+      if (!warp_wait(bar + kBarP, i & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+      tc_fence_after();
+      bwd_mma_ts<D>(tdV, tS, sdo, i > 0);
+      if (more) {
+        if (!warp_wait(bar + kBarFull + 8 * (s ^ 1), ((i + 1) >> 1) & 1, abort_flag, p.timeout_ns)) {
+          ok = false; break;
+        }
+        tc_fence_after();
+        bwd_mma_ss<D>(tS, sb + C::kFixed0, nq);
+        mma_commit_w(bar + kBarS);
+      }
+      if (!warp_wait(bar + kBarDS, i & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+      tc_fence_after();
+      bwd_mma_ts<D>(tdK, tdP, sq, i > 0);
+      mma_commit_w(bar + kBarEmpty + 8 * s);
+      if (more) {
+        if (!warp_wait(bar + kBarFull2 + 8 * (s ^ 1), ((i + 1) >> 1) & 1, abort_flag, p.timeout_ns)) {
+          ok = false; break;
+        }
+        tc_fence_after();
+        bwd_mma_ss<D>(tdP, sb + C::kFixed1, ndo);
+        mma_commit_w(bar + kBarDP);
+      }
+      ++i;
+      have = more;
+    }
+    if (ok) mma_commit_w(bar + kBarAcc);
+    // all MMAs must be complete before TMEM is freed
+    mma_commit_w(bar + kBarDrain);
+    volatile int no_abort = 0;
+    warp_wait(bar + kBarDrain, 0, &no_abort, p.timeout_ns);
+  } else {
+    // ------------------------------------------------- element-wise warps
+    // Thread = key row y (TMEM lane); warpgroup wg takes query columns
+    // [64 wg, 64 wg + 64) of every tile.
+    const int wg = warp / 4, wq = warp % 4;
+    const int y = y0 + wq * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t myS = tS + lane_off + 64 * wg, mydP = tdP + lane_off + 64 * wg;
+    QCursor cur;
+    cur.init(p, kb, y0);
+    int j, qt;
+    uint32_t i = 0;
+    bool ok = true;
+    while (cur.next(j, qt)) {
+      const int s = i & 1;
+      const BlockMask bm = block_mask(j, kb, p.striped, p.causal);
+      int lo = 0, hi = p.c - qt * kBM;          // visible query columns [lo, hi)
+      if (bm.use_diag) {
+        const int l2 = y + 1 - bm.e - qt * kBM;  // query x sees key y iff y < x + e
+        lo = l2 > 0 ? l2 : 0;
+      }
+      if (y >= p.c) hi = 0;
+      lo -= 64 * wg;
+      hi -= 64 * wg;
+      if (!warp_wait(bar + kBarS, i & 1, abort_flag, p.timeout_ns) ||
+          !warp_wait(bar + kBarFull + 8 * s, (i >> 1) & 1, abort_flag, p.timeout_ns)) {
+        ok = false; break;
+      }
+      tc_fence_after();
+      uint32_t a[2][32];
+      tmem_ld32(myS, a[0]);
+      tmem_ld32(myS + 32, a[1]);
+      tmem_wait_ld();
+      const float4* lse2 = reinterpret_cast<const float4*>(vec + (i % C::kVecSlots) * 2 * kBM + 64 * wg);
+      const float4* dcol = lse2 + kBM / 4;
+      float pr[64];
+      uint32_t pk[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) r[i] = 0u;
+      for (int q4 = 0; q4 < 16; ++q4) {
+        const float4 l4 = lse2[q4];
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int q = 4 * q4 + u;
+          const float sv = __uint_as_float(a[q / 32][q % 32]);
+          pr[q] = (q >= lo && q < hi) ? bex2(fmaf(sv, p.c2, -lv[u])) : 0.f;
+        }
       }
-      if (valid) store_row32(p.dk + row * D + q * 32, r, p.scale);
-      if (accum) {
-        tmem_ld32(tdV + lane_off + q * 32, r);
-        tmem_wait_ld();
+#pragma unroll
+      for (int q = 0; q < 32; ++q) pk[q] = pack2(pr[2 * q], pr[2 * q + 1]);
+      tmem_st32(myS, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar + kBarP);
+      if (!warp_wait(bar + kBarDP, i & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+      tc_fence_after();
+      tmem_ld32(mydP, a[0]);
+      tmem_ld32(mydP + 32, a[1]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int q4 = 0; q4 < 16; ++q4) {
+        const float4 d4 = dcol[q4];
+        const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+        float ds[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int q = 4 * q4 + u;
+          ds[u] = pr[q] * (__uint_as_float(a[q / 32][q % 32]) - dv[u]);
+        }
+        pk[2 * q4] = pack2(ds[0], ds[1]);
+        pk[2 * q4 + 1] = pack2(ds[2], ds[3]);
       }
-      if (valid) store_row32(p.dv + row * D + q * 32, r, 1.f);
+      tmem_st32(mydP, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar + kBarDS);
+      ++i;
+    }
+    // Epilogue: dK (times scale) and dV rows of this key tile, columns
+    // [wg D/2, (wg+1) D/2).  TMEM loads are warp-collective; only the stores
+    // are guarded per row.
+    if (ok && (i == 0 || warp_wait(bar + kBarAcc, 0, abort_flag, p.timeout_ns))) {
+      tc_fence_after();
+      const bool valid = y < p.c;
+      const size_t row = (size_t)bh * p.N + (size_t)kb * p.c + (size_t)(valid ? y : 0);
+#pragma unroll 1
+      for (int q = 0; q < D / 64; ++q) {
+        const int col = wg * (D / 2) + q * 32;
+        uint32_t r[32];
+        if (i) {
+          tmem_ld32(tdK + lane_off + col, r);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) r[u] = 0u;
+        }
+        if (valid) store_row32(p.dk + row * D + col, r, p.scale);
+        if (i) {
+          tmem_ld32(tdV + lane_off + col, r);
+          tmem_wait_ld();
+        }
+        if (valid) store_row32(p.dv + row * D + col, r, 1.f);
+      }
     }
   }
-  // Drain: every issued load and MMA must have completed before exit.
-  if (tid == 0) {
-    volatile int no_abort = 0;
-    mma_commit(bar_mma);
-    mbar_wait(bar_mma, mma_ph, &no_abort, p.timeout_ns);
-    if (!fixed_done) mbar_wait(bar_fixed, 0, &no_abort, p.timeout_ns);
-    for (int b2 = 0; b2 < 2; ++b2)
-      if (issued[b2] > consumed[b2])
-        mbar_wait(bar_ld0 + 8 * b2, (issued[b2] - 1) & 1, &no_abort, p.timeout_ns);
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (tid == 0 && *abort_flag && p.fault) atomicOr(p.fault, 4u);
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
-  }
+  bwd_teardown<D>(smem, tmem, warp, p, 4u);
 }
 
 // ----------------------------------------------------------------- dQ
-// Work item: query tile qt of shard j of (b, h); key tiles in ring order
-// (block (j - r) mod P in round r), skipped tiles left out.
+// Work item: query tile qt of shard j of (b, h); key tiles of every block
+// that is not hidden, blocks in ascending order (the same order in every
+// CTA, for L2 reuse; the gradient is a sum), skipped tiles left out.
+struct KCursor {
+  int kb, kt, kend, P, c, j, striped, causal, x0;
+  BlockMask bm;
+  TileSpan sp;
+  __device__ void init(const BwdParams& p, int j_, int x0_) {
+    kb = -1; kt = 0; kend = 0; P = p.P; c = p.c; j = j_; striped = p.striped; causal = p.causal;
+    x0 = x0_;
+  }
+  __device__ bool next(int& okb, int& oy0, int& kind, BlockMask& m) {
+    while (kt >= kend) {
+      if (++kb >= P) return false;
+      bm = block_mask(j, kb, striped, causal);
+      sp = tile_span(bm, x0, c);
+      kend = sp.part_end;
+      kt = 0;
+    }
+    okb = kb;
+    oy0 = kt * kBN;
+    kind = tile_kind_at(sp, kt);
+    m = bm;
+    ++kt;
+    return true;
+  }
+};
+
+// Longest first: causal striped, the last query tiles of a shard see the
+// most keys (qt descending); causal contiguous, shard j sees blocks 0..j
+// (j descending, then qt descending).  Heads vary slowest.
+__device__ __forceinline__ void dq_item(const BwdParams& p, int idx, int& bh, int& j, int& qt) {
+  const int per_head = p.P * p.T;
+  bh = idx / per_head;
+  const int r = idx % per_head;
+  if (p.causal && !p.striped) { j = p.P - 1 - r / p.T; qt = p.T - 1 - r % p.T; }
+  else { qt = p.T - 1 - r / p.P; j = r % p.P; }
+}
+
 template <int D>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(320, 1)
 bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
               const BwdParams p) {
@@ -370,182 +543,178 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  const uint32_t sb = smem_u32(smem);
-  const uint32_t bar_fixed = sb + C::kBar, bar_ld0 = bar_fixed + 8, bar_mma = bar_fixed + 24;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + C::kBar + 40);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBar + 44);
-  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-
-  const int T = p.T;
-  const int qt = blockIdx.x % T;
-  const int j = (blockIdx.x / T) % p.P;
-  const int bh = blockIdx.x / (T * p.P);
+  const uint32_t sb = smem_u32(smem), bar = sb + C::kBar;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBar + kAbort);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  int bh, j, qt;
+  dq_item(p, blockIdx.x, bh, j, qt);
   const int x0 = qt * kBM;
-  const int x = x0 + tid;                       // this thread's query (local in shard j)
-  const bool xvalid = x < p.c;
-  const size_t xrow = (size_t)bh * p.N + (size_t)j * p.c + (size_t)(xvalid ? x : 0);
-  const float lse2 = xvalid ? p.lse[xrow] * 1.4426950408889634f : INFINITY;
-  const float drow = xvalid ? p.dvec[xrow] : 0.f;
 
-  if (tid == 0) {
-    mbar_init(bar_fixed, 1);
-    mbar_init(bar_ld0, 1);
-    mbar_init(bar_ld0 + 8, 1);
-    mbar_init(bar_mma, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 0) {
-    tmem_alloc(smem_u32(tslot), 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tslot;
+  const uint32_t tmem = bwd_setup<D>(smem, warp, lane, 1, &tmQ, &tmK, &tmV, &tmdO);
   const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
 
-  struct Cursor {
-    int r, kt, kend, P, c, j, striped, causal, x0;
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar + kBarFixed, 2 * C::kTile);
+      load_tile<D>(sb + C::kFixed0, &tmQ, bar + kBarFixed, x0, j, bh);
+      load_tile<D>(sb + C::kFixed1, &tmdO, bar + kBarFixed, x0, j, bh);
+      KCursor cur;
+      cur.init(p, j, x0);
+      uint32_t n = 0;
+      int kb, y0, kind;
+      BlockMask bm;
+      while (cur.next(kb, y0, kind, bm)) {
+        const int s = n & 1;
+        if (n >= 2 && !mbar_wait(bar + kBarEmpty + 8 * s, ((n >> 1) - 1) & 1, abort_flag, p.timeout_ns))
+          break;
+        const uint32_t dst = sb + C::kStream + s * 2 * C::kTile;
+        mbar_arrive_expect_tx(bar + kBarFull + 8 * s, C::kTile);
+        load_tile<D>(dst, &tmK, bar + kBarFull + 8 * s, y0, kb, bh);
+        mbar_arrive_expect_tx(bar + kBarFull2 + 8 * s, C::kTile);
+        load_tile<D>(dst + C::kTile, &tmV, bar + kBarFull2 + 8 * s, y0, kb, bh);
+        ++n;
+      }
+      volatile int no_abort = 0;
+      mbar_wait(bar + kBarFixed, 0, &no_abort, p.timeout_ns);
+      for (uint32_t m = n > 2 ? n - 2 : 0; m < n; ++m) {
+        mbar_wait(bar + kBarFull + 8 * (m & 1), (m >> 1) & 1, &no_abort, p.timeout_ns);
+        mbar_wait(bar + kBarFull2 + 8 * (m & 1), (m >> 1) & 1, &no_abort, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ---------------------------------------------------------- MMA issuer
+    // Order per key tile i (stage s): S_{i+1} = Q K_{i+1}^T as soon as the
+    // element-wise warps have read S_i; dQ += dS_i K_i; dP_{i+1} = dO V_{i+1}^T
+    // into the columns of dS_i right after the MMA that reads them.
+    KCursor cur;
+    cur.init(p, j, x0);
+    int kb, y0, kind;
     BlockMask bm;
-    TileSpan sp;
-    int kb;
-    __device__ bool next(int& okb, int& oy0, int& kind, BlockMask& m) {
-      while (kt >= kend) {
-        if (++r >= P) return false;
-        kb = key_block(j, r, P);
-        bm = block_mask(j, kb, striped, causal);
-        sp = tile_span(bm, x0, c);
-        kend = sp.part_end;
-        kt = 0;
+    bool ok = warp_wait(bar + kBarFixed, 0, abort_flag, p.timeout_ns);
+    bool have = cur.next(kb, y0, kind, bm);
+    uint32_t i = 0;
+    if (ok && have) {
+      ok = warp_wait(bar + kBarFull, 0, abort_flag, p.timeout_ns);
+      if (ok) {
+        tc_fence_after();
+        bwd_mma_ss<D>(tS, sb + C::kFixed0, sb + C::kStream);
+        mma_commit_w(bar + kBarS);
+        ok = warp_wait(bar + kBarFull2, 0, abort_flag, p.timeout_ns);
       }
-      okb = kb;
-      oy0 = kt * kBN;
-      kind = tile_kind_at(sp, kt);
-      m = bm;
-      ++kt;
-      return true;
+      if (ok) {
+        tc_fence_after();
+        bwd_mma_ss<D>(tdP, sb + C::kFixed1, sb + C::kStream + C::kTile);
+        mma_commit_w(bar + kBarDP);
+      }
     }
-  };
-  Cursor ld;
-  ld.r = -1; ld.kt = 0; ld.kend = 0; ld.P = p.P; ld.c = p.c; ld.j = j; ld.striped = p.striped;
-  ld.causal = p.causal; ld.x0 = x0; ld.kb = 0;
-  Cursor cm = ld;
-
-  bool ok = true;
-  uint32_t issued[2] = {0, 0}, consumed[2] = {0, 0};
-  if (tid == 0) {
-    mbar_arrive_expect_tx(bar_fixed, 2 * C::kTile);
-    load_tile<D>(sb + C::kFixed0, &tmQ, bar_fixed, x0, j, bh);
-    load_tile<D>(sb + C::kFixed1, &tmdO, bar_fixed, x0, j, bh);
-  }
-  int lkb, ly0, lkind;
-  BlockMask lbm;
-  auto issue_load = [&](int buf, int kb, int y0) {
-    if (tid == 0) {
-      const uint32_t dst = sb + C::kStream + buf * 2 * C::kTile;
-      mbar_arrive_expect_tx(bar_ld0 + 8 * buf, 2 * C::kTile);
-      load_tile<D>(dst, &tmK, bar_ld0 + 8 * buf, y0, kb, bh);
-      load_tile<D>(dst + C::kTile, &tmV, bar_ld0 + 8 * buf, y0, kb, bh);
-    }
-    ++issued[buf];
-  };
-  if (ld.next(lkb, ly0, lkind, lbm)) issue_load(0, lkb, ly0);
-  bool fixed_done = cta_wait(bar_fixed, 0, abort_flag, p.timeout_ns);
-  if (!fixed_done) ok = false;
-  tc_fence_after();
-
-  uint32_t n = 0, mma_ph = 0, accum = 0;
-  int ckb, cy0, ckind;
-  BlockMask cbm;
-  while (ok && cm.next(ckb, cy0, ckind, cbm)) {
-    const int buf = n & 1;
-    __syncthreads();
-    if (ld.next(lkb, ly0, lkind, lbm)) issue_load(buf ^ 1, lkb, ly0);
-    if (!cta_wait(bar_ld0 + 8 * buf, consumed[buf] & 1, abort_flag, p.timeout_ns)) {
-      ok = false;
-      break;
-    }
-    ++consumed[buf];
-    tc_fence_after();
-    const uint32_t sk = sb + C::kStream + buf * 2 * C::kTile, sv = sk + C::kTile;
-    if (warp == 0 && lane == 0) {
-      bwd_mma_ss<D>(tS, sb + C::kFixed0, sk);     // S = Q K^T
-      bwd_mma_ss<D>(tdP, sb + C::kFixed1, sv);    // dP = dO V^T
-      mma_commit(bar_mma);
-    }
-    __syncwarp();
-    if (!cta_wait(bar_mma, mma_ph, abort_flag, p.timeout_ns)) { ok = false; break; }
-    mma_ph ^= 1;
-    tc_fence_after();
-    const int lim = xvalid ? ((ckind == TILE_PARTIAL) ? row_limit(cbm, x, cy0, p.c) : kBN) : 0;
-#pragma unroll 1
-    for (int ch = 0; ch < 4; ++ch) {
-      uint32_t s32[32], d32[32];
-      tmem_ld32(tS + lane_off + ch * 32, s32);
-      tmem_ld32(tdP + lane_off + ch * 32, d32);
-      tmem_wait_ld();
-      uint32_t dk[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float ds[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int col = ch * 32 + 2 * i + u;
-          const float pv = (col < lim) ? bex2(fmaf(__uint_as_float(s32[2 * i + u]), p.c2, -lse2)) : 0.f;
-          ds[u] = pv * (__uint_as_float(d32[2 * i + u]) - drow);
+    while (ok && have) {
+      const int s = i & 1;
+      const uint32_t sk = sb + C::kStream + s * 2 * C::kTile;
+      const uint32_t nk = sb + C::kStream + (s ^ 1) * 2 * C::kTile, nv = nk + C::kTile;
+      const bool more = cur.next(kb, y0, kind, bm);
+      if (more) {
+        // kBarP: the element-wise warps have read S_i
+        if (!warp_wait(bar + kBarP, i & 1, abort_flag, p.timeout_ns) ||
+            !warp_wait(bar + kBarFull + 8 * (s ^ 1), ((i + 1) >> 1) & 1, abort_flag, p.timeout_ns)) {
+          ok = false; break;
         }
-        dk[i] = pack2(ds[0], ds[1]);
+        tc_fence_after();
+        bwd_mma_ss<D>(tS, sb + C::kFixed0, nk);
+        mma_commit_w(bar + kBarS);
       }
-      tmem_st16(tS + lane_off + ch * 16, dk);
-    }
-    tmem_wait_st();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (warp == 0 && lane == 0) {
-      bwd_mma_ts<D>(tdQ, tS, sk, accum);    // dQ += dS K
-      mma_commit(bar_mma);
-    }
-    __syncwarp();
-    accum = 1;
-    if (!cta_wait(bar_mma, mma_ph, abort_flag, p.timeout_ns)) { ok = false; break; }
-    mma_ph ^= 1;
-    tc_fence_after();
-    ++n;
-  }
-  if (ok) {
-    __nv_bfloat16* dst = p.dq + xrow * D;
-#pragma unroll 1
-    for (int q = 0; q < D / 32; ++q) {
-      uint32_t r[32];
-      if (accum) {
-        tmem_ld32(tdQ + lane_off + q * 32, r);
-        tmem_wait_ld();
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) r[i] = 0u;
+      if (!warp_wait(bar + kBarDS, i & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+      tc_fence_after();
+      bwd_mma_ts<D>(tdQ, tdP, sk, i > 0);
+      mma_commit_w(bar + kBarEmpty + 8 * s);
+      if (more) {
+        if (!warp_wait(bar + kBarFull2 + 8 * (s ^ 1), ((i + 1) >> 1) & 1, abort_flag, p.timeout_ns)) {
+          ok = false; break;
+        }
+        tc_fence_after();
+        bwd_mma_ss<D>(tdP, sb + C::kFixed1, nv);
+        mma_commit_w(bar + kBarDP);
       }
-      if (xvalid) store_row32(dst + q * 32, r, p.scale);
+      ++i;
+      have = more;
     }
-  }
-  if (tid == 0) {
+    if (ok) mma_commit_w(bar + kBarAcc);
+    mma_commit_w(bar + kBarDrain);
     volatile int no_abort = 0;
-    mma_commit(bar_mma);
-    mbar_wait(bar_mma, mma_ph, &no_abort, p.timeout_ns);
-    if (!fixed_done) mbar_wait(bar_fixed, 0, &no_abort, p.timeout_ns);
-    for (int b2 = 0; b2 < 2; ++b2)
-      if (issued[b2] > consumed[b2])
-        mbar_wait(bar_ld0 + 8 * b2, (issued[b2] - 1) & 1, &no_abort, p.timeout_ns);
+    warp_wait(bar + kBarDrain, 0, &no_abort, p.timeout_ns);
+  } else {
+    // ------------------------------------------------- element-wise warps
+    // Thread = query row x (TMEM lane); warpgroup wg takes key columns
+    // [64 wg, 64 wg + 64) of every tile.
+    const int wg = warp / 4, wq = warp % 4;
+    const int x = x0 + wq * 32 + lane;
+    const bool xvalid = x < p.c;
+    const size_t xrow = (size_t)bh * p.N + (size_t)j * p.c + (size_t)(xvalid ? x : 0);
+    const float lse2 = xvalid ? p.lse[xrow] * 1.4426950408889634f : INFINITY;
+    const float drow = xvalid ? p.dvec[xrow] : 0.f;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t myS = tS + lane_off + 64 * wg, mydP = tdP + lane_off + 64 * wg;
+    KCursor cur;
+    cur.init(p, j, x0);
+    int kb, y0, kind;
+    BlockMask bm;
+    uint32_t i = 0;
+    bool ok = true;
+    while (cur.next(kb, y0, kind, bm)) {
+      const int lim =
+          (xvalid ? ((kind == TILE_PARTIAL) ? row_limit(bm, x, y0, p.c) : kBN) : 0) - 64 * wg;
+      if (!warp_wait(bar + kBarS, i & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t a[2][32];
+      tmem_ld32(myS, a[0]);
+      tmem_ld32(myS + 32, a[1]);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar + kBarP);   // S_i read: its columns may be reused
+      float pr[64];
+#pragma unroll
+      for (int q = 0; q < 64; ++q)
+        pr[q] = (q < lim) ? bex2(fmaf(__uint_as_float(a[q / 32][q % 32]), p.c2, -lse2)) : 0.f;
+      if (!warp_wait(bar + kBarDP, i & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+      tc_fence_after();
+      tmem_ld32(mydP, a[0]);
+      tmem_ld32(mydP + 32, a[1]);
+      tmem_wait_ld();
+      uint32_t pk[32];
+#pragma unroll
+      for (int q = 0; q < 32; ++q) {
+        const float d0 = pr[2 * q] * (__uint_as_float(a[(2 * q) / 32][(2 * q) % 32]) - drow);
+        const float d1 = pr[2 * q + 1] * (__uint_as_float(a[(2 * q + 1) / 32][(2 * q + 1) % 32]) - drow);
+        pk[q] = pack2(d0, d1);
+      }
+      tmem_st32(mydP, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar + kBarDS);
+      ++i;
+    }
+    if (ok && (i == 0 || warp_wait(bar + kBarAcc, 0, abort_flag, p.timeout_ns))) {
+      tc_fence_after();
+      __nv_bfloat16* dst = p.dq + xrow * D;
+#pragma unroll 1
+      for (int q = 0; q < D / 64; ++q) {
+        const int col = wg * (D / 2) + q * 32;
+        uint32_t r[32];
+        if (i) {
+          tmem_ld32(tdQ + lane_off + col, r);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) r[u] = 0u;
+        }
+        if (xvalid) store_row32(dst + col, r, p.scale);
+      }
+    }
   }
-  tc_fence_before();
-  __syncthreads();
-  if (tid == 0 && *abort_flag && p.fault) atomicOr(p.fault, 8u);
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
-  }
+  bwd_teardown<D>(smem, tmem, warp, p, 8u);
 }
 
 // ------------------------------------------------------------------ host
@@ -605,8 +774,8 @@ static ra_status launch_bwd(const BwdLaunch& a) {
   if (blocks > (long long)a.num_sms * 16) blocks = (long long)a.num_sms * 16;
   bwd_rowdot_kernel<D><<<(int)blocks, 256, 0, st>>>(p.o, p.dout, p.dvec, rows);
   const long long items = (long long)p.BH * p.P * p.T;
-  bwd_dkdv_kernel<D><<<(unsigned)items, 128, C::kSmem, st>>>(tq, tk, tv, tdo, p);
-  bwd_dq_kernel<D><<<(unsigned)items, 128, C::kSmem, st>>>(tq, tk, tv, tdo, p);
+  bwd_dkdv_kernel<D><<<(unsigned)items, C::kThreads, C::kSmem, st>>>(tq, tk, tv, tdo, p);
+  bwd_dq_kernel<D><<<(unsigned)items, C::kThreads, C::kSmem, st>>>(tq, tk, tv, tdo, p);
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 

@@ -63,6 +63,9 @@ CASES = [
     (1, 2, 1500, 64, 5, W.STRIPED, True, 3.0),
     (1, 1, 2048, 128, 1, W.CONTIGUOUS, True, 3.0),
     (1, 2, 512, 128, 8, W.STRIPED, False, 1.0),
+    (1, 1, 4096, 128, 8, W.STRIPED, True, 3.0),       # 4 key tiles per shard
+    (1, 1, 4096, 128, 4, W.CONTIGUOUS, True, 1.0),
+    (1, 1, 3000, 64, 3, W.CONTIGUOUS, False, 1.0),    # ragged, non-causal
 ]
 
 
