@@ -16,10 +16,11 @@
 //   bwd_dq       one CTA per query tile: loops over the key tiles it sees,
 //                S = Q K^T, dP = dO V^T, dS in TMEM, dQ += dS K
 // Both tile kernels are warp-specialised like the forward: a TMA producer
-// warp (two shared-memory stages of the streamed tile pair), an MMA warp,
-// and two element-wise warpgroups (thread = TMEM lane, each warpgroup one
-// half of the 128 columns).  The MMA order overlaps the next tile's score
-// MMA with the exponentials of the current one.
+// warp (a three-slot ring for the tile of the score MMA, a two-slot ring for
+// the other streamed tile), an MMA warp, and two element-wise warpgroups
+// (thread = TMEM lane, each warpgroup one half of the 128 columns).  The MMA
+// order overlaps the next tile's score MMA with the exponentials of the
+// current one.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -83,26 +84,56 @@ __device__ __forceinline__ float bex2(float x) {
   return y;
 }
 
+// Packed fp32 pairs (f32x2 arithmetic of sm_100).
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpk2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// Shared memory of both tile kernels (no slack: the dynamic shared memory
+// base must be 1024-byte aligned, which the kernels check):
+//   F0, F1   the fixed tile pair of the CTA
+//   ring A   3 slots of the tile that feeds the score MMA (Q, resp. K)
+//   ring B   2 slots of the other streamed tile (dO, resp. V)
+//   vectors  per ring-B slot: {lse2, D} x 128 fp32 (dK/dV kernel only)
 template <int D>
 struct BwdCfg {
   static constexpr int kTile = kBM * D * 2;   // bytes of a 128 x D bf16 tile
-  // smem: the fixed tile pair (F0, F1), two stages of the streamed tile pair,
-  // a ring of four per-column vector slots ({lse2, D} x 128 fp32), barriers
+  static constexpr int kSlotsA = 3, kSlotsB = 2;
   static constexpr int kFixed0 = 0, kFixed1 = kTile;
-  static constexpr int kStream = 2 * kTile;            // + stage * 2 * kTile
-  static constexpr int kVec = 6 * kTile;
-  static constexpr int kVecSlots = 4;
-  static constexpr int kBar = kVec + kVecSlots * 2 * kBM * 4;
-  static constexpr int kSmem = kBar + 128 + 1024;
+  static constexpr int kRingA = 2 * kTile;
+  static constexpr int kRingB = kRingA + kSlotsA * kTile;
+  static constexpr int kVec = kRingB + kSlotsB * kTile;
+  static constexpr int kBar = kVec + kSlotsB * 2 * kBM * 4;
+  static constexpr int kSmem = kBar + 256;
   static constexpr int kThreads = 320;   // 8 element-wise warps, producer, MMA
 };
 
 // Barrier offsets from BwdCfg::kBar (8 bytes each); tmem slot and abort flag
-// after them.  A stage has two full barriers: kBarFull for its first tile
-// (the operand of the score MMA), kBarFull2 for its second.
+// after them.
 enum : uint32_t {
-  kBarFixed = 0, kBarFull = 8, kBarEmpty = 24, kBarS = 40, kBarDP = 48, kBarP = 56,
-  kBarDS = 64, kBarAcc = 72, kBarDrain = 80, kBarFull2 = 88, kTmemSlot = 112, kAbort = 116
+  kBarFixed = 0, kBarFullA = 8, kBarEmptyA = 32, kBarFullB = 56, kBarEmptyB = 72, kBarS = 88,
+  kBarDP = 96, kBarP = 104, kBarDS = 112, kBarAcc = 120, kBarDrain = 128, kTmemSlot = 136,
+  kAbort = 140
 };
 
 // TMA: one 128 x D tile of a [BH, P, c, D] tensor at (shard, row0, bh).
@@ -162,17 +193,20 @@ __device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (
 // prefetch.  Returns the TMEM base.
 template <int D>
 __device__ __forceinline__ uint32_t bwd_setup(uint8_t* smem, int warp, int lane,
-                                              uint32_t full_count, const CUtensorMap* m0,
+                                              uint32_t fullb_count, const CUtensorMap* m0,
                                               const CUtensorMap* m1, const CUtensorMap* m2,
                                               const CUtensorMap* m3) {
   using C = BwdCfg<D>;
   const uint32_t bar = smem_u32(smem) + C::kBar;
   if (threadIdx.x == 0) {
     mbar_init(bar + kBarFixed, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar + kBarFull + 8 * s, full_count);
-      mbar_init(bar + kBarFull2 + 8 * s, 1);
-      mbar_init(bar + kBarEmpty + 8 * s, 1);
+    for (int s = 0; s < C::kSlotsA; ++s) {
+      mbar_init(bar + kBarFullA + 8 * s, 1);
+      mbar_init(bar + kBarEmptyA + 8 * s, 1);
+    }
+    for (int s = 0; s < C::kSlotsB; ++s) {
+      mbar_init(bar + kBarFullB + 8 * s, fullb_count);
+      mbar_init(bar + kBarEmptyB + 8 * s, 1);
     }
     mbar_init(bar + kBarS, 1);
     mbar_init(bar + kBarDP, 1);
@@ -214,23 +248,39 @@ __device__ __forceinline__ void bwd_teardown(uint8_t* smem, uint32_t tmem, int w
   }
 }
 
+// The tile layouts need a 1024-byte aligned shared memory base; the launch
+// leaves no slack to align it by hand.  A misaligned base (not expected) is
+// reported as fault code 16 and the CTA does nothing.
+__device__ __forceinline__ bool smem_base_ok(const uint8_t* smem, const BwdParams& p) {
+  if ((smem_u32(smem) & 1023u) == 0) return true;
+  if (threadIdx.x == 0 && p.fault) atomicOr(p.fault, 16u);
+  return false;
+}
+
 // ------------------------------------------------------------- dK, dV
 // Work item: key tile kt of block kb of (b, h).  Query tiles visiting it:
 // every (query shard j, tile qt) whose tile against this key tile is not
 // skipped; shards in ascending order, so that the CTAs running at the same
 // time stream the same query tiles through L2 (the gradient is a sum, its
-// order is free).
+// order is free).  On a diagonal block, query tiles before kt - 1 cannot see
+// key tile kt (a query tile qt reaches keys up to (qt + 1) * 128 - 1 + e),
+// so the walk starts there.
 struct QCursor {
   int j, qt, P, T, c, kb, striped, causal, y0;
+  BlockMask m;
   __device__ void init(const BwdParams& p, int kb_, int y0_) {
-    j = 0; qt = 0; P = p.P; T = p.T; c = p.c; kb = kb_; striped = p.striped; causal = p.causal;
+    j = 0; qt = -1; P = p.P; T = p.T; c = p.c; kb = kb_; striped = p.striped; causal = p.causal;
     y0 = y0_;
   }
   __device__ bool next(int& oj, int& oqt) {
     while (j < P) {
-      if (qt >= T) { qt = 0; ++j; continue; }
-      const BlockMask m = block_mask(j, kb, striped, causal);
-      if (m.all_hidden) { qt = T; continue; }
+      if (qt < 0) {
+        m = block_mask(j, kb, striped, causal);
+        if (m.all_hidden) { ++j; continue; }
+        const int kt = y0 / kBN;
+        qt = (m.use_diag && kt > 0) ? kt - 1 : 0;
+      }
+      if (qt >= T) { qt = -1; ++j; continue; }
       const int k = tile_kind(m, qt * kBM, y0, c);
       ++qt;
       if (k != TILE_SKIP) { oj = j; oqt = qt - 1; return true; }
@@ -257,20 +307,20 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                 const BwdParams p) {
   using C = BwdCfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (!smem_base_ok(smem, p)) return;
   const uint32_t sb = smem_u32(smem), bar = sb + C::kBar;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBar + kAbort);
-  float* vec = reinterpret_cast<float*>(smem + C::kVec);   // [stage][lse2 | D][128]
+  float* vec = reinterpret_cast<float*>(smem + C::kVec);   // [ring-B slot][lse2 | D][128]
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   int bh, kb, kt;
   dkdv_item(p, blockIdx.x, bh, kb, kt);
   const int y0 = kt * kBN;
 
-  // producer lanes all arrive on a stage after writing its vectors
+  // ring B (dO + vectors): the 32 producer lanes arrive after their writes
   const uint32_t tmem = bwd_setup<D>(smem, warp, lane, 32, &tmQ, &tmK, &tmV, &tmdO);
   const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 256 + D;
+  const uint32_t ringA = sb + C::kRingA, ringB = sb + C::kRingB;
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
@@ -281,49 +331,60 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
     QCursor cur;
     cur.init(p, kb, y0);
-    uint32_t n = 0;
+    uint32_t na = 0, nb = 0;   // tiles issued into ring A / ring B
     int j, qt;
     while (cur.next(j, qt)) {
-      const int s = n & 1;
-      // Per-column lse (log2 units) and D of this query tile, into vector
-      // slot n mod 4 before the stage is free, so that their load latency
-      // is off the critical path.  Slot n mod 4 was last read for tile n-4,
-      // which finished before the stage wait of tile n-2 passed.
-      float* v = vec + (n % C::kVecSlots) * 2 * kBM;
+      // per-column lse (log2 units) and D of this query tile, loaded before
+      // the waits so that their latency is hidden
+      float lv[4], dv[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int q = lane + 32 * u, x = qt * kBM + q;
+        const int x = qt * kBM + lane + 32 * u;
         const bool valid = x < p.c;
         const size_t row = (size_t)bh * p.N + (size_t)j * p.c + (size_t)(valid ? x : 0);
-        v[q] = valid ? p.lse[row] * 1.4426950408889634f : INFINITY;
-        v[kBM + q] = valid ? p.dvec[row] : 0.f;
+        lv[u] = valid ? p.lse[row] * 1.4426950408889634f : INFINITY;
+        dv[u] = valid ? p.dvec[row] : 0.f;
       }
-      if (n >= 2 && !warp_wait(bar + kBarEmpty + 8 * s, ((n >> 1) - 1) & 1, abort_flag, p.timeout_ns))
+      const uint32_t a = na % C::kSlotsA;
+      if (na >= C::kSlotsA &&
+          !warp_wait(bar + kBarEmptyA + 8 * a, (na / C::kSlotsA - 1) & 1, abort_flag, p.timeout_ns))
         break;
-      const uint32_t dst = sb + C::kStream + s * 2 * C::kTile;
       if (lane == 0) {
-        mbar_arrive_expect_tx(bar + kBarFull + 8 * s, C::kTile);
-        load_tile<D>(dst, &tmQ, bar + kBarFull + 8 * s, qt * kBM, j, bh);
-        mbar_arrive_expect_tx(bar + kBarFull2 + 8 * s, C::kTile);
-        load_tile<D>(dst + C::kTile, &tmdO, bar + kBarFull2 + 8 * s, qt * kBM, j, bh);
-      } else {
-        mbar_arrive(bar + kBarFull + 8 * s);
+        mbar_arrive_expect_tx(bar + kBarFullA + 8 * a, C::kTile);
+        load_tile<D>(ringA + a * C::kTile, &tmQ, bar + kBarFullA + 8 * a, qt * kBM, j, bh);
       }
-      ++n;
+      ++na;
+      const uint32_t b = nb & 1;
+      if (nb >= 2 && !warp_wait(bar + kBarEmptyB + 8 * b, ((nb >> 1) - 1) & 1, abort_flag, p.timeout_ns))
+        break;
+      float* v = vec + b * 2 * kBM;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        v[lane + 32 * u] = lv[u];
+        v[kBM + lane + 32 * u] = dv[u];
+      }
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar + kBarFullB + 8 * b, C::kTile);
+        load_tile<D>(ringB + b * C::kTile, &tmdO, bar + kBarFullB + 8 * b, qt * kBM, j, bh);
+      } else {
+        mbar_arrive(bar + kBarFullB + 8 * b);
+      }
+      ++nb;
     }
     // every issued load must have landed before the CTA exits
     if (lane == 0) {
       volatile int no_abort = 0;
       mbar_wait(bar + kBarFixed, 0, &no_abort, p.timeout_ns);
-      for (uint32_t m = n > 2 ? n - 2 : 0; m < n; ++m) {
-        mbar_wait(bar + kBarFull + 8 * (m & 1), (m >> 1) & 1, &no_abort, p.timeout_ns);
-        mbar_wait(bar + kBarFull2 + 8 * (m & 1), (m >> 1) & 1, &no_abort, p.timeout_ns);
-      }
+      for (uint32_t m = na > (uint32_t)C::kSlotsA ? na - C::kSlotsA : 0; m < na; ++m)
+        mbar_wait(bar + kBarFullA + 8 * (m % C::kSlotsA), (m / C::kSlotsA) & 1, &no_abort,
+                  p.timeout_ns);
+      for (uint32_t m = nb > 2u ? nb - 2 : 0; m < nb; ++m)
+        mbar_wait(bar + kBarFullB + 8 * (m & 1), (m >> 1) & 1, &no_abort, p.timeout_ns);
     }
     __syncwarp();
   } else if (warp == 9) {
     // ---------------------------------------------------------- MMA issuer
-    // Order per query tile i (stage s):  dV += P_i^T dO_i, S_{i+1} = K Q_{i+1}^T,
+    // Order per query tile i:  dV += P_i^T dO_i, S_{i+1} = K Q_{i+1}^T,
     // dK += dS_i^T Q_i, dP_{i+1} = V dO_{i+1}^T.  S_{i+1} reuses the columns
     // of P_i right after the MMA that reads them (tcgen05 MMAs of one CTA
     // run in issue order), so the tensor core computes the next scores while
@@ -335,45 +396,46 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     bool have = cur.next(j, qt);
     uint32_t i = 0;
     if (ok && have) {
-      ok = warp_wait(bar + kBarFull, 0, abort_flag, p.timeout_ns);
+      ok = warp_wait(bar + kBarFullA, 0, abort_flag, p.timeout_ns);
       if (ok) {
         tc_fence_after();
-        bwd_mma_ss<D>(tS, sb + C::kFixed0, sb + C::kStream);
+        bwd_mma_ss<D>(tS, sb + C::kFixed0, ringA);
         mma_commit_w(bar + kBarS);
-        ok = warp_wait(bar + kBarFull2, 0, abort_flag, p.timeout_ns);
+        ok = warp_wait(bar + kBarFullB, 0, abort_flag, p.timeout_ns);
       }
       if (ok) {
         tc_fence_after();
-        bwd_mma_ss<D>(tdP, sb + C::kFixed1, sb + C::kStream + C::kTile);
+        bwd_mma_ss<D>(tdP, sb + C::kFixed1, ringB);
         mma_commit_w(bar + kBarDP);
       }
     }
     while (ok && have) {
-      const int s = i & 1;
-      const uint32_t sq = sb + C::kStream + s * 2 * C::kTile, sdo = sq + C::kTile;
-      const uint32_t nq = sb + C::kStream + (s ^ 1) * 2 * C::kTile, ndo = nq + C::kTile;
+      const uint32_t a = i % C::kSlotsA, b = i & 1;
+      const uint32_t an = (i + 1) % C::kSlotsA, bn = b ^ 1;
       const bool more = cur.next(j, qt);
       if (!warp_wait(bar + kBarP, i & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
       tc_fence_after();
-      bwd_mma_ts<D>(tdV, tS, sdo, i > 0);
+      bwd_mma_ts<D>(tdV, tS, ringB + b * C::kTile, i > 0);
       if (more) {
-        if (!warp_wait(bar + kBarFull + 8 * (s ^ 1), ((i + 1) >> 1) & 1, abort_flag, p.timeout_ns)) {
+        if (!warp_wait(bar + kBarFullA + 8 * an, ((i + 1) / C::kSlotsA) & 1, abort_flag,
+                       p.timeout_ns)) {
           ok = false; break;
         }
         tc_fence_after();
-        bwd_mma_ss<D>(tS, sb + C::kFixed0, nq);
+        bwd_mma_ss<D>(tS, sb + C::kFixed0, ringA + an * C::kTile);
         mma_commit_w(bar + kBarS);
       }
       if (!warp_wait(bar + kBarDS, i & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
       tc_fence_after();
-      bwd_mma_ts<D>(tdK, tdP, sq, i > 0);
-      mma_commit_w(bar + kBarEmpty + 8 * s);
+      bwd_mma_ts<D>(tdK, tdP, ringA + a * C::kTile, i > 0);
+      mma_commit_w(bar + kBarEmptyA + 8 * a);
+      mma_commit_w(bar + kBarEmptyB + 8 * b);
       if (more) {
-        if (!warp_wait(bar + kBarFull2 + 8 * (s ^ 1), ((i + 1) >> 1) & 1, abort_flag, p.timeout_ns)) {
+        if (!warp_wait(bar + kBarFullB + 8 * bn, ((i + 1) >> 1) & 1, abort_flag, p.timeout_ns)) {
           ok = false; break;
         }
         tc_fence_after();
-        bwd_mma_ss<D>(tdP, sb + C::kFixed1, ndo);
+        bwd_mma_ss<D>(tdP, sb + C::kFixed1, ringB + bn * C::kTile);
         mma_commit_w(bar + kBarDP);
       }
       ++i;
@@ -392,24 +454,25 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const int y = y0 + wq * 32 + lane;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t myS = tS + lane_off + 64 * wg, mydP = tdP + lane_off + 64 * wg;
+    const uint64_t c2x2 = pk2(p.c2, p.c2);
     QCursor cur;
     cur.init(p, kb, y0);
     int j, qt;
     uint32_t i = 0;
     bool ok = true;
     while (cur.next(j, qt)) {
-      const int s = i & 1;
-      const BlockMask bm = block_mask(j, kb, p.striped, p.causal);
+      const uint32_t b = i & 1;
       int lo = 0, hi = p.c - qt * kBM;          // visible query columns [lo, hi)
-      if (bm.use_diag) {
-        const int l2 = y + 1 - bm.e - qt * kBM;  // query x sees key y iff y < x + e
+      if (cur.m.use_diag) {
+        const int l2 = y + 1 - cur.m.e - qt * kBM;   // query x sees key y iff y < x + e
         lo = l2 > 0 ? l2 : 0;
       }
       if (y >= p.c) hi = 0;
       lo -= 64 * wg;
       hi -= 64 * wg;
+      const bool all_vis = __all_sync(0xffffffffu, lo <= 0 && hi >= 64) != 0;
       if (!warp_wait(bar + kBarS, i & 1, abort_flag, p.timeout_ns) ||
-          !warp_wait(bar + kBarFull + 8 * s, (i >> 1) & 1, abort_flag, p.timeout_ns)) {
+          !warp_wait(bar + kBarFullB + 8 * b, (i >> 1) & 1, abort_flag, p.timeout_ns)) {
         ok = false; break;
       }
       tc_fence_after();
@@ -417,24 +480,34 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tmem_ld32(myS, a[0]);
       tmem_ld32(myS + 32, a[1]);
       tmem_wait_ld();
-      const float4* lse2 = reinterpret_cast<const float4*>(vec + (i % C::kVecSlots) * 2 * kBM + 64 * wg);
+      const float4* lse2 = reinterpret_cast<const float4*>(vec + b * 2 * kBM + 64 * wg);
       const float4* dcol = lse2 + kBM / 4;
       float pr[64];
-      uint32_t pk[32];
+      uint32_t pkd[32];
+      // P = exp2(S * c2 - lse2), packed pairs
 #pragma unroll
       for (int q4 = 0; q4 < 16; ++q4) {
         const float4 l4 = lse2[q4];
-        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int q = 4 * q4 + u;
-          const float sv = __uint_as_float(a[q / 32][q % 32]);
-          pr[q] = (q >= lo && q < hi) ? bex2(fmaf(sv, p.c2, -lv[u])) : 0.f;
+        for (int h = 0; h < 2; ++h) {
+          const int q = 4 * q4 + 2 * h;
+          const uint64_t nl = pk2(-(h ? l4.z : l4.x), -(h ? l4.w : l4.y));
+          const uint64_t t = fma2(pk2(__uint_as_float(a[q / 32][q % 32]),
+                                      __uint_as_float(a[q / 32][q % 32 + 1])), c2x2, nl);
+          float t0, t1;
+          unpk2(t, t0, t1);
+          pr[q] = bex2(t0);
+          pr[q + 1] = bex2(t1);
         }
       }
+      if (!all_vis) {
 #pragma unroll
-      for (int q = 0; q < 32; ++q) pk[q] = pack2(pr[2 * q], pr[2 * q + 1]);
-      tmem_st32(myS, pk);
+        for (int q = 0; q < 64; ++q)
+          if (q < lo || q >= hi) pr[q] = 0.f;
+      }
+#pragma unroll
+      for (int q = 0; q < 32; ++q) pkd[q] = pack2(pr[2 * q], pr[2 * q + 1]);
+      tmem_st32(myS, pkd);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -444,20 +517,23 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tmem_ld32(mydP, a[0]);
       tmem_ld32(mydP + 32, a[1]);
       tmem_wait_ld();
+      // dS = P (dP - D), packed pairs
 #pragma unroll
       for (int q4 = 0; q4 < 16; ++q4) {
         const float4 d4 = dcol[q4];
-        const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
-        float ds[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int q = 4 * q4 + u;
-          ds[u] = pr[q] * (__uint_as_float(a[q / 32][q % 32]) - dv[u]);
+        for (int h = 0; h < 2; ++h) {
+          const int q = 4 * q4 + 2 * h;
+          const uint64_t dp = pk2(__uint_as_float(a[q / 32][q % 32]),
+                                  __uint_as_float(a[q / 32][q % 32 + 1]));
+          const uint64_t ds =
+              mul2(pk2(pr[q], pr[q + 1]), sub2(dp, pk2(h ? d4.z : d4.x, h ? d4.w : d4.y)));
+          float d0, d1;
+          unpk2(ds, d0, d1);
+          pkd[q / 2] = pack2(d0, d1);
         }
-        pk[2 * q4] = pack2(ds[0], ds[1]);
-        pk[2 * q4 + 1] = pack2(ds[2], ds[3]);
       }
-      tmem_st32(mydP, pk);
+      tmem_st32(mydP, pkd);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -540,9 +616,8 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
               const BwdParams p) {
   using C = BwdCfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (!smem_base_ok(smem, p)) return;
   const uint32_t sb = smem_u32(smem), bar = sb + C::kBar;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBar + kAbort);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -552,6 +627,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 
   const uint32_t tmem = bwd_setup<D>(smem, warp, lane, 1, &tmQ, &tmK, &tmV, &tmdO);
   const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
+  const uint32_t ringA = sb + C::kRingA, ringB = sb + C::kRingB;
 
   if (warp == 8) {
     // ------------------------------------------------------------ producer
@@ -561,33 +637,38 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       load_tile<D>(sb + C::kFixed1, &tmdO, bar + kBarFixed, x0, j, bh);
       KCursor cur;
       cur.init(p, j, x0);
-      uint32_t n = 0;
+      uint32_t na = 0, nb = 0;
       int kb, y0, kind;
       BlockMask bm;
       while (cur.next(kb, y0, kind, bm)) {
-        const int s = n & 1;
-        if (n >= 2 && !mbar_wait(bar + kBarEmpty + 8 * s, ((n >> 1) - 1) & 1, abort_flag, p.timeout_ns))
+        const uint32_t a = na % C::kSlotsA;
+        if (na >= C::kSlotsA &&
+            !mbar_wait(bar + kBarEmptyA + 8 * a, (na / C::kSlotsA - 1) & 1, abort_flag, p.timeout_ns))
           break;
-        const uint32_t dst = sb + C::kStream + s * 2 * C::kTile;
-        mbar_arrive_expect_tx(bar + kBarFull + 8 * s, C::kTile);
-        load_tile<D>(dst, &tmK, bar + kBarFull + 8 * s, y0, kb, bh);
-        mbar_arrive_expect_tx(bar + kBarFull2 + 8 * s, C::kTile);
-        load_tile<D>(dst + C::kTile, &tmV, bar + kBarFull2 + 8 * s, y0, kb, bh);
-        ++n;
+        mbar_arrive_expect_tx(bar + kBarFullA + 8 * a, C::kTile);
+        load_tile<D>(ringA + a * C::kTile, &tmK, bar + kBarFullA + 8 * a, y0, kb, bh);
+        ++na;
+        const uint32_t b = nb & 1;
+        if (nb >= 2 && !mbar_wait(bar + kBarEmptyB + 8 * b, ((nb >> 1) - 1) & 1, abort_flag, p.timeout_ns))
+          break;
+        mbar_arrive_expect_tx(bar + kBarFullB + 8 * b, C::kTile);
+        load_tile<D>(ringB + b * C::kTile, &tmV, bar + kBarFullB + 8 * b, y0, kb, bh);
+        ++nb;
       }
       volatile int no_abort = 0;
       mbar_wait(bar + kBarFixed, 0, &no_abort, p.timeout_ns);
-      for (uint32_t m = n > 2 ? n - 2 : 0; m < n; ++m) {
-        mbar_wait(bar + kBarFull + 8 * (m & 1), (m >> 1) & 1, &no_abort, p.timeout_ns);
-        mbar_wait(bar + kBarFull2 + 8 * (m & 1), (m >> 1) & 1, &no_abort, p.timeout_ns);
-      }
+      for (uint32_t m = na > (uint32_t)C::kSlotsA ? na - C::kSlotsA : 0; m < na; ++m)
+        mbar_wait(bar + kBarFullA + 8 * (m % C::kSlotsA), (m / C::kSlotsA) & 1, &no_abort,
+                  p.timeout_ns);
+      for (uint32_t m = nb > 2u ? nb - 2 : 0; m < nb; ++m)
+        mbar_wait(bar + kBarFullB + 8 * (m & 1), (m >> 1) & 1, &no_abort, p.timeout_ns);
     }
     __syncwarp();
   } else if (warp == 9) {
     // ---------------------------------------------------------- MMA issuer
-    // Order per key tile i (stage s): S_{i+1} = Q K_{i+1}^T as soon as the
-    // element-wise warps have read S_i; dQ += dS_i K_i; dP_{i+1} = dO V_{i+1}^T
-    // into the columns of dS_i right after the MMA that reads them.
+    // Order per key tile i: S_{i+1} = Q K_{i+1}^T as soon as the element-wise
+    // warps have read S_i; dQ += dS_i K_i; dP_{i+1} = dO V_{i+1}^T into the
+    // columns of dS_i right after the MMA that reads them.
     KCursor cur;
     cur.init(p, j, x0);
     int kb, y0, kind;
@@ -596,44 +677,45 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     bool have = cur.next(kb, y0, kind, bm);
     uint32_t i = 0;
     if (ok && have) {
-      ok = warp_wait(bar + kBarFull, 0, abort_flag, p.timeout_ns);
+      ok = warp_wait(bar + kBarFullA, 0, abort_flag, p.timeout_ns);
       if (ok) {
         tc_fence_after();
-        bwd_mma_ss<D>(tS, sb + C::kFixed0, sb + C::kStream);
+        bwd_mma_ss<D>(tS, sb + C::kFixed0, ringA);
         mma_commit_w(bar + kBarS);
-        ok = warp_wait(bar + kBarFull2, 0, abort_flag, p.timeout_ns);
+        ok = warp_wait(bar + kBarFullB, 0, abort_flag, p.timeout_ns);
       }
       if (ok) {
         tc_fence_after();
-        bwd_mma_ss<D>(tdP, sb + C::kFixed1, sb + C::kStream + C::kTile);
+        bwd_mma_ss<D>(tdP, sb + C::kFixed1, ringB);
         mma_commit_w(bar + kBarDP);
       }
     }
     while (ok && have) {
-      const int s = i & 1;
-      const uint32_t sk = sb + C::kStream + s * 2 * C::kTile;
-      const uint32_t nk = sb + C::kStream + (s ^ 1) * 2 * C::kTile, nv = nk + C::kTile;
+      const uint32_t a = i % C::kSlotsA, b = i & 1;
+      const uint32_t an = (i + 1) % C::kSlotsA, bn = b ^ 1;
       const bool more = cur.next(kb, y0, kind, bm);
       if (more) {
         // kBarP: the element-wise warps have read S_i
         if (!warp_wait(bar + kBarP, i & 1, abort_flag, p.timeout_ns) ||
-            !warp_wait(bar + kBarFull + 8 * (s ^ 1), ((i + 1) >> 1) & 1, abort_flag, p.timeout_ns)) {
+            !warp_wait(bar + kBarFullA + 8 * an, ((i + 1) / C::kSlotsA) & 1, abort_flag,
+                       p.timeout_ns)) {
           ok = false; break;
         }
         tc_fence_after();
-        bwd_mma_ss<D>(tS, sb + C::kFixed0, nk);
+        bwd_mma_ss<D>(tS, sb + C::kFixed0, ringA + an * C::kTile);
         mma_commit_w(bar + kBarS);
       }
       if (!warp_wait(bar + kBarDS, i & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
       tc_fence_after();
-      bwd_mma_ts<D>(tdQ, tdP, sk, i > 0);
-      mma_commit_w(bar + kBarEmpty + 8 * s);
+      bwd_mma_ts<D>(tdQ, tdP, ringA + a * C::kTile, i > 0);
+      mma_commit_w(bar + kBarEmptyA + 8 * a);
+      mma_commit_w(bar + kBarEmptyB + 8 * b);
       if (more) {
-        if (!warp_wait(bar + kBarFull2 + 8 * (s ^ 1), ((i + 1) >> 1) & 1, abort_flag, p.timeout_ns)) {
+        if (!warp_wait(bar + kBarFullB + 8 * bn, ((i + 1) >> 1) & 1, abort_flag, p.timeout_ns)) {
           ok = false; break;
         }
         tc_fence_after();
-        bwd_mma_ss<D>(tdP, sb + C::kFixed1, nv);
+        bwd_mma_ss<D>(tdP, sb + C::kFixed1, ringB + bn * C::kTile);
         mma_commit_w(bar + kBarDP);
       }
       ++i;
@@ -653,6 +735,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const size_t xrow = (size_t)bh * p.N + (size_t)j * p.c + (size_t)(xvalid ? x : 0);
     const float lse2 = xvalid ? p.lse[xrow] * 1.4426950408889634f : INFINITY;
     const float drow = xvalid ? p.dvec[xrow] : 0.f;
+    const uint64_t c2x2 = pk2(p.c2, p.c2), nl2 = pk2(-lse2, -lse2), d2 = pk2(drow, drow);
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t myS = tS + lane_off + 64 * wg, mydP = tdP + lane_off + 64 * wg;
     KCursor cur;
@@ -664,6 +747,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     while (cur.next(kb, y0, kind, bm)) {
       const int lim =
           (xvalid ? ((kind == TILE_PARTIAL) ? row_limit(bm, x, y0, p.c) : kBN) : 0) - 64 * wg;
+      const bool all_vis = __all_sync(0xffffffffu, lim >= 64) != 0;
       if (!warp_wait(bar + kBarS, i & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
       tc_fence_after();
       uint32_t a[2][32];
@@ -675,21 +759,35 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       if (lane == 0) mbar_arrive(bar + kBarP);   // S_i read: its columns may be reused
       float pr[64];
 #pragma unroll
-      for (int q = 0; q < 64; ++q)
-        pr[q] = (q < lim) ? bex2(fmaf(__uint_as_float(a[q / 32][q % 32]), p.c2, -lse2)) : 0.f;
+      for (int q = 0; q < 64; q += 2) {
+        const uint64_t t = fma2(pk2(__uint_as_float(a[q / 32][q % 32]),
+                                    __uint_as_float(a[q / 32][q % 32 + 1])), c2x2, nl2);
+        float t0, t1;
+        unpk2(t, t0, t1);
+        pr[q] = bex2(t0);
+        pr[q + 1] = bex2(t1);
+      }
+      if (!all_vis) {
+#pragma unroll
+        for (int q = 0; q < 64; ++q)
+          if (q >= lim) pr[q] = 0.f;
+      }
       if (!warp_wait(bar + kBarDP, i & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
       tc_fence_after();
       tmem_ld32(mydP, a[0]);
       tmem_ld32(mydP + 32, a[1]);
       tmem_wait_ld();
-      uint32_t pk[32];
+      uint32_t pkd[32];
 #pragma unroll
-      for (int q = 0; q < 32; ++q) {
-        const float d0 = pr[2 * q] * (__uint_as_float(a[(2 * q) / 32][(2 * q) % 32]) - drow);
-        const float d1 = pr[2 * q + 1] * (__uint_as_float(a[(2 * q + 1) / 32][(2 * q + 1) % 32]) - drow);
-        pk[q] = pack2(d0, d1);
+      for (int q = 0; q < 64; q += 2) {
+        const uint64_t dp = pk2(__uint_as_float(a[q / 32][q % 32]),
+                                __uint_as_float(a[q / 32][q % 32 + 1]));
+        const uint64_t ds = mul2(pk2(pr[q], pr[q + 1]), sub2(dp, d2));
+        float d0, d1;
+        unpk2(ds, d0, d1);
+        pkd[q / 2] = pack2(d0, d1);
       }
-      tmem_st32(mydP, pk);
+      tmem_st32(mydP, pkd);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
