@@ -53,10 +53,15 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+# The sources the forward kernel is compiled from (its file and what it
+# includes): a recorded ncu traffic figure is valid while these are unchanged.
+FWD_SOURCES = ("attn_fwd.cu", "exp2_poly.h", "ra_internal.h", "ra_ptx.cuh", "ra_tiles.cuh")
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "long_context_exact_attn_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in FWD_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -400,8 +405,16 @@ def main():
         bms = timed(bwd_step, max(1, min(args.steps, 3)), world)
         if ops.device_fault():
             raise RuntimeError("device fault during the backward pass")
-        backward = {"ms": bms, "useful_tflops": 2.5 * flops / (bms * 1e-3) / 1e12,
-                    "flop_convention": "10 d per visible pair (QK^T, dO V^T, dV, dK, dQ)"}
+        # useful: 10 d FLOP per visible pair (the five products of the
+        # gradient); executed: 14 d (the dQ kernel recomputes S and dP)
+        useful = 2.5 * flops / (bms * 1e-3) / 1e12
+        executed = 3.5 * flops / (bms * 1e-3) / 1e12
+        backward = {"ms": bms, "useful_tflops": useful, "executed_tflops": executed,
+                    "frac_executed_of_sustained_peak":
+                        executed / float(peaks.get("bf16_tflops_sustained",
+                                                   FALLBACK_PEAKS["bf16_tflops_sustained"])),
+                    "flop_convention": "useful 10 d per visible pair (QK^T, dO V^T, dV, dK, dQ); "
+                                       "executed 14 d (S and dP recomputed for dQ)"}
 
     # ---- CPU oracle baseline (rank 0, one GPU only)
     cpu = None
