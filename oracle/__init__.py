@@ -23,6 +23,9 @@ source pages:
   Ring Attention 工作负载 / Striped Attention 工作负载) and brute-force counts.
 * ``backward``     -- gradients dQ, dK, dV of the definition (the pages give
   no backward; the textbook softmax derivative of 核心公式).
+* ``rope``         -- rotary position embedding at the original token
+  positions, then the stripe (Striped review, 位置编码处理 names RoPE; the
+  rotation itself is RoFormer's, not defined on the pages).
 * ``merge``        -- merging two partial (O, lse) results by splitting the
   softmax denominator into per-node partial sums (1cademy page "Computing
   Attention Weights in Sequence Parallelism").
@@ -34,4 +37,4 @@ Functions with no such pin say "parity unpinned" in their docstring; there are
 none at present.
 """
 
-from . import attention, backward, merge, masks, partition, ring, work  # noqa: F401
+from . import attention, backward, merge, masks, partition, ring, rope, work  # noqa: F401

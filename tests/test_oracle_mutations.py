@@ -170,3 +170,37 @@ def test_backward_mutants_fail_autograd_pin(monkeypatch, kind):
     monkeypatch.setattr(OB, "attention_backward", _backward_mutant(kind))
     with pytest.raises(AssertionError):
         TB.test_backward_equals_torch_autograd(True, 9, 8)
+
+
+def _rope_mutant(kind):
+    from oracle import rope as R
+
+    def f(x, pos, base=10000.0, pairing=R.INTERLEAVED):
+        x = np.asarray(x, dtype=np.float64)
+        d = x.shape[-1]
+        i = np.arange(d // 2, dtype=np.float64)
+        expo = -i / d if kind == "freq_exponent" else -2.0 * i / d
+        ang = np.asarray(pos, dtype=np.float64)[:, None] * np.power(float(base), expo)[None, :]
+        cos, sin = np.cos(ang), np.sin(ang)
+        use = R.HALF if (kind == "pairing_swapped" and pairing == R.INTERLEAVED) else pairing
+        a, b = R.pair_index(d, use)
+        u, w = x[..., a], x[..., b]
+        out = np.empty_like(x)
+        if kind == "sign":
+            out[..., a] = u * cos + w * sin
+            out[..., b] = -u * sin + w * cos
+        else:
+            out[..., a] = u * cos - w * sin
+            out[..., b] = u * sin + w * cos
+        return out
+    return f
+
+
+@pytest.mark.parametrize("kind", ["sign", "freq_exponent", "pairing_swapped"])
+def test_rope_mutants_fail_closed_form_pins(monkeypatch, kind):
+    import tests.test_oracle_rope as TR
+    from oracle import rope as R
+    monkeypatch.setattr(R, "rope", _rope_mutant(kind))
+    with pytest.raises(AssertionError):
+        TR.test_d2_rotation_values()
+        TR.test_d4_frequencies_and_pairings()
