@@ -282,6 +282,8 @@ def main():
     ap.add_argument("--no-compare", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-rope", action="store_true",
+                    help="skip timing the stripe + RoPE partition of q")
     ap.add_argument("--backward", action="store_true",
                     help="also time the backward pass (dQ, dK, dV) on the same workload")
     ap.add_argument("--ref-budget", type=float, default=15.0,
@@ -416,6 +418,26 @@ def main():
                     "flop_convention": "useful 10 d per visible pair (QK^T, dO V^T, dV, dK, dQ); "
                                        "executed 14 d (S and dP recomputed for dQ)"}
 
+    # ---- stripe + RoPE of q and k (memory-bound side path, not in the step)
+    rope = None
+    if not args.no_rope:
+        dst = torch.empty_like(path.q)
+
+        def rope_step():
+            ops.partition_rope(path.q, w.P, w.layout, 10000.0, ops.ROPE_HALF, out=dst)
+
+        rope_step()
+        rms = timed(rope_step, 5, world)
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        moved = 2 * path.q.numel() * path.q.element_size()   # read + write
+        rope = {"kernel": "partition_rope_kernel<1>", "ms": rms, "bytes": moved,
+                "gbs": moved / (rms * 1e-3) / 1e9, "peak_gbs": hbm,
+                "frac_of_hbm": moved / (rms * 1e-3) / 1e9 / hbm, "bound": "hbm",
+                "tensor": "q [B, H, N, d] bf16, RoPE split-halves pairs, base 1e4"}
+        del dst
+        if ops.device_fault():
+            raise RuntimeError("device fault during the RoPE partition")
+
     # ---- CPU oracle baseline (rank 0, one GPU only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -455,6 +477,7 @@ def main():
         "e2e": e2e,
         "layout_compare": compare,
         "backward": backward,
+        "rope_partition": rope,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

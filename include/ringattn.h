@@ -64,6 +64,7 @@ typedef int ra_status;
 #define RA_ERR_DEVICE_FAULT 11 /* a kernel gave up a bounded wait (see below)  */
 #define RA_ERR_SCRATCH 12    /* problem larger than the built-in scratch of    */
                              /* ra_attn_bwd_noalloc (B*H*N > 1048576)          */
+#define RA_ERR_ROPE 13       /* unknown RoPE pairing, or base not > 1 / finite */
 
 /* Layouts (low byte of `layout`). */
 #define RA_CONTIGUOUS 0      /* shard j = tokens [j*c, (j+1)*c)  (Ring)        */
@@ -77,6 +78,10 @@ typedef int ra_status;
  * RA_SCHED_FREE: every SM takes work from every shard (a single-GPU
  * load-balanced schedule; same results, same tile skipping). */
 #define RA_SCHED_FREE 0x100
+
+/* Rotation pairs of ra_partition_rope. */
+#define RA_ROPE_INTERLEAVED 0 /* pair i = dimensions (2i, 2i+1)                */
+#define RA_ROPE_HALF 1        /* pair i = dimensions (i, i + d/2)              */
 
 /* Element types for ra_partition. */
 #define RA_BF16 0
@@ -112,6 +117,33 @@ int ra_version(void);
  */
 ra_status ra_partition(const void* src, void* dst, int64_t B, int64_t H, int64_t N, int64_t d,
                        int P, int layout, int inverse, int dtype, void* stream);
+
+/*
+ * ra_partition_rope -- token order -> layout order with rotary position
+ * embedding applied at the ORIGINAL token positions.
+ *
+ * The Striped review (位置编码处理) requires a position encoding such as RoPE
+ * to see the same stripe permutation as the tokens.  The pages name RoPE but
+ * do not define it; this is RoFormer's rotation: with theta_i =
+ * base^(-2i/d), pair i of row t is turned by the angle t * theta_i,
+ *     (u, w) -> (u cos - w sin, u sin + w cos),
+ * the pair being dimensions (2i, 2i+1) (RA_ROPE_INTERLEAVED) or (i, i + d/2)
+ * (RA_ROPE_HALF).  dst[b,h,s,:] = RoPE(src[b,h,t(s),:], t(s)), with t(s) the
+ * token held by layout slot s (as ra_partition, inverse = 0).  Apply it to q
+ * and k; v goes through ra_partition.  The same result as striping the
+ * position ids first and rotating in layout order.
+ *
+ *   src, dst  device bf16 [B, H, N, d], 16-byte aligned, not overlapping
+ *             (RA_ERR_ALIAS).
+ *   d         a multiple of 16, 16 <= d <= 512 (else RA_ERR_HEADDIM).
+ *   base      RoPE base (e.g. 10000), finite and > 1 (else RA_ERR_ROPE).
+ *   pairing   RA_ROPE_INTERLEAVED or RA_ROPE_HALF (else RA_ERR_ROPE).
+ * Angles are evaluated in double precision, the rotation in fp32, and the
+ * result is rounded to bf16 once (within one bf16 rounding of the exact
+ * value).  RA_CONTIGUOUS applies the rotation without moving rows.
+ */
+ra_status ra_partition_rope(const void* src, void* dst, int64_t B, int64_t H, int64_t N,
+                            int64_t d, int P, int layout, int pairing, float base, void* stream);
 
 /*
  * ra_attn_fwd -- exact blockwise attention forward over P virtual shards.

@@ -1,5 +1,6 @@
 // C-ABI entry points of libringattn.so: host-side validation, then a launch
 // on the caller's stream.  Declarations and contracts: include/ringattn.h.
+#include <cmath>
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -82,6 +83,7 @@ const char* ra_status_string(ra_status s) {
     case RA_ERR_CUDA: return "a CUDA runtime/driver call failed";
     case RA_ERR_DEVICE: return "current device is not an sm_100 GPU";
     case RA_ERR_DEVICE_FAULT: return "a kernel gave up a bounded wait; outputs incomplete";
+    case RA_ERR_ROPE: return "unknown RoPE pairing, or RoPE base not finite and > 1";
     case RA_ERR_SCRATCH:
       return "B*H*N exceeds the built-in scratch of ra_attn_bwd_noalloc (1048576 rows); "
              "use ra_attn_bwd with a workspace";
@@ -114,6 +116,27 @@ ra_status ra_partition(const void* src, void* dst, int64_t B, int64_t H, int64_t
   if (st) return st;
   return partition_launch(src, dst, B * H, N, P, row_bytes, layout == RA_STRIPED, inverse != 0,
                           stream);
+}
+
+ra_status ra_partition_rope(const void* src, void* dst, int64_t B, int64_t H, int64_t N,
+                            int64_t d, int P, int layout, int pairing, float base, void* stream) {
+  if (!src || !dst) return RA_ERR_NULL;
+  if (layout != RA_CONTIGUOUS && layout != RA_STRIPED) return RA_ERR_LAYOUT;
+  if (d < 16 || d > 512 || d % 16 != 0) return RA_ERR_HEADDIM;
+  if (B < 1 || H < 1 || N < 1 || P < 1 || N % P != 0) return RA_ERR_SHAPE;
+  if (B * H * N >= ((int64_t)1 << 31)) return RA_ERR_SHAPE;
+  if (pairing != RA_ROPE_INTERLEAVED && pairing != RA_ROPE_HALF) return RA_ERR_ROPE;
+  if (!(base > 1.f) || !isfinite(base)) return RA_ERR_ROPE;
+  if (!aligned(src, 16) || !aligned(dst, 16)) return RA_ERR_ALIGN;
+  const int64_t bytes = B * H * N * d * 2;
+  if (overlap(src, bytes, dst, bytes)) return RA_ERR_ALIAS;
+  int dev;
+  DevInfo info;
+  ra_status st = current_device(&dev, &info);
+  if (st) return st;
+  return partition_rope_launch(src, dst, B * H, N, P, d, layout == RA_STRIPED,
+                               pairing == RA_ROPE_HALF, std::log2((double)base), info.num_sms,
+                               stream);
 }
 
 ra_status ra_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,

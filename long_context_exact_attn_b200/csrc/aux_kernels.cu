@@ -81,6 +81,88 @@ ra_status partition_launch(const void* src, void* dst, int64_t rows_outer, int64
                                      stream);
 }
 
+// --------------------------------------------------- partition with RoPE
+// dst[bh, s(t), :] = RoPE(src[bh, t, :]) at position t, in layout order
+// (Striped review, 位置编码处理: the position encoding sees the same stripe as
+// the tokens).  RoPE as in RoFormer: pair i turns by t * base^(-2i/d); the
+// pairs are dimensions (2i, 2i+1) (interleaved) or (i, i + d/2) (half).
+// One thread owns one chunk of one token row and walks all (b, h), so the
+// angles are computed once per (token, pair): in double precision (the
+// angle reaches N radians), rotated in fp32, rounded to bf16 once.
+template <int HALF>
+__global__ void partition_rope_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                      int BH, int N, int P, int c, int striped, int d,
+                                      double log2_base) {
+  constexpr int kPairs = HALF ? 8 : 4;       // rotation pairs per work chunk
+  const int u16 = d / 8;                     // 16-byte units per row
+  const int cpr = HALF ? d / 16 : d / 8;     // work chunks per row
+  const long long total = (long long)N * cpr;
+  for (long long w = (long long)blockIdx.x * blockDim.x + threadIdx.x; w < total;
+       w += (long long)gridDim.x * blockDim.x) {
+    const int t = (int)(w / cpr), ch = (int)(w % cpr);
+    const int s = striped ? (t % P) * c + t / P : t;
+    float cs[kPairs], sn[kPairs];
+#pragma unroll
+    for (int k = 0; k < kPairs; ++k) {
+      const int i = ch * kPairs + k;
+      const double ang = (double)t * exp2(-(2.0 * i / d) * log2_base);
+      double sd, cd;
+      sincos(ang, &sd, &cd);
+      cs[k] = (float)cd;
+      sn[k] = (float)sd;
+    }
+#pragma unroll 4
+    for (int bh = 0; bh < BH; ++bh) {
+      const uint4* in = src + ((size_t)bh * N + t) * u16;
+      uint4* out = dst + ((size_t)bh * N + s) * u16;
+      if (HALF) {
+        uint4 a = in[ch], b = in[ch + u16 / 2];
+        __nv_bfloat162* a2 = reinterpret_cast<__nv_bfloat162*>(&a);
+        __nv_bfloat162* b2 = reinterpret_cast<__nv_bfloat162*>(&b);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 u = __bfloat1622float2(a2[j]), v = __bfloat1622float2(b2[j]);
+          const float c0 = cs[2 * j], s0 = sn[2 * j], c1 = cs[2 * j + 1], s1 = sn[2 * j + 1];
+          a2[j] = __floats2bfloat162_rn(fmaf(u.x, c0, -v.x * s0), fmaf(u.y, c1, -v.y * s1));
+          b2[j] = __floats2bfloat162_rn(fmaf(u.x, s0, v.x * c0), fmaf(u.y, s1, v.y * c1));
+        }
+        out[ch] = a;
+        out[ch + u16 / 2] = b;
+      } else {
+        uint4 a = in[ch];
+        __nv_bfloat162* a2 = reinterpret_cast<__nv_bfloat162*>(&a);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 u = __bfloat1622float2(a2[j]);
+          a2[j] = __floats2bfloat162_rn(fmaf(u.x, cs[j], -u.y * sn[j]),
+                                        fmaf(u.x, sn[j], u.y * cs[j]));
+        }
+        out[ch] = a;
+      }
+    }
+  }
+}
+
+ra_status partition_rope_launch(const void* src, void* dst, int64_t BH, int64_t N, int64_t P,
+                                int64_t d, int striped, int half, double log2_base, int num_sms,
+                                void* stream) {
+  const long long cpr = half ? d / 16 : d / 8;
+  const long long total = N * cpr;
+  if (total == 0) return RA_OK;
+  long long blocks = (total + 255) / 256;
+  if (blocks > (long long)num_sms * 8) blocks = (long long)num_sms * 8;
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+  uint4* t = reinterpret_cast<uint4*>(dst);
+  cudaStream_t st = (cudaStream_t)stream;
+  if (half)
+    partition_rope_kernel<1><<<(int)blocks, 256, 0, st>>>(s, t, (int)BH, (int)N, (int)P,
+                                                           (int)(N / P), striped, (int)d, log2_base);
+  else
+    partition_rope_kernel<0><<<(int)blocks, 256, 0, st>>>(s, t, (int)BH, (int)N, (int)P,
+                                                           (int)(N / P), striped, (int)d, log2_base);
+  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
 // -------------------------------------------------------------- lse merge
 // One warp per row: every lane reads both lse values before lane 0 writes
 // lse_out (which may alias lse_a); each 8-element chunk of o is read and

@@ -64,6 +64,9 @@ ra_status wait_selftest_launch(int64_t limit_ns, void* stream);
 ra_status partition_launch(const void* src, void* dst, int64_t rows_outer, int64_t N, int64_t P,
                            int64_t row_bytes, int striped, int inverse, void* stream);
 
+ra_status partition_rope_launch(const void* src, void* dst, int64_t BH, int64_t N, int64_t P,
+                                int64_t d, int striped, int half, double log2_base, int num_sms,
+                                void* stream);
 ra_status lse_merge_launch(const void* o_a, const float* lse_a, const void* o_b,
                            const float* lse_b, void* o_out, float* lse_out, int64_t rows,
                            int64_t d, int num_sms, void* stream);

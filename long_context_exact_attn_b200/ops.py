@@ -54,6 +54,8 @@ def lib():
         L.ra_attn_bwd.restype = i32
         L.ra_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i32,
                                   i32, i32, f32, vp]
+        L.ra_partition_rope.restype = i32
+        L.ra_partition_rope.argtypes = [vp, vp, i64, i64, i64, i64, i32, i32, i32, f32, vp]
         L.ra_attn_bwd_noalloc.restype = i32
         L.ra_attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64,
                                           i32, i32, i32, f32, vp]
@@ -178,6 +180,23 @@ def attn_bwd(q, k, v, o, dout, lse, P, layout, causal=True, scale=None, workspac
                              _ptr(dk), _ptr(dv), _ptr(workspace), B, H, N, d, int(P), int(layout),
                              int(bool(causal)), float(scale), _stream(q)), "ra_attn_bwd")
     return dq, dk, dv
+
+
+ROPE_INTERLEAVED, ROPE_HALF = 0, 1
+
+
+def partition_rope(x, P, layout, base=10000.0, pairing=ROPE_INTERLEAVED, out=None):
+    """Token order -> layout order of q or k [B, H, N, d] (bf16) with rotary
+    position embedding applied at the original token positions."""
+    _cuda_contig(x, "x")
+    if x.dim() != 4 or x.dtype != torch.bfloat16:
+        raise ValueError("x must be bfloat16 [B, H, N, d]")
+    B, H, N, d = x.shape
+    out = torch.empty_like(x) if out is None else out
+    _cuda_contig(out, "out")
+    _check(lib().ra_partition_rope(_ptr(x), _ptr(out), B, H, N, d, int(P), int(layout),
+                                   int(pairing), float(base), _stream(x)), "ra_partition_rope")
+    return out
 
 
 def attn_bwd_noalloc(q, k, v, o, dout, lse, P, layout, causal, scale, dq, dk, dv):

@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(L):
 
 def test_status_strings(L):
     assert ops.status_string(0) == "ok"
-    for code in range(1, 13):
+    for code in range(1, 14):
         assert ops.status_string(code) not in ("", "unknown status")
     assert ops.status_string(999) == "unknown status"
     assert L.ra_version() >= 100
@@ -138,3 +138,17 @@ def bwd_noalloc(L, q=A, k=Bp, v=Cp, o=Op, do=6 << 40, lse=Lp, dq=7 << 40, dk=8 <
 ])
 def test_attn_bwd_noalloc_rejects_invalid_arguments(L, kw, code):
     assert bwd_noalloc(L, **kw) == code
+
+
+def prope(L, src=A, dst=Bp, B=1, H=2, N=1024, d=128, P=4, layout=1, pairing=0, base=10000.0):
+    return L.ra_partition_rope(vp(src), vp(dst), B, H, N, d, P, layout, pairing, base, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(src=0), 1), (dict(dst=A + 16), 8), (dict(dst=Bp + 8), 2), (dict(N=1000, P=3), 3),
+    (dict(d=72), 4), (dict(d=8), 4), (dict(d=1024), 4), (dict(layout=2), 5),
+    (dict(pairing=2), 13), (dict(base=1.0), 13), (dict(base=float("inf")), 13),
+    (dict(base=float("nan")), 13), (dict(B=0), 3),
+])
+def test_partition_rope_rejects_invalid_arguments(L, kw, code):
+    assert prope(L, **kw) == code
