@@ -85,3 +85,57 @@ def ring_attention(q, k, v, P, layout, causal, scale, normalise_each_round=False
         out[j * c:(j + 1) * c] = o
         lse_out[j * c:(j + 1) * c] = m + np.log(l)
     return out, lse_out
+
+
+def block_attention(qj, kb_k, kb_v, j, kb, P, layout, causal, scale):
+    """One round of one device: query block j against key/value block kb,
+    normalised over that block alone.
+
+    Returns (O_r [c, dv], lse_r [c]); a row that sees no key of the block
+    (GetMask hides all of them) gets O_r = 0, lse_r = -inf, so that it
+    contributes nothing when merged (1cademy page, per-node partial sums;
+    the pages are silent on empty rows).
+    """
+    qj = np.asarray(qj, dtype=np.float64)
+    kk = np.asarray(kb_k, dtype=np.float64)
+    vv = np.asarray(kb_v, dtype=np.float64)
+    c = qj.shape[0]
+    s = (qj @ kk.T) * float(scale)
+    if causal:
+        s = np.where(getmask(j, kb, c, layout).T, -np.inf, s)
+    mx = np.max(s, axis=1)
+    empty = np.isneginf(mx)
+    e = np.exp(s - np.where(empty, 0.0, mx)[:, None])
+    den = np.sum(e, axis=1)
+    with np.errstate(invalid="ignore", divide="ignore"):
+        o = np.where(empty[:, None], 0.0, (e @ vv) / den[:, None])
+        lse = np.where(empty, -np.inf, mx + np.log(den))
+    return o, lse
+
+
+def ring_by_merge(q, k, v, P, layout, causal, scale):
+    """The ring with per-round partial results merged through their
+    normalisers (1cademy page, "Computing Attention Weights in Sequence
+    Parallelism") instead of an online-softmax state: device j merges
+    block_attention(j, (j - r) mod P) for r = 0..P-1.  Layout order in and
+    out, as ``ring_attention``."""
+    from .merge import lse_merge
+
+    q = np.asarray(q, dtype=np.float64)
+    N = q.shape[0]
+    c = shard_len(N, P)
+    out = np.empty((N, np.asarray(v).shape[1]))
+    lse_out = np.empty(N)
+    for j in range(P):
+        o_acc, l_acc = None, None
+        for r in range(P):
+            kb = (j - r) % P
+            o_r, l_r = block_attention(q[j * c:(j + 1) * c], k[kb * c:(kb + 1) * c],
+                                       v[kb * c:(kb + 1) * c], j, kb, P, layout, causal, scale)
+            if o_acc is None:
+                o_acc, l_acc = o_r, l_r
+            else:
+                o_acc, l_acc = lse_merge(o_acc, l_acc, o_r, l_r)
+        out[j * c:(j + 1) * c] = o_acc
+        lse_out[j * c:(j + 1) * c] = l_acc
+    return out, lse_out

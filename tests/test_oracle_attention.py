@@ -197,3 +197,46 @@ def test_lse_merge_empty_sides():
     om, lm = merge.lse_merge(zero, ninf, zero, ninf)
     np.testing.assert_array_equal(om, zero)
     assert np.all(np.isneginf(lm))
+
+
+@pytest.mark.parametrize("layout", [CONTIGUOUS, STRIPED])
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("N,P", [(16, 1), (24, 4), (30, 5), (16, 16)])
+def test_ring_by_merging_round_partials_equals_full_softmax(layout, causal, N, P):
+    """Per-round partial results merged through their normalisers (1cademy
+    page: the denominator is a sum of per-node partial sums) reach the plain
+    result, including rounds in which a row sees no key (N = P: one row per
+    shard)."""
+    q, k, v = rand_qkv(N, 8, 3 * N + P, dv=5)
+    q, k = 3 * q, 3 * k
+    scale = 8 ** -0.5
+    o_ref, lse_ref = att.attention(q, k, v, scale, causal)
+    qp, kp, vp = (partition.partition(a, P, layout, axis=0) for a in (q, k, v))
+    o, lse = ring.ring_by_merge(qp, kp, vp, P, layout, causal, scale)
+    np.testing.assert_allclose(partition.unpartition(o, P, layout, axis=0), o_ref, atol=1e-12)
+    np.testing.assert_allclose(partition.unpartition(lse, P, layout, axis=0), lse_ref, atol=1e-12)
+
+
+def test_block_attention_empty_rows_and_positions():
+    """A round's partial equals the plain definition over the block's keys
+    with the original positions; rows that see none of them are (0, -inf)."""
+    N, P = 20, 4
+    c = N // P
+    q, k, v = rand_qkv(N, 6, 5)
+    for layout in (CONTIGUOUS, STRIPED):
+        toks = partition.shard_tokens(N, P, layout)
+        qp, kp, vp = (partition.partition(a, P, layout, axis=0) for a in (q, k, v))
+        for j in range(P):
+            for kb in range(P):
+                o, lse = ring.block_attention(qp[j * c:(j + 1) * c], kp[kb * c:(kb + 1) * c],
+                                              vp[kb * c:(kb + 1) * c], j, kb, P, layout, True, 0.4)
+                for x in range(c):
+                    vis = [y for y in range(c) if toks[kb][y] <= toks[j][x]]
+                    if not vis:
+                        assert lse[x] == -np.inf and np.all(o[x] == 0)
+                        continue
+                    s = np.array([q[toks[j][x]] @ k[toks[kb][y]] * 0.4 for y in vis])
+                    w = np.exp(s - s.max())
+                    ref_o = (w / w.sum()) @ np.array([v[toks[kb][y]] for y in vis])
+                    np.testing.assert_allclose(o[x], ref_o, atol=1e-12)
+                    np.testing.assert_allclose(lse[x], s.max() + np.log(w.sum()), atol=1e-12)
