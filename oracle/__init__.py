@@ -18,7 +18,9 @@ source pages:
   and the same masks derived from global token positions.
 * ``ring``         -- the method itself, restated step by step: Q block fixed,
   KV blocks visiting in ring order, online-softmax fold per round (Ring
-  Attention explainer ステップ2/ステップ3 and its 実装例).
+  Attention explainer ステップ2/ステップ3 and its 実装例); one device's
+  per-round partial (``block_attention``) and the ring restated as a merge
+  of those partials (``ring_by_merge``, 1cademy page).
 * ``work``         -- the per-device/per-round work formulas (Striped review,
   Ring Attention 工作负载 / Striped Attention 工作负载) and brute-force counts.
 * ``backward``     -- gradients dQ, dK, dV of the definition (the pages give
