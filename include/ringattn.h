@@ -228,6 +228,53 @@ ra_status ra_attn_bwd_noalloc(const void* q, const void* k, const void* v, const
                               int causal, float scale, void* stream);
 
 /*
+ * ra_attn_fwd_block -- one round of one device of the ring: query shard j
+ * against key/value block kb, normalised over that block alone.
+ *
+ * The physical ring (Ring explainer ステップ2 and its 実装例: each device keeps
+ * its Q block, sends its K/V block to rank+1 and receives from rank-1, so in
+ * round r device j holds block (j - r) mod P) computes, every round, the
+ * attention of its query block against the block it holds, and the rounds
+ * are combined through their softmax normalisers (1cademy page "Computing
+ * Attention Weights in Sequence Parallelism": the denominator is a sum of
+ * per-node partial sums).  This is that per-round computation with the
+ * GetMask of the pair (j, kb) (Striped review, GetMask 函数); combine rounds
+ * with ra_lse_merge_acc.
+ *
+ *   q         device bf16 [B, H, c, d]: query shard j in layout order.
+ *   k, v      device bf16 [B, H, c, d]: key/value block kb in layout order.
+ *   o, lse    outputs: bf16 [B, H, c, d] and float32 [B, H, c].  A query row
+ *             that sees no key of the block gets o = 0, lse = -inf.
+ *   j, kb, P  0 <= j, kb < P: the pair's shard indices (masks only).
+ *   d         64 or 128; c = N / P >= 1.
+ * Same tile skipping and precision as ra_attn_fwd.  Errors as ra_attn_fwd.
+ */
+ra_status ra_attn_fwd_block(const void* q, const void* k, const void* v, void* o, float* lse,
+                            int64_t B, int64_t H, int64_t c, int64_t d, int j, int kb, int P,
+                            int layout, int causal, float scale, void* stream);
+
+/* Modes of ra_lse_merge_acc (OR-ed). */
+#define RA_MERGE_FIRST 1     /* accumulator not yet set: it becomes the partial */
+#define RA_MERGE_FINAL 2     /* also write the merged O as bf16 to o_final      */
+
+/*
+ * ra_lse_merge_acc -- fold a bf16 partial result into a float32 accumulator
+ * (the same merge as ra_lse_merge; 1cademy page "Computing Attention Weights
+ * in Sequence Parallelism"), so that P rounds round to bf16 once.
+ *
+ *   o_acc, lse_acc   device float32 [rows, d] and [rows], read and written.
+ *   o_b, lse_b       device bf16 [rows, d] and float32 [rows]: the partial.
+ *   o_final          device bf16 [rows, d], written when mode has
+ *                    RA_MERGE_FINAL (may be NULL otherwise).
+ *   d                a multiple of 8.
+ * No buffer may overlap another (RA_ERR_ALIAS); o_acc, o_b, o_final 16-byte
+ * aligned.  Unknown mode bits: RA_ERR_LAYOUT.  Empty sides (lse = -inf)
+ * contribute nothing; both empty give o = 0, lse = -inf.
+ */
+ra_status ra_lse_merge_acc(float* o_acc, float* lse_acc, const void* o_b, const float* lse_b,
+                           void* o_final, int64_t rows, int64_t d, int mode, void* stream);
+
+/*
  * ra_lse_merge -- merge two partial attention results over disjoint key sets.
  *
  * From the split of the softmax denominator into per-node partial sums

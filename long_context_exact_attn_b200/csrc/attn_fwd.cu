@@ -56,6 +56,10 @@ struct AttnParams {
   int ctas_per_group;
   float c2;           // scale * log2(e)
   unsigned long long timeout_ns;
+  // Single-block mode (blk_kb >= 0): Q is one query shard, K/V one key
+  // block (both stored as shard 0 of a P = 1 tensor); the mask is the
+  // GetMask of the real pair (blk_j, blk_kb).
+  int blk_j, blk_kb;
 };
 
 template <int D>
@@ -119,7 +123,7 @@ __device__ __forceinline__ bool cta_item(const AttnParams& p, int k, Item& it) {
 // query tiles' FULL / PARTIAL / SKIP thresholds are computed once; per tile
 // the classification is two compares each.
 struct TileSeq {
-  int j, P, c, striped, causal;
+  int j, P, c, striped, causal, blk_j, blk_kb;
   int x0;                   // first row of query tile 0
   int r, kt, kend;
   TileSpan s0, s1;
@@ -128,6 +132,7 @@ struct TileSeq {
 
   __device__ __forceinline__ void init(const AttnParams& p, const Item& it) {
     j = it.j; P = p.P; c = p.c; striped = p.striped; causal = p.causal;
+    blk_j = p.blk_j; blk_kb = p.blk_kb;
     x0 = it.pair * 2 * kBM;
     r = -1; kt = 0; kend = 0;
   }
@@ -136,8 +141,13 @@ struct TileSeq {
   __device__ __forceinline__ bool next(int& kb_out, int& y0, int& k0, int& k1, BlockMask& m) {
     while (kt >= kend) {
       if (++r >= P) return false;
-      kb = key_block(j, r, P);
-      bm = block_mask(j, kb, striped, causal);
+      if (blk_kb >= 0) {
+        kb = 0;
+        bm = block_mask(blk_j, blk_kb, striped, causal);
+      } else {
+        kb = key_block(j, r, P);
+        bm = block_mask(j, kb, striped, causal);
+      }
       s0 = tile_span(bm, x0, c);
       s1 = tile_span(bm, x0 + kBM, c);
       kend = s0.part_end > s1.part_end ? s0.part_end : s1.part_end;
@@ -396,6 +406,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const uint32_t full0 = bars + 2 * 8, empty0 = bars + (2 + C::kSlots) * 8;
       uint32_t slot = 0, phase = 0;       // next K/V tile to consume, in producer order
       uint32_t pc0 = 0, pc1 = 0;          // p_full phases consumed per query tile
+      // o_free phases consumed per query tile.  The waits catch up one phase
+      // at a time: a parity wait is only unambiguous one phase ahead, and a
+      // query tile without key tiles in an item skips its lazy wait.
+      uint32_t of0 = 0, of1 = 0;
       Item it;
       bool ok = true;
       for (int k = 0; ok && cta_item(p, k, it); ++k) {
@@ -406,6 +420,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         BlockMask bm;
         uint32_t acc0 = 0, acc1 = 0;
         bool have = seq.next(kb, y0, c0, c1, bm);
+        if (!have) {
+          // no visible key tile for either query tile (only possible for a
+          // single block): release the item without touching O, once the
+          // previous item's epilogue has passed (keeps o_full one phase ahead
+          // of the softmax warps at most)
+          bool okw = true;
+          while (okw && of0 < (uint32_t)k) okw = wmbar_wait(o_free0, of0++ & 1, abort_flag, p.timeout_ns);
+          while (okw && of1 < (uint32_t)k) okw = wmbar_wait(o_free1, of1++ & 1, abort_flag, p.timeout_ns);
+          if (!okw) { ok = false; break; }
+          mma_commit_w(bar_o_full + 0);
+          mma_commit_w(bar_o_full + 8);
+          mma_commit_w(bar_q_empty);
+          continue;
+        }
         // prologue: Q K^T of the first tile
         uint32_t kslot = slot;
         if (!wmbar_wait(full0 + 8 * kslot, phase, abort_flag, p.timeout_ns)) { ok = false; break; }
@@ -430,9 +458,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           const uint32_t nka = sRing + nkslot * C::kTileBytes;
           // query tile 0: P0 V, then the next Q0 K^T into the freed S0/P0 columns
           if (c0 != TILE_SKIP) {
-            if (acc0 == 0 && k > 0 && !wmbar_wait(o_free0, (k - 1) & 1, abort_flag, p.timeout_ns)) {
-              ok = false; break;
-            }
+            bool okw = true;
+            while (okw && of0 < (uint32_t)k) okw = wmbar_wait(o_free0, of0++ & 1, abort_flag, p.timeout_ns);
+            if (!okw) { ok = false; break; }
             // P in two halves: the first 4 k-steps (keys 0-63) start while the
             // softmax is still producing keys 64-127.
             if (!wmbar_wait(p_full0, pc0 & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
@@ -447,9 +475,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           if (more && n0 != TILE_SKIP) { tc_fence_after(); mma_qk<D>(tS0, sQ0, nka); mma_commit_w(s_full0); }
           // query tile 1
           if (c1 != TILE_SKIP) {
-            if (acc1 == 0 && k > 0 && !wmbar_wait(o_free1, (k - 1) & 1, abort_flag, p.timeout_ns)) {
-              ok = false; break;
-            }
+            bool okw = true;
+            while (okw && of1 < (uint32_t)k) okw = wmbar_wait(o_free1, of1++ & 1, abort_flag, p.timeout_ns);
+            if (!okw) { ok = false; break; }
             // P in two halves: the first 4 k-steps (keys 0-63) start while the
             // softmax is still producing keys 64-127.
             if (!wmbar_wait(p_full1, pc1 & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
@@ -469,6 +497,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           c1 = n1;
         }
         if (!ok) break;
+        {
+          bool okw = true;
+          while (okw && of0 < (uint32_t)k) okw = wmbar_wait(o_free0, of0++ & 1, abort_flag, p.timeout_ns);
+          while (okw && of1 < (uint32_t)k) okw = wmbar_wait(o_free1, of1++ & 1, abort_flag, p.timeout_ns);
+          if (!okw) { ok = false; break; }
+        }
         mma_commit_w(bar_o_full + 0);
         mma_commit_w(bar_o_full + 8);
         mma_commit_w(bar_q_empty);
@@ -619,7 +653,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (!mbar_wait(my_o_full, k & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
       tc_fence_after();
       const bool valid = x < p.c;
-      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      // a row that saw no key (possible only for a single block) gets O = 0
+      // and lse = -inf; its O columns in TMEM were never written
+      const float inv_l = (acc && l > 0.f) ? 1.f / l : 0.f;
       const size_t grow = (size_t)it.bh * p.N + (size_t)it.j * p.c + (size_t)(valid ? x : 0);
       __nv_bfloat16* orow_g = p.o + grow * D;
 #pragma unroll 1
@@ -627,6 +663,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         uint32_t orow[32];
         tmem_ld32(tO + q * 32, orow);
         tmem_wait_ld();
+        if (!acc) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) orow[i] = 0u;
+        }
         if (valid) {
           uint32_t w[16];
 #pragma unroll
@@ -639,7 +679,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
         }
       }
-      if (valid) p.lse[grow] = (m2 + __log2f(l)) * 0.69314718055994530942f;
+      if (valid) p.lse[grow] = (acc && l > 0.f) ? (m2 + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(my_o_free);
@@ -700,6 +740,8 @@ static ra_status launch(const AttnLaunch& a) {
   p.causal = a.causal;
   p.c2 = (float)((double)a.scale * 1.4426950408889634074);
   p.timeout_ns = 2000000000ull;
+  p.blk_j = a.blk_j;
+  p.blk_kb = a.blk_kb;
   const long long items_total = (long long)p.npairs * a.P * a.BH;
   int grid;
   if (a.sched_free) {

@@ -222,6 +222,94 @@ ra_status lse_merge_launch(const void* o_a, const float* lse_a, const void* o_b,
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
+// ------------------------------------------------ merge into an accumulator
+// (O_acc, lse_acc) <- merge of (O_acc, lse_acc) and a bf16 partial (O_b,
+// lse_b) through their normalisers (1cademy page "Computing Attention
+// Weights in Sequence Parallelism"), with O_acc kept in fp32 so that P
+// rounds round to bf16 only once.  first: the accumulator is not yet set
+// (it becomes the partial).  final: also write O_acc as bf16 to o_final.
+// Both sides empty (lse = -inf) give O = 0, lse = -inf.
+__global__ void lse_merge_acc_kernel(float* __restrict__ oacc, float* __restrict__ lacc,
+                                     const uint4* __restrict__ ob, const float* __restrict__ lb_,
+                                     uint4* __restrict__ ofin, long long rows, int chunks,
+                                     int first, int final_) {
+  const int lane = threadIdx.x & 31;
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long r = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows;
+       r += warps) {
+    const float lb = lb_[r];
+    const float la = first ? -INFINITY : lacc[r];
+    const float mx = fmaxf(la, lb);
+    float wa = 0.f, wb = 0.f, lse = -INFINITY;
+    if (mx != -INFINITY) {
+      const float ea = expf(la - mx);
+      const float eb = expf(lb - mx);
+      const float sum = ea + eb;
+      wa = ea / sum;
+      wb = eb / sum;
+      lse = mx + logf(sum);
+    }
+    __syncwarp();
+    for (int ch = lane; ch < chunks; ch += 32) {
+      const size_t idx = (size_t)r * chunks + ch;
+      const uint4 b = ob[idx];
+      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+      float4* a4 = reinterpret_cast<float4*>(oacc) + idx * 2;
+      float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+      if (!first) {
+        a0 = a4[0];
+        a1 = a4[1];
+      }
+      const float2 b0 = __bfloat1622float2(b2[0]), b1 = __bfloat1622float2(b2[1]);
+      const float2 b2v = __bfloat1622float2(b2[2]), b3 = __bfloat1622float2(b2[3]);
+      a0 = make_float4(wa * a0.x + wb * b0.x, wa * a0.y + wb * b0.y, wa * a0.z + wb * b1.x,
+                       wa * a0.w + wb * b1.y);
+      a1 = make_float4(wa * a1.x + wb * b2v.x, wa * a1.y + wb * b2v.y, wa * a1.z + wb * b3.x,
+                       wa * a1.w + wb * b3.y);
+      a4[0] = a0;
+      a4[1] = a1;
+      if (final_) {
+        uint4 out;
+        __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(&out);
+        o2[0] = __floats2bfloat162_rn(a0.x, a0.y);
+        o2[1] = __floats2bfloat162_rn(a0.z, a0.w);
+        o2[2] = __floats2bfloat162_rn(a1.x, a1.y);
+        o2[3] = __floats2bfloat162_rn(a1.z, a1.w);
+        ofin[idx] = out;
+      }
+    }
+    if (lane == 0) lacc[r] = lse;
+    __syncwarp();
+  }
+}
+
+ra_status lse_merge_acc_launch(float* o_acc, float* lse_acc, const void* o_b,
+                               const float* lse_b, void* o_final, int64_t rows, int64_t d,
+                               int first, int final_, void* stream) {
+  if (rows == 0) return RA_OK;
+  const int chunks = (int)(d / 8);
+  long long blocks = (rows + 7) / 8;
+  if (blocks > 148LL * 16) blocks = 148LL * 16;
+  lse_merge_acc_kernel<<<(int)blocks, 256, 0, (cudaStream_t)stream>>>(
+      o_acc, lse_acc, reinterpret_cast<const uint4*>(o_b), lse_b, reinterpret_cast<uint4*>(o_final),
+      (long long)rows, chunks, first, final_);
+  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
+__global__ void fill_f32_kernel(float* __restrict__ dst, long long n, float value) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x)
+    dst[i] = value;
+}
+
+ra_status fill_f32_launch(float* dst, int64_t n, float value, void* stream) {
+  if (n == 0) return RA_OK;
+  long long blocks = (n + 255) / 256;
+  if (blocks > 148LL * 8) blocks = 148LL * 8;
+  fill_f32_kernel<<<(int)blocks, 256, 0, (cudaStream_t)stream>>>(dst, (long long)n, value);
+  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
 // ------------------------------------------------------------ tile census
 // One thread per (query shard j, round r, query tile qt); classification and
 // per-row limits are the attention kernel's own (ra_tiles.cuh).

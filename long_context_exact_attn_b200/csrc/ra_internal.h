@@ -29,6 +29,7 @@ struct AttnLaunch {
   float scale;
   int device, num_sms;
   void* stream;
+  int blk_j = -1, blk_kb = -1;   // single-block mode when blk_kb >= 0 (P = 1)
 };
 
 ra_status attn_fwd_launch(const AttnLaunch& a);
@@ -67,6 +68,10 @@ ra_status partition_launch(const void* src, void* dst, int64_t rows_outer, int64
 ra_status partition_rope_launch(const void* src, void* dst, int64_t BH, int64_t N, int64_t P,
                                 int64_t d, int striped, int half, double log2_base, int num_sms,
                                 void* stream);
+ra_status lse_merge_acc_launch(float* o_acc, float* lse_acc, const void* o_b,
+                               const float* lse_b, void* o_final, int64_t rows, int64_t d,
+                               int first, int final_, void* stream);
+ra_status fill_f32_launch(float* dst, int64_t n, float value, void* stream);
 ra_status lse_merge_launch(const void* o_a, const float* lse_a, const void* o_b,
                            const float* lse_b, void* o_out, float* lse_out, int64_t rows,
                            int64_t d, int num_sms, void* stream);

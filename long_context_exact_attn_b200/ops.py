@@ -54,6 +54,11 @@ def lib():
         L.ra_attn_bwd.restype = i32
         L.ra_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i32,
                                   i32, i32, f32, vp]
+        L.ra_attn_fwd_block.restype = i32
+        L.ra_attn_fwd_block.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, i32, i32,
+                                        i32, i32, f32, vp]
+        L.ra_lse_merge_acc.restype = i32
+        L.ra_lse_merge_acc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, vp]
         L.ra_partition_rope.restype = i32
         L.ra_partition_rope.argtypes = [vp, vp, i64, i64, i64, i64, i32, i32, i32, f32, vp]
         L.ra_attn_bwd_noalloc.restype = i32
@@ -180,6 +185,53 @@ def attn_bwd(q, k, v, o, dout, lse, P, layout, causal=True, scale=None, workspac
                              _ptr(dk), _ptr(dv), _ptr(workspace), B, H, N, d, int(P), int(layout),
                              int(bool(causal)), float(scale), _stream(q)), "ra_attn_bwd")
     return dq, dk, dv
+
+
+def attn_fwd_block(q, k, v, j, kb, P, layout, causal=True, scale=None, out=None, lse=None):
+    """One round of the ring on this device: query shard j [B, H, c, d]
+    against key/value block kb [B, H, c, d] (layout order), normalised over
+    the block; rows that see no key of it get o = 0, lse = -inf."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _cuda_contig(t, n)
+        if t.dtype != torch.bfloat16 or t.dim() != 4 or t.shape != q.shape:
+            raise ValueError(f"{n} must be bfloat16 [B, H, c, d] like q")
+    B, H, c, d = q.shape
+    if scale is None:
+        scale = d ** -0.5
+    o = torch.empty_like(q) if out is None else out
+    lse = torch.empty(B, H, c, dtype=torch.float32, device=q.device) if lse is None else lse
+    _cuda_contig(o, "out")
+    _cuda_contig(lse, "lse")
+    _check(lib().ra_attn_fwd_block(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, c, d,
+                                   int(j), int(kb), int(P), int(layout), int(bool(causal)),
+                                   float(scale), _stream(q)), "ra_attn_fwd_block")
+    return o, lse
+
+
+MERGE_FIRST, MERGE_FINAL = 1, 2
+
+
+def lse_merge_acc(o_acc, lse_acc, o_b, lse_b, first=False, final_out=None):
+    """Fold a bf16 partial (o_b, lse_b) into the float32 accumulator
+    (o_acc, lse_acc) in place; with ``final_out`` also write the merged O as
+    bf16 there."""
+    d = o_b.shape[-1]
+    rows = o_b.numel() // d
+    if o_acc.dtype != torch.float32 or o_acc.shape != o_b.shape or o_b.dtype != torch.bfloat16:
+        raise ValueError("o_acc float32 and o_b bfloat16 of the same shape")
+    if lse_acc.dtype != torch.float32 or lse_b.dtype != torch.float32 or \
+            lse_acc.numel() != rows or lse_b.numel() != rows:
+        raise ValueError("lse_acc, lse_b: float32 with one value per row")
+    for n, t in (("o_acc", o_acc), ("lse_acc", lse_acc), ("o_b", o_b), ("lse_b", lse_b)):
+        _cuda_contig(t, n)
+    mode = (MERGE_FIRST if first else 0) | (MERGE_FINAL if final_out is not None else 0)
+    fin = None
+    if final_out is not None:
+        _cuda_contig(final_out, "final_out")
+        fin = _ptr(final_out)
+    _check(lib().ra_lse_merge_acc(_ptr(o_acc), _ptr(lse_acc), _ptr(o_b), _ptr(lse_b), fin, rows,
+                                  d, mode, _stream(o_b)), "ra_lse_merge_acc")
+    return o_acc, lse_acc
 
 
 ROPE_INTERLEAVED, ROPE_HALF = 0, 1

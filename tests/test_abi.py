@@ -152,3 +152,30 @@ def prope(L, src=A, dst=Bp, B=1, H=2, N=1024, d=128, P=4, layout=1, pairing=0, b
 ])
 def test_partition_rope_rejects_invalid_arguments(L, kw, code):
     assert prope(L, **kw) == code
+
+
+def blk(L, q=A, k=Bp, v=Cp, o=Op, lse=Lp, B=1, H=2, c=256, d=128, j=1, kb=0, P=4, layout=1,
+        causal=1, scale=0.088):
+    return L.ra_attn_fwd_block(vp(q), vp(k), vp(v), vp(o), vp(lse), B, H, c, d, j, kb, P, layout,
+                               causal, scale, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(v=0), 1), (dict(o=Op + 8), 2), (dict(j=4), 3), (dict(kb=-1), 3), (dict(c=0), 3),
+    (dict(d=96), 4), (dict(layout=0x101), 5), (dict(scale=0.0), 6), (dict(o=A), 8),
+    (dict(lse=Cp + 64), 8),
+])
+def test_attn_fwd_block_rejects_invalid_arguments(L, kw, code):
+    assert blk(L, **kw) == code
+
+
+def macc(L, oa=A, la=Bp, ob=Cp, lb=Op, of=Lp, rows=256, d=128, mode=2):
+    return L.ra_lse_merge_acc(vp(oa), vp(la), vp(ob), vp(lb), vp(of), rows, d, mode, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(oa=0), 1), (dict(of=0), 1), (dict(mode=4), 5), (dict(d=12), 3), (dict(rows=-1), 3),
+    (dict(oa=A + 4), 2), (dict(ob=A + 4096), 8), (dict(of=Cp), 8),
+])
+def test_lse_merge_acc_rejects_invalid_arguments(L, kw, code):
+    assert macc(L, **kw) == code

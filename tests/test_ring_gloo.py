@@ -1,0 +1,101 @@
+"""The process ring (long_context_exact_attn_b200/ring.py) on CPU ranks over
+gloo: the K/V exchange of the Ring explainer (send to rank+1, receive from
+rank-1; block (j - r) mod P in round r) and the merge of round partials.
+
+The two device steps are the oracle's (tests may use it): the round partial
+``oracle.ring.block_attention`` and the normaliser merge
+``oracle.merge.lse_merge``, here on float64 host tensors.  Every rank checks
+that the block it holds in round r is block (j - r) mod P of the global
+tensors, and the gathered result must equal the plain definition to 1e-12.
+"""
+
+import datetime
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, layout, causal, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        from long_context_exact_attn_b200 import ring
+        from oracle import merge as OM
+        from oracle import partition as OP
+        from oracle import ring as OR
+
+        N, d, P = 6 * world, 8, world
+        c = N // P
+        g = np.random.default_rng(11)
+        q, k, v = (g.standard_normal((N, d)) * s for s in (3.0, 3.0, 1.0))
+        lay = OP.STRIPED if layout else OP.CONTIGUOUS
+        qp, kp, vp = (OP.partition(a, P, lay, axis=0) for a in (q, k, v))
+        shard = lambda a, j: torch.from_numpy(np.ascontiguousarray(a[j * c:(j + 1) * c]))[None, None]
+        seen = []
+
+        def block_fn(qt, kt, vt, j, kb, P_, layout_, causal_, scale):
+            assert np.array_equal(kt[0, 0].numpy(), kp[kb * c:(kb + 1) * c])
+            assert np.array_equal(vt[0, 0].numpy(), vp[kb * c:(kb + 1) * c])
+            seen.append(kb)
+            o, lse = OR.block_attention(qt[0, 0].numpy(), kt[0, 0].numpy(), vt[0, 0].numpy(), j,
+                                        kb, P_, lay, causal_, scale)
+            return torch.from_numpy(o)[None, None], torch.from_numpy(lse)[None, None]
+
+        def merge_fn(o_acc, lse_acc, o_r, lse_r, first=False, final_out=None):
+            if first:
+                o_acc.copy_(o_r)
+                lse_acc.copy_(lse_r)
+            else:
+                o, lse = OM.lse_merge(o_acc.numpy(), lse_acc.numpy(), o_r.numpy(), lse_r.numpy())
+                o_acc.copy_(torch.from_numpy(o))
+                lse_acc.copy_(torch.from_numpy(lse))
+            if final_out is not None:
+                final_out.copy_(o_acc)
+
+        o, lse = ring.ring_attn_fwd(shard(qp, rank).double(), shard(kp, rank).double(),
+                                    shard(vp, rank).double(), layout, causal, d ** -0.5,
+                                    block_fn=block_fn, merge_fn=merge_fn)
+        assert seen == [(rank - r) % P for r in range(P)]
+        out.put((rank, o[0, 0].numpy().copy(), lse[0, 0].numpy().copy()))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("layout,causal", [(1, True), (0, True), (1, False)])
+def test_process_ring_equals_definition(world, layout, causal):
+    from oracle import attention as OA
+    from oracle import partition as OP
+
+    ctx = mp.get_context("spawn")
+    q_ = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, layout, causal, q_))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = dict((r, (o, l)) for r, o, l in (q_.get(timeout=120) for _ in procs))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    N, d, P = 6 * world, 8, world
+    g = np.random.default_rng(11)
+    q, k, v = (g.standard_normal((N, d)) * s for s in (3.0, 3.0, 1.0))
+    lay = OP.STRIPED if layout else OP.CONTIGUOUS
+    o_ref, lse_ref = OA.attention(q, k, v, d ** -0.5, causal)
+    o = np.concatenate([res[r][0] for r in range(P)])
+    lse = np.concatenate([res[r][1] for r in range(P)])
+    np.testing.assert_allclose(OP.unpartition(o, P, lay, axis=0), o_ref, atol=1e-12)
+    np.testing.assert_allclose(OP.unpartition(lse, P, lay, axis=0), lse_ref, atol=1e-12)
