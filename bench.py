@@ -282,6 +282,8 @@ def main():
     ap.add_argument("--no-compare", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-chunks", type=int, default=8,
+                    help="head chunks of the host-buffer path (copies overlap compute)")
     ap.add_argument("--no-rope", action="store_true",
                     help="skip timing the stripe + RoPE partition of q")
     ap.add_argument("--backward", action="store_true",
@@ -339,25 +341,30 @@ def main():
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
+        # ra_attn_fwd_host: token-order host q, k, v in, host o, lse out; the
+        # heads go through a device workspace in chunks of a quarter of the
+        # heads, copies of neighbouring chunks overlapping the compute
         hq, hk, hv = (t.pin_memory() for t in (q, k, v))
         ho = torch.empty(path.o.shape, dtype=path.o.dtype).pin_memory()
         hl = torch.empty(path.lse.shape, dtype=path.lse.dtype).pin_memory()
+        g = max(1, -(-(w.B * w.H) // args.e2e_chunks))
+        wsb = ops.attn_fwd_host_workspace_bytes(w.N, w.d, path.layout, g)
+        ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
 
         def e2e_step():
-            path.q.copy_(hq, non_blocking=True)
-            path.k.copy_(hk, non_blocking=True)
-            path.v.copy_(hv, non_blocking=True)
-            path.step()
-            ho.copy_(path.o, non_blocking=True)
-            hl.copy_(path.lse, non_blocking=True)
+            ops.attn_fwd_host(hq, hk, hv, w.P, w.layout, w.causal, workspace=ws, out=ho, lse=hl,
+                              sched_free=args.sched == "free")
 
         e2e_step()
         torch.cuda.synchronize()
         e2e_ms = timed(e2e_step, max(1, min(args.steps, 5)), world)
+        del ws
+        torch.cuda.empty_cache()
         h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
         d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
         e2e = {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "api": "ra_attn_fwd_host (pinned host buffers)", "heads_per_chunk": g}
 
     # ---- the layout/schedule comparison at equal shapes (attention only)
     compare = None

@@ -65,6 +65,7 @@ typedef int ra_status;
 #define RA_ERR_SCRATCH 12    /* problem larger than the built-in scratch of    */
                              /* ra_attn_bwd_noalloc (B*H*N > 1048576)          */
 #define RA_ERR_ROPE 13       /* unknown RoPE pairing, or base not > 1 / finite */
+#define RA_ERR_WORKSPACE 14  /* device workspace too small                     */
 
 /* Layouts (low byte of `layout`). */
 #define RA_CONTIGUOUS 0      /* shard j = tokens [j*c, (j+1)*c)  (Ring)        */
@@ -226,6 +227,41 @@ ra_status ra_attn_bwd_noalloc(const void* q, const void* k, const void* v, const
                               const void* dout, const float* lse, void* dq, void* dk, void* dv,
                               int64_t B, int64_t H, int64_t N, int64_t d, int P, int layout,
                               int causal, float scale, void* stream);
+
+/*
+ * ra_attn_fwd_host -- the whole forward path from host memory: token-order
+ * q, k, v in host memory -> (partition, attention, un-partition) -> token-
+ * order o, lse in host memory.
+ *
+ * Same computation and results as ra_partition + ra_attn_fwd + ra_partition
+ * (inverse) on device copies (bit-identical: every (b, h) is computed alone).
+ * The heads are processed in chunks through two staging slots of the
+ * caller's device workspace: the host-to-device copy of chunk i+1 and the
+ * device-to-host copy of chunk i-1 run on the library's own copy streams
+ * while chunk i computes on `stream`.  Host buffers should be page-locked
+ * (pinned) for the copies to overlap.
+ *
+ *   q, k, v     host bf16 [B, H, N, d], token order.
+ *   o, lse      host bf16 [B, H, N, d] and float32 [B, H, N], token order.
+ *   workspace   device buffer, 256-byte aligned, of workspace_bytes >=
+ *               ra_attn_fwd_host_workspace(N, d, layout, 1) (else
+ *               RA_ERR_WORKSPACE); more allows larger chunks (up to a
+ *               quarter of the heads each).
+ *   other arguments and errors as ra_attn_fwd.
+ * Stream-ordered: work on `stream` after this call sees o and lse written.
+ * The library allocates nothing; its two copy streams and a few events are
+ * created on the first call on a device (make that call before any stream
+ * capture).  Calls on one device are enqueued one at a time; two calls that
+ * share a workspace must be ordered on one stream.
+ */
+ra_status ra_attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse,
+                           int64_t B, int64_t H, int64_t N, int64_t d, int P, int layout,
+                           int causal, float scale, void* workspace, int64_t workspace_bytes,
+                           void* stream);
+
+/* Device workspace bytes for ra_attn_fwd_host with `heads_per_chunk` heads
+ * per chunk (two staging slots); -1 for invalid sizes. */
+int64_t ra_attn_fwd_host_workspace(int64_t N, int64_t d, int layout, int64_t heads_per_chunk);
 
 /*
  * ra_attn_fwd_block -- one round of one device of the ring: query shard j

@@ -62,6 +62,60 @@ bool overlap(const void* a, int64_t na, const void* b, int64_t nb) {
   return x < y + (uintptr_t)nb && y < x + (uintptr_t)na;
 }
 
+// ------------------------------------------------------------ host path
+// Device staging of ra_attn_fwd_host: two slots, each holding a chunk of G
+// heads: q, k, v (token order), for the striped layout also qp, kp, vp, op
+// (layout order) and lsep, then o and lse (token order).
+struct HostPlan {
+  int64_t tok;      // bytes of one [N, d] bf16 head
+  int64_t lsz;      // bytes of one [N] float32 head
+  int64_t per_head; // staging bytes per head per slot (256-byte rounded parts)
+  bool striped;
+};
+
+int64_t round256(int64_t x) { return (x + 255) / 256 * 256; }
+
+HostPlan host_plan(int64_t N, int64_t d, bool striped) {
+  HostPlan h;
+  h.tok = N * d * 2;
+  h.lsz = N * 4;
+  h.striped = striped;
+  h.per_head = (striped ? 8 : 4) * round256(h.tok) + (striped ? 2 : 1) * round256(h.lsz);
+  return h;
+}
+
+struct HostStreams {
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t entry = nullptr, end = nullptr, h2d[2] = {}, comp[2] = {}, d2h[2] = {};
+  bool ready = false;
+};
+
+// Copy streams and events per device, created on first use (no device
+// memory); every call on a device holds the device's lock while enqueuing.
+ra_status host_streams(int dev, HostStreams** out, std::mutex** mu) {
+  static HostStreams hs[64];
+  static std::mutex mus[64];
+  *mu = &mus[dev];
+  std::lock_guard<std::mutex> lock(mus[dev]);
+  HostStreams& h = hs[dev];
+  if (!h.ready) {
+    const unsigned ef = cudaEventDisableTiming;
+    if (cudaStreamCreateWithFlags(&h.in, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&h.out, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&h.entry, ef) != cudaSuccess ||
+        cudaEventCreateWithFlags(&h.end, ef) != cudaSuccess)
+      return RA_ERR_CUDA;
+    for (int s = 0; s < 2; ++s)
+      if (cudaEventCreateWithFlags(&h.h2d[s], ef) != cudaSuccess ||
+          cudaEventCreateWithFlags(&h.comp[s], ef) != cudaSuccess ||
+          cudaEventCreateWithFlags(&h.d2h[s], ef) != cudaSuccess)
+        return RA_ERR_CUDA;
+    h.ready = true;
+  }
+  *out = &h;
+  return RA_OK;
+}
+
 }  // namespace
 }  // namespace ra
 
@@ -84,6 +138,7 @@ const char* ra_status_string(ra_status s) {
     case RA_ERR_DEVICE: return "current device is not an sm_100 GPU";
     case RA_ERR_DEVICE_FAULT: return "a kernel gave up a bounded wait; outputs incomplete";
     case RA_ERR_ROPE: return "unknown RoPE pairing, or RoPE base not finite and > 1";
+    case RA_ERR_WORKSPACE: return "device workspace too small (see ra_attn_fwd_host_workspace)";
     case RA_ERR_SCRATCH:
       return "B*H*N exceeds the built-in scratch of ra_attn_bwd_noalloc (1048576 rows); "
              "use ra_attn_bwd with a workspace";
@@ -329,6 +384,117 @@ ra_status ra_lse_merge_acc(float* o_acc, float* lse_acc, const void* o_b, const 
   ra_status st = current_device(&dev, &info);
   if (st) return st;
   return lse_merge_acc_launch(o_acc, lse_acc, o_b, lse_b, o_final, rows, d, first, final_, stream);
+}
+
+int64_t ra_attn_fwd_host_workspace(int64_t N, int64_t d, int layout, int64_t heads_per_chunk) {
+  if (N < 1 || d < 1 || heads_per_chunk < 1) return -1;
+  const HostPlan h = host_plan(N, d, (layout & 0xff) == RA_STRIPED);
+  return 2 * heads_per_chunk * h.per_head;
+}
+
+ra_status ra_attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse,
+                           int64_t B, int64_t H, int64_t N, int64_t d, int P, int layout,
+                           int causal, float scale, void* workspace, int64_t workspace_bytes,
+                           void* stream) {
+  if (!q || !k || !v || !o || !lse || !workspace) return RA_ERR_NULL;
+  if (layout & ~(0xff | RA_SCHED_FREE)) return RA_ERR_LAYOUT;
+  const int base = layout & 0xff;
+  if (base != RA_CONTIGUOUS && base != RA_STRIPED) return RA_ERR_LAYOUT;
+  if (d != 64 && d != 128) return RA_ERR_HEADDIM;
+  if (B < 1 || H < 1 || N < 1 || P < 1 || N % P != 0) return RA_ERR_SHAPE;
+  if (B * H * N >= ((int64_t)1 << 31) || N / P > ((int64_t)1 << 30) / 128) return RA_ERR_SHAPE;
+  if (!(scale > 0.f) || !isfinite(scale)) return RA_ERR_SCALE;
+  if (!aligned(workspace, 256)) return RA_ERR_ALIGN;
+  const bool striped = base == RA_STRIPED;
+  const HostPlan hp = host_plan(N, d, striped);
+  const int64_t BH = B * H;
+  int64_t G = workspace_bytes / (2 * hp.per_head);
+  if (G < 1) return RA_ERR_WORKSPACE;
+  // at least four chunks when there are enough heads, so that copies overlap
+  const int64_t want = (BH + 3) / 4;
+  if (G > want) G = want;
+  if (G > BH) G = BH;
+  int dev;
+  DevInfo info;
+  ra_status st = current_device(&dev, &info);
+  if (st) return st;
+  HostStreams* hs;
+  std::mutex* mu;
+  if ((st = host_streams(dev, &hs, &mu))) return st;
+  std::lock_guard<std::mutex> lock(*mu);
+  cudaStream_t cs = (cudaStream_t)stream;
+  auto chk = [](cudaError_t e) { return e == cudaSuccess; };
+  if (!chk(cudaEventRecord(hs->entry, cs)) || !chk(cudaStreamWaitEvent(hs->in, hs->entry, 0)) ||
+      !chk(cudaStreamWaitEvent(hs->out, hs->entry, 0)))
+    return RA_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int64_t T = round256(hp.tok) * G, L = round256(hp.lsz) * G;
+  const int64_t nch = (BH + G - 1) / G;
+  for (int64_t i = 0; i < nch; ++i) {
+    const int s = (int)(i & 1);
+    const int64_t h0 = i * G, g = (BH - h0 < G) ? BH - h0 : G;
+    const int64_t tb = g * hp.tok, lb = g * hp.lsz;
+    uint8_t* slot = ws + s * G * hp.per_head;
+    uint8_t *dq = slot, *dk = dq + T, *dv = dk + T, *dqp = nullptr, *dkp = nullptr, *dvp = nullptr,
+            *dop = nullptr, *dlp = nullptr;
+    uint8_t* cur = dv + T;
+    if (striped) {
+      dqp = cur; dkp = dqp + T; dvp = dkp + T; dop = dvp + T; cur = dop + T;
+    }
+    uint8_t* dout = cur;
+    cur += T;
+    if (striped) { dlp = cur; cur += L; }
+    float* dl = reinterpret_cast<float*>(cur);
+    // inputs of chunk i (the slot's previous chunk has been read back)
+    if (i >= 2 && !chk(cudaStreamWaitEvent(hs->in, hs->d2h[s], 0))) return RA_ERR_CUDA;
+    const uint8_t* hq = static_cast<const uint8_t*>(q) + h0 * hp.tok;
+    const uint8_t* hk = static_cast<const uint8_t*>(k) + h0 * hp.tok;
+    const uint8_t* hv = static_cast<const uint8_t*>(v) + h0 * hp.tok;
+    if (!chk(cudaMemcpyAsync(dq, hq, tb, cudaMemcpyHostToDevice, hs->in)) ||
+        !chk(cudaMemcpyAsync(dk, hk, tb, cudaMemcpyHostToDevice, hs->in)) ||
+        !chk(cudaMemcpyAsync(dv, hv, tb, cudaMemcpyHostToDevice, hs->in)) ||
+        !chk(cudaEventRecord(hs->h2d[s], hs->in)))
+      return RA_ERR_CUDA;
+    // compute on the caller's stream
+    if (!chk(cudaStreamWaitEvent(cs, hs->h2d[s], 0))) return RA_ERR_CUDA;
+    AttnLaunch a;
+    a.BH = g; a.N = N; a.d = d; a.P = P;
+    a.striped = striped;
+    a.causal = causal != 0;
+    a.sched_free = (layout & RA_SCHED_FREE) != 0;
+    a.scale = scale;
+    a.device = dev;
+    a.num_sms = info.num_sms;
+    a.stream = stream;
+    const int64_t row = d * 2;
+    if (striped) {
+      if ((st = partition_launch(dq, dqp, g, N, P, row, 1, 0, stream)) ||
+          (st = partition_launch(dk, dkp, g, N, P, row, 1, 0, stream)) ||
+          (st = partition_launch(dv, dvp, g, N, P, row, 1, 0, stream)))
+        return st;
+      a.q = dqp; a.k = dkp; a.v = dvp; a.o = dop; a.lse = reinterpret_cast<float*>(dlp);
+      if ((st = attn_fwd_launch(a))) return st;
+      if ((st = partition_launch(dop, dout, g, N, P, row, 1, 1, stream)) ||
+          (st = partition_launch(dlp, dl, g, N, P, 4, 1, 1, stream)))
+        return st;
+    } else {
+      a.q = dq; a.k = dk; a.v = dv; a.o = dout; a.lse = dl;
+      if ((st = attn_fwd_launch(a))) return st;
+    }
+    if (!chk(cudaEventRecord(hs->comp[s], cs))) return RA_ERR_CUDA;
+    // results of chunk i back to the host
+    if (!chk(cudaStreamWaitEvent(hs->out, hs->comp[s], 0)) ||
+        !chk(cudaMemcpyAsync(static_cast<uint8_t*>(o) + h0 * hp.tok, dout, tb,
+                             cudaMemcpyDeviceToHost, hs->out)) ||
+        !chk(cudaMemcpyAsync(reinterpret_cast<uint8_t*>(lse) + h0 * hp.lsz, dl, lb,
+                             cudaMemcpyDeviceToHost, hs->out)) ||
+        !chk(cudaEventRecord(hs->d2h[s], hs->out)))
+      return RA_ERR_CUDA;
+  }
+  // the caller's stream continues once every result is on the host
+  if (!chk(cudaEventRecord(hs->end, hs->out)) || !chk(cudaStreamWaitEvent(cs, hs->end, 0)))
+    return RA_ERR_CUDA;
+  return RA_OK;
 }
 
 ra_status ra_lse_merge(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,

@@ -54,6 +54,11 @@ def lib():
         L.ra_attn_bwd.restype = i32
         L.ra_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i32,
                                   i32, i32, f32, vp]
+        L.ra_attn_fwd_host.restype = i32
+        L.ra_attn_fwd_host.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, i32, i32,
+                                       f32, vp, i64, vp]
+        L.ra_attn_fwd_host_workspace.restype = i64
+        L.ra_attn_fwd_host_workspace.argtypes = [i64, i64, i32, i64]
         L.ra_attn_fwd_block.restype = i32
         L.ra_attn_fwd_block.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, i32, i32,
                                         i32, i32, f32, vp]
@@ -185,6 +190,39 @@ def attn_bwd(q, k, v, o, dout, lse, P, layout, causal=True, scale=None, workspac
                              _ptr(dk), _ptr(dv), _ptr(workspace), B, H, N, d, int(P), int(layout),
                              int(bool(causal)), float(scale), _stream(q)), "ra_attn_bwd")
     return dq, dk, dv
+
+
+def attn_fwd_host_workspace_bytes(N, d, layout, heads_per_chunk):
+    """Device workspace bytes ra_attn_fwd_host needs for chunks of
+    ``heads_per_chunk`` heads."""
+    return int(lib().ra_attn_fwd_host_workspace(N, d, int(layout), heads_per_chunk))
+
+
+def attn_fwd_host(q, k, v, P, layout, causal=True, scale=None, workspace=None, out=None,
+                  lse=None, sched_free=False, stream=None):
+    """The whole forward from host memory: token-order host q, k, v (bf16
+    [B, H, N, d], pinned for overlap) -> token-order host o, lse.  The heads
+    stream through ``workspace`` (a uint8 CUDA tensor) in chunks while the
+    copies of neighbouring chunks overlap the compute.  Returns (o, lse)."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        if t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16 or t.shape != q.shape:
+            raise ValueError(f"{n} must be a contiguous host bfloat16 tensor like q")
+    if q.dim() != 4:
+        raise ValueError("expected [B, H, N, d]")
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = d ** -0.5
+    if workspace is None or not workspace.is_cuda:
+        raise ValueError("workspace must be a CUDA tensor")
+    o = torch.empty(q.shape, dtype=q.dtype, pin_memory=True) if out is None else out
+    lse = torch.empty((B, H, N), dtype=torch.float32, pin_memory=True) if lse is None else lse
+    lay = int(layout) | (SCHED_FREE if sched_free else 0)
+    st = torch.cuda.current_stream(workspace.device) if stream is None else stream
+    _check(lib().ra_attn_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
+                                  int(P), lay, int(bool(causal)), float(scale), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(),
+                                  ctypes.c_void_p(st.cuda_stream)), "ra_attn_fwd_host")
+    return o, lse
 
 
 def attn_fwd_block(q, k, v, j, kb, P, layout, causal=True, scale=None, out=None, lse=None):

@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(L):
 
 def test_status_strings(L):
     assert ops.status_string(0) == "ok"
-    for code in range(1, 14):
+    for code in range(1, 15):
         assert ops.status_string(code) not in ("", "unknown status")
     assert ops.status_string(999) == "unknown status"
     assert L.ra_version() >= 100
@@ -179,3 +179,27 @@ def macc(L, oa=A, la=Bp, ob=Cp, lb=Op, of=Lp, rows=256, d=128, mode=2):
 ])
 def test_lse_merge_acc_rejects_invalid_arguments(L, kw, code):
     assert macc(L, **kw) == code
+
+
+def host(L, q=A, k=Bp, v=Cp, o=Op, lse=Lp, B=1, H=2, N=1024, d=128, P=4, layout=1, causal=1,
+         scale=0.088, ws=6 << 40, wsb=1 << 30):
+    return L.ra_attn_fwd_host(vp(q), vp(k), vp(v), vp(o), vp(lse), B, H, N, d, P, layout, causal,
+                              scale, vp(ws), wsb, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ws=0), 1), (dict(o=0), 1), (dict(ws=(6 << 40) + 128), 2), (dict(N=1000, P=3), 3),
+    (dict(d=96), 4), (dict(layout=2), 5), (dict(scale=-1.0), 6), (dict(wsb=4210687), 14),
+    (dict(wsb=0), 14),
+])
+def test_attn_fwd_host_rejects_invalid_arguments(L, kw, code):
+    assert host(L, **kw) == code
+
+
+def test_host_workspace_formula(L):
+    # per head and slot: striped 8 bf16 [N, d] buffers + 2 float32 [N];
+    # contiguous 4 + 1; two slots
+    assert L.ra_attn_fwd_host_workspace(1024, 128, 1, 1) == 2 * (8 * 262144 + 2 * 4096)
+    assert L.ra_attn_fwd_host_workspace(1024, 128, 0, 3) == 2 * 3 * (4 * 262144 + 4096)
+    assert L.ra_attn_fwd_host_workspace(1000, 64, 1, 1) == 2 * (8 * 128000 + 2 * 4096)
+    assert L.ra_attn_fwd_host_workspace(0, 64, 1, 1) == -1
