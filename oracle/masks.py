@@ -21,7 +21,7 @@ orientation; the pins check that one is the transpose of the other.
 
 import numpy as np
 
-from .partition import CONTIGUOUS, STRIPED, token_of
+from .partition import CONTIGUOUS, STRIPED, ZIGZAG, token_of
 
 
 def getmask_ring(j, k, c):
@@ -49,11 +49,22 @@ def getmask_striped(j, k, c):
     return mask
 
 
-def getmask(j, k, c, layout):
+def getmask_zigzag(j, k, c, P):
+    """The zigzag layout has no printed GetMask; its block mask in the same
+    MASK[x (key), y (query)] orientation, from C over the token positions."""
+    N = c * P
+    qpos = np.array([token_of(j, y, N, P, ZIGZAG) for y in range(c)])
+    kpos = np.array([token_of(k, x, N, P, ZIGZAG) for x in range(c)])
+    return kpos[:, None] > qpos[None, :]
+
+
+def getmask(j, k, c, layout, P=None):
     if layout == CONTIGUOUS:
         return getmask_ring(j, k, c)
     if layout == STRIPED:
         return getmask_striped(j, k, c)
+    if layout == ZIGZAG:
+        return getmask_zigzag(j, k, c, P)
     raise ValueError(layout)
 
 

@@ -14,6 +14,12 @@ tokens keep ascending order, so token t sits at local index t // P, and the
 shards are concatenated in order p = 0..P-1.  The physical ("layout") order
 is therefore slot s = shard * c + local.
 
+Zigzag: the pages only name it (the Ring-attention overview page, a
+variant that, like striping, rebalances the causal work).  Reading taken
+(the standard definition of that layout; not given on the pages): the
+sequence is cut into 2P chunks of h = c/2 tokens and shard p holds chunk p
+followed by chunk 2P-1-p, so every shard has one early and one late chunk.
+
 ``slot_to_token[s]`` is the original token index (its position id) of the
 token stored in physical slot s.  Position ids are striped with the same map
 (Striped review, 位置编码处理).
@@ -23,6 +29,7 @@ import numpy as np
 
 CONTIGUOUS = "contiguous"
 STRIPED = "striped"
+ZIGZAG = "zigzag"
 
 
 def shard_len(N, P):
@@ -38,6 +45,11 @@ def token_of(shard, local, N, P, layout):
         return shard * c + local
     if layout == STRIPED:
         return local * P + shard
+    if layout == ZIGZAG:
+        if c % 2:
+            raise ValueError("zigzag needs an even shard length")
+        h = c // 2
+        return shard * h + local if local < h else (2 * P - 1 - shard) * h + (local - h)
     raise ValueError(layout)
 
 

@@ -65,7 +65,7 @@ def ring_attention(q, k, v, P, layout, causal, scale, normalise_each_round=False
             vj = v[kb * c:(kb + 1) * c]
             s = (qj @ kj.T) * float(scale)
             if causal:
-                blocked = getmask(j, kb, c, layout).T   # -> [query, key]
+                blocked = getmask(j, kb, c, layout, P).T   # -> [query, key]
                 s = np.where(blocked, -np.inf, s)
             m_new = np.maximum(m, np.max(s, axis=1))
             m_sub = np.where(np.isneginf(m_new), 0.0, m_new)
@@ -102,7 +102,7 @@ def block_attention(qj, kb_k, kb_v, j, kb, P, layout, causal, scale):
     c = qj.shape[0]
     s = (qj @ kk.T) * float(scale)
     if causal:
-        s = np.where(getmask(j, kb, c, layout).T, -np.inf, s)
+        s = np.where(getmask(j, kb, c, layout, P).T, -np.inf, s)
     mx = np.max(s, axis=1)
     empty = np.isneginf(mx)
     e = np.exp(s - np.where(empty, 0.0, mx)[:, None])

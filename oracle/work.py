@@ -58,6 +58,15 @@ def work_exact_closed_form(j, r, c, P, layout, causal=True):
     raise ValueError(layout)
 
 
+def work_zigzag_device_total(c, P):
+    """Visible pairs of one device over all rounds, zigzag layout (the
+    reading of the partition module): chunks a and 2P-1-a of h = c/2 tokens
+    give sum over their tokens t of (t + 1) = h^2 (2P - 1) + h (h + 1), the
+    same for every device (the balance the layout exists for)."""
+    h = c // 2
+    return h * h * (2 * P - 1) + h * (h + 1)
+
+
 def work_brute_force(j, r, N, P, layout, causal=True):
     """Unmasked pairs counted element by element from token positions."""
     kb = key_block(j, r, P)

@@ -240,3 +240,20 @@ def test_block_attention_empty_rows_and_positions():
                     ref_o = (w / w.sum()) @ np.array([v[toks[kb][y]] for y in vis])
                     np.testing.assert_allclose(o[x], ref_o, atol=1e-12)
                     np.testing.assert_allclose(lse[x], s.max() + np.log(w.sum()), atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("N,P", [(16, 2), (24, 4), (40, 5)])
+def test_zigzag_ring_equals_full_softmax(causal, N, P):
+    """The ring over the zigzag layout (both folds) reaches the plain
+    result, like the two layouts of the pages."""
+    from oracle.partition import ZIGZAG
+    q, k, v = rand_qkv(N, 8, 7 * N + P, dv=6)
+    q, k = 3 * q, 3 * k
+    o_ref, lse_ref = att.attention(q, k, v, 0.35, causal)
+    qp, kp, vp = (partition.partition(a, P, ZIGZAG, axis=0) for a in (q, k, v))
+    for o, lse in (ring.ring_attention(qp, kp, vp, P, ZIGZAG, causal, 0.35),
+                   ring.ring_by_merge(qp, kp, vp, P, ZIGZAG, causal, 0.35)):
+        np.testing.assert_allclose(partition.unpartition(o, P, ZIGZAG, axis=0), o_ref, atol=1e-12)
+        np.testing.assert_allclose(partition.unpartition(lse, P, ZIGZAG, axis=0), lse_ref,
+                                   atol=1e-12)

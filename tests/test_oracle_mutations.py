@@ -204,3 +204,18 @@ def test_rope_mutants_fail_closed_form_pins(monkeypatch, kind):
     with pytest.raises(AssertionError):
         TR.test_d2_rotation_values()
         TR.test_d4_frequencies_and_pairings()
+
+
+def test_zigzag_mutant_fails_example_and_balance(monkeypatch):
+    """Planted: shard p holds chunk p and chunk 2P-2-p (an off-by-one mirror)."""
+    import tests.test_oracle_partition_masks_work as TP2
+    orig = partition.token_of
+
+    def wrong(shard, local, N, P, layout):
+        if layout != partition.ZIGZAG:
+            return orig(shard, local, N, P, layout)
+        h = N // P // 2
+        return shard * h + local if local < h else ((2 * P - 2 - shard) % (2 * P)) * h + local - h
+    monkeypatch.setattr(partition, "token_of", wrong)
+    with pytest.raises(AssertionError):
+        TP2.test_zigzag_example_N16_P4()

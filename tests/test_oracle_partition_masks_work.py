@@ -129,3 +129,42 @@ def test_striped_balances_per_round_work():
         strp = [work.work_brute_force(j, r, N, P, STRIPED) for j in range(P)]
         assert max(ring) == c * c and min(ring) == 0
         assert set(strp) <= {c * (c + 1) // 2, c * (c - 1) // 2}
+
+
+# ------------------------------------------------------------------ zigzag
+# The pages only name the zigzag layout; the oracle's reading (chunk p and
+# chunk 2P-1-p of 2P chunks on shard p) is pinned here by a hand-written
+# example of that definition, the permutation property, the equal work of
+# every device and the ring's exactness.
+from oracle.partition import ZIGZAG  # noqa: E402
+
+
+def test_zigzag_example_N16_P4():
+    want = [[0, 1, 14, 15], [2, 3, 12, 13], [4, 5, 10, 11], [6, 7, 8, 9]]
+    assert partition.shard_tokens(16, 4, ZIGZAG) == want
+
+
+@pytest.mark.parametrize("N,P", [(16, 4), (24, 3), (8, 1), (16, 8), (60, 5)])
+def test_zigzag_partition_is_a_permutation_and_inverts(N, P):
+    perm = partition.slot_to_token(N, P, ZIGZAG)
+    assert sorted(perm.tolist()) == list(range(N))
+    x = np.arange(N * 3).reshape(N, 3)
+    assert np.array_equal(partition.unpartition(partition.partition(x, P, ZIGZAG, axis=0), P,
+                                                ZIGZAG, axis=0), x)
+
+
+@pytest.mark.parametrize("N,P", [(16, 4), (24, 3), (40, 5), (32, 8)])
+def test_zigzag_work_is_equal_on_every_device(N, P):
+    c = N // P
+    totals = [sum(work.work_brute_force(j, r, N, P, ZIGZAG) for r in range(P)) for j in range(P)]
+    assert totals == [work.work_zigzag_device_total(c, P)] * P
+    assert sum(totals) == N * (N + 1) // 2
+
+
+def test_zigzag_mask_orientation_matches_positions():
+    N, P = 24, 3
+    c = N // P
+    for j in range(P):
+        for k in range(P):
+            assert np.array_equal(masks.getmask(j, k, c, ZIGZAG, P).T,
+                                  masks.mask_from_positions(j, k, N, P, ZIGZAG))
