@@ -204,11 +204,11 @@ class Path:
         self.lsep = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
         self.lse = torch.empty_like(self.lsep)
         self.ev_attn = []
-        self.launches_per_step = 6 if self.layout == W.STRIPED else 1
+        self.launches_per_step = 1 if self.layout == W.CONTIGUOUS else 6
 
     def step(self, time_attn=False):
         ops, w, P, lay = self.ops, self.w, self.w.P, self.layout
-        if lay == W.STRIPED:
+        if lay != W.CONTIGUOUS:
             for src, dst in ((self.q, self.qp), (self.k, self.kp), (self.v, self.vp)):
                 ops.partition(src, P, lay, out=dst)
             qq, kk, vv = self.qp, self.kp, self.vp
@@ -219,12 +219,12 @@ class Path:
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(s)
         ops.attn_fwd(qq, kk, vv, P, lay, w.causal, sched_free=self.sched_free,
-                     out=self.op if lay == W.STRIPED else self.o,
-                     lse=self.lsep if lay == W.STRIPED else self.lse)
+                     out=self.o if lay == W.CONTIGUOUS else self.op,
+                     lse=self.lse if lay == W.CONTIGUOUS else self.lsep)
         if time_attn:
             e1.record(s)
             self.ev_attn.append((e0, e1))
-        if lay == W.STRIPED:
+        if lay != W.CONTIGUOUS:
             ops.partition(self.op, P, lay, inverse=True, out=self.o)
             ops.partition(self.lsep, P, lay, inverse=True, out=self.lse)
 
@@ -370,7 +370,10 @@ def main():
     compare = None
     if not args.no_compare:
         compare = {}
-        for lay in (W.STRIPED, W.CONTIGUOUS):
+        lays = [W.STRIPED, W.CONTIGUOUS]
+        if (w.N // w.P) % 512 == 0:
+            lays.append(W.ZIGZAG)      # zigzag attention needs N/P a multiple of 512
+        for lay in lays:
             for sched in ("owner", "free"):
                 pth = path if (lay == w.layout and sched == args.sched) else None
                 if pth is None:

@@ -70,6 +70,10 @@ typedef int ra_status;
 /* Layouts (low byte of `layout`). */
 #define RA_CONTIGUOUS 0      /* shard j = tokens [j*c, (j+1)*c)  (Ring)        */
 #define RA_STRIPED 1         /* shard j = tokens j, j+P, j+2P, ...  (Striped)  */
+#define RA_ZIGZAG 2          /* shard j = chunks j and 2P-1-j of 2P chunks      */
+                             /* (a reading: the pages only name "zigzag";      */
+                             /* needs N/P even; attention needs N/P % 512 == 0, */
+                             /* forward paths only)                             */
 
 /* Optional scheduling flag for ra_attn_fwd, OR-ed into `layout`.
  * Default ("owner" schedule): each virtual shard j is served by its own fixed

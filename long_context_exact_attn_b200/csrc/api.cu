@@ -151,7 +151,7 @@ int ra_version(void) { return 100; }
 ra_status ra_partition(const void* src, void* dst, int64_t B, int64_t H, int64_t N, int64_t d,
                        int P, int layout, int inverse, int dtype, void* stream) {
   if (!src || !dst) return RA_ERR_NULL;
-  if (layout != RA_CONTIGUOUS && layout != RA_STRIPED) return RA_ERR_LAYOUT;
+  if (layout != RA_CONTIGUOUS && layout != RA_STRIPED && layout != RA_ZIGZAG) return RA_ERR_LAYOUT;
   int64_t esz;
   switch (dtype) {
     case RA_BF16: esz = 2; break;
@@ -159,6 +159,7 @@ ra_status ra_partition(const void* src, void* dst, int64_t B, int64_t H, int64_t
     default: return RA_ERR_DTYPE;
   }
   if (B < 1 || H < 1 || N < 1 || d < 1 || P < 1 || N % P != 0) return RA_ERR_SHAPE;
+  if (layout == RA_ZIGZAG && (N / P) % 2 != 0) return RA_ERR_SHAPE;
   if (B * H * N >= ((int64_t)1 << 31) || d * esz >= ((int64_t)1 << 30)) return RA_ERR_SHAPE;
   const int64_t row_bytes = d * esz;
   const uintptr_t need = (row_bytes % 16 == 0) ? 16 : (esz == 2 ? 2 : 4);
@@ -169,16 +170,16 @@ ra_status ra_partition(const void* src, void* dst, int64_t B, int64_t H, int64_t
   DevInfo info;
   ra_status st = current_device(&dev, &info);
   if (st) return st;
-  return partition_launch(src, dst, B * H, N, P, row_bytes, layout == RA_STRIPED, inverse != 0,
-                          stream);
+  return partition_launch(src, dst, B * H, N, P, row_bytes, layout, inverse != 0, stream);
 }
 
 ra_status ra_partition_rope(const void* src, void* dst, int64_t B, int64_t H, int64_t N,
                             int64_t d, int P, int layout, int pairing, float base, void* stream) {
   if (!src || !dst) return RA_ERR_NULL;
-  if (layout != RA_CONTIGUOUS && layout != RA_STRIPED) return RA_ERR_LAYOUT;
+  if (layout != RA_CONTIGUOUS && layout != RA_STRIPED && layout != RA_ZIGZAG) return RA_ERR_LAYOUT;
   if (d < 16 || d > 512 || d % 16 != 0) return RA_ERR_HEADDIM;
   if (B < 1 || H < 1 || N < 1 || P < 1 || N % P != 0) return RA_ERR_SHAPE;
+  if (layout == RA_ZIGZAG && (N / P) % 2 != 0) return RA_ERR_SHAPE;
   if (B * H * N >= ((int64_t)1 << 31)) return RA_ERR_SHAPE;
   if (pairing != RA_ROPE_INTERLEAVED && pairing != RA_ROPE_HALF) return RA_ERR_ROPE;
   if (!(base > 1.f) || !isfinite(base)) return RA_ERR_ROPE;
@@ -189,7 +190,7 @@ ra_status ra_partition_rope(const void* src, void* dst, int64_t B, int64_t H, in
   DevInfo info;
   ra_status st = current_device(&dev, &info);
   if (st) return st;
-  return partition_rope_launch(src, dst, B * H, N, P, d, layout == RA_STRIPED,
+  return partition_rope_launch(src, dst, B * H, N, P, d, layout,
                                pairing == RA_ROPE_HALF, std::log2((double)base), info.num_sms,
                                stream);
 }
@@ -200,9 +201,10 @@ ra_status ra_attn_fwd(const void* q, const void* k, const void* v, void* o, floa
   if (!q || !k || !v || !o || !lse) return RA_ERR_NULL;
   if (layout & ~(0xff | RA_SCHED_FREE)) return RA_ERR_LAYOUT;
   const int base = layout & 0xff;
-  if (base != RA_CONTIGUOUS && base != RA_STRIPED) return RA_ERR_LAYOUT;
+  if (base != RA_CONTIGUOUS && base != RA_STRIPED && base != RA_ZIGZAG) return RA_ERR_LAYOUT;
   if (d != 64 && d != 128) return RA_ERR_HEADDIM;
   if (B < 1 || H < 1 || N < 1 || P < 1 || N % P != 0) return RA_ERR_SHAPE;
+  if (base == RA_ZIGZAG && (N / P) % 512 != 0) return RA_ERR_SHAPE;
   if (B * H * N >= ((int64_t)1 << 31) || B * H >= ((int64_t)1 << 31)) return RA_ERR_SHAPE;
   if (N / P > ((int64_t)1 << 30) / 128) return RA_ERR_SHAPE;
   if (!(scale > 0.f) || !isfinite(scale)) return RA_ERR_SCALE;
@@ -222,6 +224,7 @@ ra_status ra_attn_fwd(const void* q, const void* k, const void* v, void* o, floa
   a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
   a.BH = B * H; a.N = N; a.d = d; a.P = P;
   a.striped = base == RA_STRIPED;
+  a.zigzag = base == RA_ZIGZAG;
   a.causal = causal != 0;
   a.sched_free = (layout & RA_SCHED_FREE) != 0;
   a.scale = scale;
@@ -388,7 +391,7 @@ ra_status ra_lse_merge_acc(float* o_acc, float* lse_acc, const void* o_b, const 
 
 int64_t ra_attn_fwd_host_workspace(int64_t N, int64_t d, int layout, int64_t heads_per_chunk) {
   if (N < 1 || d < 1 || heads_per_chunk < 1) return -1;
-  const HostPlan h = host_plan(N, d, (layout & 0xff) == RA_STRIPED);
+  const HostPlan h = host_plan(N, d, (layout & 0xff) != RA_CONTIGUOUS);
   return 2 * heads_per_chunk * h.per_head;
 }
 
@@ -399,13 +402,14 @@ ra_status ra_attn_fwd_host(const void* q, const void* k, const void* v, void* o,
   if (!q || !k || !v || !o || !lse || !workspace) return RA_ERR_NULL;
   if (layout & ~(0xff | RA_SCHED_FREE)) return RA_ERR_LAYOUT;
   const int base = layout & 0xff;
-  if (base != RA_CONTIGUOUS && base != RA_STRIPED) return RA_ERR_LAYOUT;
+  if (base != RA_CONTIGUOUS && base != RA_STRIPED && base != RA_ZIGZAG) return RA_ERR_LAYOUT;
   if (d != 64 && d != 128) return RA_ERR_HEADDIM;
   if (B < 1 || H < 1 || N < 1 || P < 1 || N % P != 0) return RA_ERR_SHAPE;
+  if (base == RA_ZIGZAG && (N / P) % 512 != 0) return RA_ERR_SHAPE;
   if (B * H * N >= ((int64_t)1 << 31) || N / P > ((int64_t)1 << 30) / 128) return RA_ERR_SHAPE;
   if (!(scale > 0.f) || !isfinite(scale)) return RA_ERR_SCALE;
   if (!aligned(workspace, 256)) return RA_ERR_ALIGN;
-  const bool striped = base == RA_STRIPED;
+  const bool striped = base != RA_CONTIGUOUS;   // a permuted layout: stage both orders
   const HostPlan hp = host_plan(N, d, striped);
   const int64_t BH = B * H;
   int64_t G = workspace_bytes / (2 * hp.per_head);
@@ -459,7 +463,8 @@ ra_status ra_attn_fwd_host(const void* q, const void* k, const void* v, void* o,
     if (!chk(cudaStreamWaitEvent(cs, hs->h2d[s], 0))) return RA_ERR_CUDA;
     AttnLaunch a;
     a.BH = g; a.N = N; a.d = d; a.P = P;
-    a.striped = striped;
+    a.striped = base == RA_STRIPED;
+    a.zigzag = base == RA_ZIGZAG;
     a.causal = causal != 0;
     a.sched_free = (layout & RA_SCHED_FREE) != 0;
     a.scale = scale;
@@ -468,14 +473,14 @@ ra_status ra_attn_fwd_host(const void* q, const void* k, const void* v, void* o,
     a.stream = stream;
     const int64_t row = d * 2;
     if (striped) {
-      if ((st = partition_launch(dq, dqp, g, N, P, row, 1, 0, stream)) ||
-          (st = partition_launch(dk, dkp, g, N, P, row, 1, 0, stream)) ||
-          (st = partition_launch(dv, dvp, g, N, P, row, 1, 0, stream)))
+      if ((st = partition_launch(dq, dqp, g, N, P, row, base, 0, stream)) ||
+          (st = partition_launch(dk, dkp, g, N, P, row, base, 0, stream)) ||
+          (st = partition_launch(dv, dvp, g, N, P, row, base, 0, stream)))
         return st;
       a.q = dqp; a.k = dkp; a.v = dvp; a.o = dop; a.lse = reinterpret_cast<float*>(dlp);
       if ((st = attn_fwd_launch(a))) return st;
-      if ((st = partition_launch(dop, dout, g, N, P, row, 1, 1, stream)) ||
-          (st = partition_launch(dlp, dl, g, N, P, 4, 1, 1, stream)))
+      if ((st = partition_launch(dop, dout, g, N, P, row, base, 1, stream)) ||
+          (st = partition_launch(dlp, dl, g, N, P, 4, base, 1, stream)))
         return st;
     } else {
       a.q = dq; a.k = dk; a.v = dv; a.o = dout; a.lse = dl;

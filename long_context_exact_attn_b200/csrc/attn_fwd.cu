@@ -50,7 +50,8 @@ struct AttnParams {
   int c;              // shard length N / P
   int P;              // shards
   int npairs;         // query-tile pairs per shard = ceil(ceil(c/128) / 2)
-  int striped;        // layout
+  int striped;        // layout: striped
+  int zigzag;         // layout: zigzag (c a multiple of 512)
   int causal;
   int groups;         // shard groups (owner schedule) or 1 (free schedule)
   int ctas_per_group;
@@ -121,7 +122,12 @@ __device__ __forceinline__ bool cta_item(const AttnParams& p, int k, Item& it) {
 
 // The key tiles met by a query-tile pair, in ring order.  Per block the two
 // query tiles' FULL / PARTIAL / SKIP thresholds are computed once; per tile
-// the classification is two compares each.
+// the classification is two compares each.  In the zigzag layout (ZZ) every
+// block is walked as its two chunks (the thresholds are per chunk pair, in
+// chunk-local rows); mxo() / myo() / mc() give the partial-tile mask its
+// coordinates: query x and key y0 of the shard are x - mxo() and y0 - myo()
+// in a block of length mc().
+template <bool ZZ>
 struct TileSeq {
   int j, P, c, striped, causal, blk_j, blk_kb;
   int x0;                   // first row of query tile 0
@@ -129,32 +135,51 @@ struct TileSeq {
   TileSpan s0, s1;
   BlockMask bm;
   int kb;
+  int zx, zy, kt_off;       // zigzag: chunk offsets of the current chunk pair
+
+  __device__ __forceinline__ int mxo() const { return ZZ ? zx : 0; }
+  __device__ __forceinline__ int myo() const { return ZZ ? zy : 0; }
+  __device__ __forceinline__ int mc() const { return ZZ ? (c >> 1) : c; }
 
   __device__ __forceinline__ void init(const AttnParams& p, const Item& it) {
     j = it.j; P = p.P; c = p.c; striped = p.striped; causal = p.causal;
     blk_j = p.blk_j; blk_kb = p.blk_kb;
     x0 = it.pair * 2 * kBM;
     r = -1; kt = 0; kend = 0;
+    zx = 0; zy = 0; kt_off = 0;
   }
   // Next tile; false at the end.  Fills block index, key start and the kind
   // of the tile for each of the two query tiles.
   __device__ __forceinline__ bool next(int& kb_out, int& y0, int& k0, int& k1, BlockMask& m) {
     while (kt >= kend) {
-      if (++r >= P) return false;
-      if (blk_kb >= 0) {
-        kb = 0;
-        bm = block_mask(blk_j, blk_kb, striped, causal);
+      if (ZZ) {
+        // sub-round r = 2 * round + chunk half of the key block
+        if (++r >= 2 * P) return false;
+        kb = key_block(j, r >> 1, P);
+        const int h = c >> 1, hk = r & 1;
+        zx = x0 < h ? 0 : h;
+        zy = hk * h;
+        bm = chunk_mask(zz_chunk(j, x0, h, P), hk ? 2 * P - 1 - kb : kb, causal);
+        s0 = tile_span(bm, x0 - zx, h);
+        s1 = tile_span(bm, x0 - zx + kBM, h);
+        kt_off = hk * (h / kBN);
       } else {
-        kb = key_block(j, r, P);
-        bm = block_mask(j, kb, striped, causal);
+        if (++r >= P) return false;
+        if (blk_kb >= 0) {
+          kb = 0;
+          bm = block_mask(blk_j, blk_kb, striped, causal);
+        } else {
+          kb = key_block(j, r, P);
+          bm = block_mask(j, kb, striped, causal);
+        }
+        s0 = tile_span(bm, x0, c);
+        s1 = tile_span(bm, x0 + kBM, c);
       }
-      s0 = tile_span(bm, x0, c);
-      s1 = tile_span(bm, x0 + kBM, c);
       kend = s0.part_end > s1.part_end ? s0.part_end : s1.part_end;
       kt = 0;
     }
     kb_out = kb;
-    y0 = kt * kBN;
+    y0 = ((ZZ ? kt_off : 0) + kt) * kBN;
     k0 = tile_kind_at(s0, kt);
     k1 = tile_kind_at(s1, kt);
     m = bm;
@@ -289,7 +314,7 @@ __device__ __forceinline__ void mma_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_
 #endif
 constexpr int kPolyEvery = RA_POLY_EVERY;
 
-template <int D>
+template <int D, bool ZZ>
 __global__ void __launch_bounds__(320, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
@@ -363,7 +388,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           for (int ch = 0; ch < C::kChunks; ++ch)
             tma_load_4d(sQ + t * C::kTileBytes + ch * 16384, &tmQ, bar_q_full, ch * 64,
                         x0 + t * kBM, it.j, it.bh);
-        TileSeq seq;
+        TileSeq<ZZ> seq;
         seq.init(p, it);
         int kb, y0, k0, k1;
         BlockMask bm;
@@ -414,7 +439,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       bool ok = true;
       for (int k = 0; ok && cta_item(p, k, it); ++k) {
         if (!wmbar_wait(bar_q_full, k & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
-        TileSeq seq;
+        TileSeq<ZZ> seq;
         seq.init(p, it);
         int kb, y0, c0, c1, n0 = TILE_SKIP, n1 = TILE_SKIP;
         BlockMask bm;
@@ -531,7 +556,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     Item it;
     bool ok = true;
     for (int k = 0; ok && cta_item(p, k, it); ++k) {
-      TileSeq seq;
+      TileSeq<ZZ> seq;
       seq.init(p, it);
       const int x = it.pair * 2 * kBM + t * kBM + row;   // local query row in shard
       float m2 = -INFINITY;   // running max, in units of log2 (scores * c2)
@@ -555,7 +580,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
           for (int i = 0; i < 32; ++i) s[q * 32 + i] = __uint_as_float(sr[q][i]);
         if (kind == TILE_PARTIAL) {
-          const int lim = row_limit(bm, x, y0, p.c);
+          const int lim = row_limit(bm, x - seq.mxo(), y0 - seq.myo(), seq.mc());
 #pragma unroll
           for (int i = 0; i < 128; ++i)
             if (i >= lim) s[i] = -INFINITY;
@@ -711,7 +736,7 @@ static bool encode_qkv_map(CUtensorMap* map, const void* base, int64_t BH, int64
   return r == CUDA_SUCCESS;
 }
 
-template <int D>
+template <int D, bool ZZ>
 static ra_status launch(const AttnLaunch& a) {
   using C = Cfg<D>;
   CUtensorMap tq, tk, tv;
@@ -722,7 +747,7 @@ static ra_status launch(const AttnLaunch& a) {
     return RA_ERR_CUDA;
   static int attr_set[64] = {0};
   if (a.device < 64 && !attr_set[a.device]) {
-    if (cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(attn_fwd_kernel<D, ZZ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmemBytes) != cudaSuccess)
       return RA_ERR_CUDA;
     attr_set[a.device] = 1;
@@ -737,6 +762,7 @@ static ra_status launch(const AttnLaunch& a) {
   const int T = (int)((c + kBM - 1) / kBM);
   p.npairs = (T + 1) / 2;
   p.striped = a.striped;
+  p.zigzag = a.zigzag;
   p.causal = a.causal;
   p.c2 = (float)((double)a.scale * 1.4426950408889634074);
   p.timeout_ns = 2000000000ull;
@@ -757,13 +783,19 @@ static ra_status launch(const AttnLaunch& a) {
     p.ctas_per_group = G;
     grid = G * p.groups;
   }
-  attn_fwd_kernel<D><<<grid, C::kThreads, C::kSmemBytes, (cudaStream_t)a.stream>>>(tq, tk, tv, p);
+  attn_fwd_kernel<D, ZZ><<<grid, C::kThreads, C::kSmemBytes, (cudaStream_t)a.stream>>>(tq, tk, tv,
+                                                                                        p);
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
 ra_status attn_fwd_launch(const AttnLaunch& a) {
-  if (a.d == 128) return launch<128>(a);
-  if (a.d == 64) return launch<64>(a);
+  if (a.zigzag) {
+    if (a.d == 128) return launch<128, true>(a);
+    if (a.d == 64) return launch<64, true>(a);
+  } else {
+    if (a.d == 128) return launch<128, false>(a);
+    if (a.d == 64) return launch<64, false>(a);
+  }
   return RA_ERR_HEADDIM;
 }
 

@@ -13,10 +13,23 @@ namespace ra {
 // Row n of the destination (within one (b, h)) comes from source row
 //   forward (token -> layout): slot n holds token (n % c) * P + n / c
 //   inverse (layout -> token): token n sits in slot (n % P) * c + n / P
-// (striped placement of the Striped Attention review, 分区策略对比).
+// (striped placement of the Striped Attention review, 分区策略对比), or, for
+// the zigzag layout (zz; chunks j and 2P-1-j of h = c/2 tokens on shard j)
+//   forward: slot n = (j, l) holds token j*h + l (l < h), (2P-1-j)*h + l-h
+//   inverse: token n in chunk a = n / h sits in shard a (a < P) or 2P-1-a.
+__device__ __forceinline__ int zz_token_of_slot(int n, int c, int P) {
+  const int h = c >> 1, j = n / c, l = n - j * c;
+  return l < h ? j * h + l : (2 * P - 1 - j) * h + (l - h);
+}
+__device__ __forceinline__ int zz_slot_of_token(int n, int c, int P) {
+  const int h = c >> 1, a = n / h, l = n - a * h;
+  return a < P ? a * c + l : (2 * P - 1 - a) * c + h + l;
+}
+
 template <typename U>
 __global__ void partition_kernel(const U* __restrict__ src, U* __restrict__ dst, int rows_total,
-                                 int N, int P, int c, int upr, int rows_per_block, int inverse) {
+                                 int N, int P, int c, int upr, int rows_per_block, int inverse,
+                                 int zz) {
   const int row0 = blockIdx.x * rows_per_block;
   int nrows = rows_total - row0;
   if (nrows > rows_per_block) nrows = rows_per_block;
@@ -28,7 +41,9 @@ __global__ void partition_kernel(const U* __restrict__ src, U* __restrict__ dst,
     const int bh = row / N;
     const int n = row - bh * N;
     int sn;
-    if (inverse) {
+    if (zz) {
+      sn = inverse ? zz_slot_of_token(n, c, P) : zz_token_of_slot(n, c, P);
+    } else if (inverse) {
       const int sh = n % P;
       sn = sh * c + n / P;
     } else {
@@ -41,22 +56,22 @@ __global__ void partition_kernel(const U* __restrict__ src, U* __restrict__ dst,
 
 template <typename U>
 static ra_status launch_partition_t(const void* src, void* dst, int rows_total, int N, int P,
-                                    int64_t row_bytes, int inverse, void* stream) {
+                                    int64_t row_bytes, int inverse, int zz, void* stream) {
   const int upr = (int)(row_bytes / (int64_t)sizeof(U));
   int rpb = 2048 / upr;
   if (rpb < 1) rpb = 1;
   const int blocks = (rows_total + rpb - 1) / rpb;
   partition_kernel<U><<<blocks, 256, 0, (cudaStream_t)stream>>>(
       reinterpret_cast<const U*>(src), reinterpret_cast<U*>(dst), rows_total, N, P, N / P, upr,
-      rpb, inverse);
+      rpb, inverse, zz);
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
 ra_status partition_launch(const void* src, void* dst, int64_t rows_outer, int64_t N, int64_t P,
-                           int64_t row_bytes, int striped, int inverse, void* stream) {
+                           int64_t row_bytes, int layout, int inverse, void* stream) {
   const int64_t total_bytes = rows_outer * N * row_bytes;
   if (total_bytes == 0) return RA_OK;
-  if (!striped) {
+  if (layout == RA_CONTIGUOUS) {
     // the contiguous placement is the identity
     return cudaMemcpyAsync(dst, src, (size_t)total_bytes, cudaMemcpyDeviceToDevice,
                            (cudaStream_t)stream) == cudaSuccess
@@ -67,18 +82,18 @@ ra_status partition_launch(const void* src, void* dst, int64_t rows_outer, int64
   const uintptr_t al = reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst);
   if (row_bytes % 16 == 0 && al % 16 == 0)
     return launch_partition_t<uint4>(src, dst, rows_total, (int)N, (int)P, row_bytes, inverse,
-                                     stream);
+                                     layout == RA_ZIGZAG, stream);
   if (row_bytes % 8 == 0 && al % 8 == 0)
     return launch_partition_t<uint2>(src, dst, rows_total, (int)N, (int)P, row_bytes, inverse,
-                                     stream);
+                                     layout == RA_ZIGZAG, stream);
   if (row_bytes % 4 == 0 && al % 4 == 0)
     return launch_partition_t<uint32_t>(src, dst, rows_total, (int)N, (int)P, row_bytes,
-                                        inverse, stream);
+                                        inverse, layout == RA_ZIGZAG, stream);
   if (row_bytes % 2 == 0 && al % 2 == 0)
     return launch_partition_t<uint16_t>(src, dst, rows_total, (int)N, (int)P, row_bytes,
-                                        inverse, stream);
+                                        inverse, layout == RA_ZIGZAG, stream);
   return launch_partition_t<uint8_t>(src, dst, rows_total, (int)N, (int)P, row_bytes, inverse,
-                                     stream);
+                                     layout == RA_ZIGZAG, stream);
 }
 
 // --------------------------------------------------- partition with RoPE
@@ -91,7 +106,7 @@ ra_status partition_launch(const void* src, void* dst, int64_t rows_outer, int64
 // angle reaches N radians), rotated in fp32, rounded to bf16 once.
 template <int HALF>
 __global__ void partition_rope_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
-                                      int BH, int N, int P, int c, int striped, int d,
+                                      int BH, int N, int P, int c, int layout, int d,
                                       double log2_base) {
   constexpr int kPairs = HALF ? 8 : 4;       // rotation pairs per work chunk
   const int u16 = d / 8;                     // 16-byte units per row
@@ -100,7 +115,8 @@ __global__ void partition_rope_kernel(const uint4* __restrict__ src, uint4* __re
   for (long long w = (long long)blockIdx.x * blockDim.x + threadIdx.x; w < total;
        w += (long long)gridDim.x * blockDim.x) {
     const int t = (int)(w / cpr), ch = (int)(w % cpr);
-    const int s = striped ? (t % P) * c + t / P : t;
+    const int s = layout == RA_STRIPED ? (t % P) * c + t / P
+                  : layout == RA_ZIGZAG ? zz_slot_of_token(t, c, P) : t;
     float cs[kPairs], sn[kPairs];
 #pragma unroll
     for (int k = 0; k < kPairs; ++k) {
@@ -144,7 +160,7 @@ __global__ void partition_rope_kernel(const uint4* __restrict__ src, uint4* __re
 }
 
 ra_status partition_rope_launch(const void* src, void* dst, int64_t BH, int64_t N, int64_t P,
-                                int64_t d, int striped, int half, double log2_base, int num_sms,
+                                int64_t d, int layout, int half, double log2_base, int num_sms,
                                 void* stream) {
   const long long cpr = half ? d / 16 : d / 8;
   const long long total = N * cpr;
@@ -156,10 +172,10 @@ ra_status partition_rope_launch(const void* src, void* dst, int64_t BH, int64_t 
   cudaStream_t st = (cudaStream_t)stream;
   if (half)
     partition_rope_kernel<1><<<(int)blocks, 256, 0, st>>>(s, t, (int)BH, (int)N, (int)P,
-                                                           (int)(N / P), striped, (int)d, log2_base);
+                                                           (int)(N / P), layout, (int)d, log2_base);
   else
     partition_rope_kernel<0><<<(int)blocks, 256, 0, st>>>(s, t, (int)BH, (int)N, (int)P,
-                                                           (int)(N / P), striped, (int)d, log2_base);
+                                                           (int)(N / P), layout, (int)d, log2_base);
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 

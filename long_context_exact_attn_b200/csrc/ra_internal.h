@@ -30,6 +30,7 @@ struct AttnLaunch {
   int device, num_sms;
   void* stream;
   int blk_j = -1, blk_kb = -1;   // single-block mode when blk_kb >= 0 (P = 1)
+  int zigzag = 0;                // zigzag layout (striped == 0)
 };
 
 ra_status attn_fwd_launch(const AttnLaunch& a);
@@ -63,10 +64,10 @@ unsigned int* device_fault_word();
 ra_status wait_selftest_launch(int64_t limit_ns, void* stream);
 
 ra_status partition_launch(const void* src, void* dst, int64_t rows_outer, int64_t N, int64_t P,
-                           int64_t row_bytes, int striped, int inverse, void* stream);
+                           int64_t row_bytes, int layout, int inverse, void* stream);
 
 ra_status partition_rope_launch(const void* src, void* dst, int64_t BH, int64_t N, int64_t P,
-                                int64_t d, int striped, int half, double log2_base, int num_sms,
+                                int64_t d, int layout, int half, double log2_base, int num_sms,
                                 void* stream);
 ra_status lse_merge_acc_launch(float* o_acc, float* lse_acc, const void* o_b,
                                const float* lse_b, void* o_final, int64_t rows, int64_t d,

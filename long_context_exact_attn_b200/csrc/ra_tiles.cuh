@@ -123,6 +123,24 @@ RA_HD int row_limit(const BlockMask& m, int x, int y0, int c) {
   return lim;
 }
 
+// Zigzag layout (a reading: the pages only name it): shard j holds chunk j
+// (local rows [0, h)) followed by chunk 2P-1-j (local rows [h, 2h)), with
+// h = c / 2.  Within a pair of chunks the causal structure is that of the
+// contiguous layout: an earlier key chunk is fully visible, the same chunk
+// is the diagonal (key y' visible to query x' iff y' < x' + 1), a later
+// chunk is hidden.
+RA_HD int zz_chunk(int shard, int local, int h, int P) {
+  return local < h ? shard : 2 * P - 1 - shard;
+}
+
+RA_HD BlockMask chunk_mask(int query_chunk, int key_chunk, int causal) {
+  BlockMask m{0, 0, 1};
+  if (!causal) return m;
+  if (key_chunk > query_chunk) m.all_hidden = 1;
+  else if (key_chunk == query_chunk) m.use_diag = 1;
+  return m;
+}
+
 RA_HD int key_block(int j, int r, int P) {
   int kb = j - r;
   return kb < 0 ? kb + P : kb;

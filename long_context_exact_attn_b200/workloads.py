@@ -17,7 +17,8 @@ import torch
 
 CONTIGUOUS = 0
 STRIPED = 1
-LAYOUT_NAMES = {CONTIGUOUS: "contiguous", STRIPED: "striped"}
+ZIGZAG = 2
+LAYOUT_NAMES = {CONTIGUOUS: "contiguous", STRIPED: "striped", ZIGZAG: "zigzag"}
 
 
 @dataclass(frozen=True)

@@ -68,7 +68,7 @@ def attn(L, q=A, k=Bp, v=Cp, o=Op, lse=Lp, B=1, H=2, N=1024, d=128, P=4, layout=
     (dict(q=A + 8), 2), (dict(o=Op + 2), 2), (dict(lse=Lp + 4), 2),
     (dict(N=1000, P=3), 3), (dict(P=0), 3), (dict(N=0), 3), (dict(B=0), 3),
     (dict(d=96), 4), (dict(d=256), 4),
-    (dict(layout=2), 5), (dict(layout=0x400), 5),
+    (dict(layout=3), 5), (dict(layout=0x400), 5),
     (dict(scale=0.0), 6), (dict(scale=float("inf")), 6), (dict(scale=float("nan")), 6),
     (dict(scale=-1.0), 6),
     (dict(o=A), 8), (dict(lse=Op + 64), 8),
@@ -146,7 +146,7 @@ def prope(L, src=A, dst=Bp, B=1, H=2, N=1024, d=128, P=4, layout=1, pairing=0, b
 
 @pytest.mark.parametrize("kw,code", [
     (dict(src=0), 1), (dict(dst=A + 16), 8), (dict(dst=Bp + 8), 2), (dict(N=1000, P=3), 3),
-    (dict(d=72), 4), (dict(d=8), 4), (dict(d=1024), 4), (dict(layout=2), 5),
+    (dict(d=72), 4), (dict(d=8), 4), (dict(d=1024), 4), (dict(layout=3), 5),
     (dict(pairing=2), 13), (dict(base=1.0), 13), (dict(base=float("inf")), 13),
     (dict(base=float("nan")), 13), (dict(B=0), 3),
 ])
@@ -189,7 +189,7 @@ def host(L, q=A, k=Bp, v=Cp, o=Op, lse=Lp, B=1, H=2, N=1024, d=128, P=4, layout=
 
 @pytest.mark.parametrize("kw,code", [
     (dict(ws=0), 1), (dict(o=0), 1), (dict(ws=(6 << 40) + 128), 2), (dict(N=1000, P=3), 3),
-    (dict(d=96), 4), (dict(layout=2), 5), (dict(scale=-1.0), 6), (dict(wsb=4210687), 14),
+    (dict(d=96), 4), (dict(layout=3), 5), (dict(scale=-1.0), 6), (dict(wsb=4210687), 14),
     (dict(wsb=0), 14),
 ])
 def test_attn_fwd_host_rejects_invalid_arguments(L, kw, code):
@@ -203,3 +203,23 @@ def test_host_workspace_formula(L):
     assert L.ra_attn_fwd_host_workspace(1024, 128, 0, 3) == 2 * 3 * (4 * 262144 + 4096)
     assert L.ra_attn_fwd_host_workspace(1000, 64, 1, 1) == 2 * (8 * 128000 + 2 * 4096)
     assert L.ra_attn_fwd_host_workspace(0, 64, 1, 1) == -1
+
+
+@pytest.mark.parametrize("fn,kw,code", [
+    ("fwd", dict(layout=2, N=1024, P=4), 3),          # c = 256: not a multiple of 512
+    ("fwd", dict(layout=2, N=2048, P=4), None),       # valid sizes: passes validation
+    ("bwd", dict(layout=2), 5),                        # backward: contiguous / striped only
+])
+def test_zigzag_validation(L, fn, kw, code):
+    if fn == "fwd":
+        st = attn(L, **kw)
+        if code is None:
+            assert st not in (3, 5)                  # fails later (no GPU here), not on sizes
+        else:
+            assert st == code
+    else:
+        assert bwd(L, **kw) == code
+
+
+def test_zigzag_partition_needs_even_shards(L):
+    assert L.ra_partition(vp(A), vp(Bp), 1, 1, 600, 8, 200, 2, 0, 0, None) == 3   # c = 3

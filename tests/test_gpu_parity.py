@@ -20,7 +20,7 @@ from oracle import work as OW
 pytestmark = pytest.mark.gpu
 
 O_MAX, O_MEAN, LSE_MAX = 2e-2, 2e-3, 1e-3
-LAYOUT = {W.CONTIGUOUS: OP.CONTIGUOUS, W.STRIPED: OP.STRIPED}
+LAYOUT = {W.CONTIGUOUS: OP.CONTIGUOUS, W.STRIPED: OP.STRIPED, W.ZIGZAG: OP.ZIGZAG}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -36,10 +36,10 @@ def run_path(q, k, v, P, layout, causal, sched_free=False, scale=None):
     q, k, v: CPU bf16 [B, H, N, d] in token order.  Returns O (float32 numpy,
     token order) and lse (numpy, token order)."""
     dq, dk, dv = (t.cuda() for t in (q, k, v))
-    if layout == W.STRIPED:
+    if layout != W.CONTIGUOUS:
         dq, dk, dv = (ops.partition(t, P, layout) for t in (dq, dk, dv))
     o, lse = ops.attn_fwd(dq, dk, dv, P, layout, causal, scale=scale, sched_free=sched_free)
-    if layout == W.STRIPED:
+    if layout != W.CONTIGUOUS:
         o = ops.partition(o, P, layout, inverse=True)
         lse = ops.partition(lse, P, layout, inverse=True)
     torch.cuda.synchronize()
