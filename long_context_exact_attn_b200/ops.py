@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(_HERE, "libringattn.so")
 
 CONTIGUOUS = 0
 STRIPED = 1
+ZIGZAG = 2
 SCHED_FREE = 0x100
 
 BF16 = 0
