@@ -284,6 +284,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-chunks", type=int, default=8,
                     help="head chunks of the host-buffer path (copies overlap compute)")
+    ap.add_argument("--ring-emulate", action="store_true",
+                    help="time every (rank, round) block of the physical ring on this GPU")
     ap.add_argument("--no-rope", action="store_true",
                     help="skip timing the stripe + RoPE partition of q")
     ap.add_argument("--backward", action="store_true",
@@ -428,6 +430,60 @@ def main():
                     "flop_convention": "useful 10 d per visible pair (QK^T, dO V^T, dV, dK, dQ); "
                                        "executed 14 d (S and dP recomputed for dQ)"}
 
+    # ---- the physical ring, emulated on this GPU: every (rank j, round r)
+    # block of ra_attn_fwd_block timed alone; on P devices round r lasts as
+    # long as its slowest rank, so sum_r max_j t(j, r) predicts the ring's
+    # compute time (the K/V exchange, 2 B H c d 2 bytes per rank per round,
+    # overlaps it)
+    ring = None
+    if args.ring_emulate and rank == 0 and world == 1:
+        ring = {}
+        c = w.N // w.P
+        for lay in (W.STRIPED, W.CONTIGUOUS):
+            pth = Path(ops, w, q, k, v, layout=lay)
+            src = (pth.q, pth.k, pth.v)
+            if lay != W.CONTIGUOUS:
+                for a, b in ((pth.q, pth.qp), (pth.k, pth.kp), (pth.v, pth.vp)):
+                    ops.partition(a, w.P, lay, out=b)
+                src = (pth.qp, pth.kp, pth.vp)
+            shards = [[t[:, :, j * c:(j + 1) * c].contiguous() for j in range(w.P)] for t in src]
+            del pth
+            o_blk = torch.empty_like(shards[0][0])
+            l_blk = torch.empty(w.B, w.H, c, dtype=torch.float32, device="cuda")
+            acc = torch.empty(o_blk.shape, dtype=torch.float32, device="cuda")
+            lacc = torch.empty_like(l_blk)
+            t = [[0.0] * w.P for _ in range(w.P)]
+            for rep in range(2):                       # first pass warms up
+                for j in range(w.P):
+                    for r in range(w.P):
+                        kb = (j - r) % w.P
+                        e0 = torch.cuda.Event(enable_timing=True)
+                        e1 = torch.cuda.Event(enable_timing=True)
+                        e0.record()
+                        ops.attn_fwd_block(shards[0][j], shards[1][kb], shards[2][kb], j, kb, w.P,
+                                           lay, w.causal, out=o_blk, lse=l_blk)
+                        ops.lse_merge_acc(acc, lacc, o_blk, l_blk, first=(r == 0))
+                        e1.record()
+                        e1.synchronize()
+                        t[j][r] = e0.elapsed_time(e1)
+            del shards, o_blk, l_blk, acc, lacc
+            torch.cuda.empty_cache()
+            round_max = [max(t[j][r] for j in range(w.P)) for r in range(w.P)]
+            total = sum(round_max)
+            per_rank = [sum(t[j]) for j in range(w.P)]
+            xfer = 2 * w.B * w.H * c * w.d * 2
+            ring[W.LAYOUT_NAMES[lay]] = {
+                "predicted_ring_ms": total,
+                "useful_tflops_on_P_gpus": flops / (total * 1e-3) / 1e12,
+                "round_max_ms": [round(x, 3) for x in round_max],
+                "rank_busy_ms_min_max": [round(min(per_rank), 3), round(max(per_rank), 3)],
+                "kv_bytes_per_rank_per_round": xfer,
+                "kv_ms_per_round_at_770GBs": xfer / 770e9 * 1e3}
+        if ops.device_fault():
+            raise RuntimeError("device fault during the ring emulation")
+        ring["note"] = ("per-round block + merge kernels of every rank run one at a time on "
+                        "this GPU; P GPUs would run each round's ranks concurrently")
+
     # ---- stripe + RoPE of q and k (memory-bound side path, not in the step)
     rope = None
     if not args.no_rope:
@@ -488,6 +544,7 @@ def main():
         "layout_compare": compare,
         "backward": backward,
         "rope_partition": rope,
+        "ring_emulation": ring,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -38,3 +38,22 @@ def attention_backward(q, k, v, do, scale, causal, q_pos=None, k_pos=None):
     dq = (ds @ k) * float(scale)
     dk = (ds.T @ q) * float(scale)
     return dq, dk, dv, d_row
+
+
+def dq_rows(q, k, v, do, scale, causal, rows):
+    """dQ of the chosen query rows only, by the same definition (row i needs
+    its own scores, lse_i, O_i and D_i = dO_i . O_i; nothing of other rows),
+    for sequences too long for the full matrices.  [len(rows), d] float64."""
+    q, k, v, do = (np.asarray(a, dtype=np.float64) for a in (q, k, v, do))
+    out = np.empty((len(rows), k.shape[1]))
+    for n, i in enumerate(rows):
+        nk = (int(i) + 1) if causal else k.shape[0]
+        s = (k[:nk] @ q[i]) * float(scale)
+        mx = np.max(s)
+        e = np.exp(s - mx)
+        p = e / np.sum(e)
+        o = p @ v[:nk]
+        dp = v[:nk] @ do[i]
+        ds = p * (dp - np.dot(do[i], o))
+        out[n] = (ds @ k[:nk]) * float(scale)
+    return out

@@ -97,3 +97,31 @@ def test_backward_striped_equals_contiguous():
     b = run_bwd(q, k, v, do, w.P, W.STRIPED, True)
     for x, y in zip(a, b):
         assert np.abs(x - y).max() <= 2 * REL_MAX * max(np.abs(x).max(), 1e-6)
+
+
+def test_backward_full_stress_size():
+    """The backward at the stress shape (B1 H16 N262144 d128 P16 striped,
+    q,k x3): dQ of sampled rows against the oracle's per-row gradient, and
+    two identities of the gradients that hold at any size: every row of P
+    sums to 1, so sum_j dV_j = sum_i dO_i; every row of dS sums to 0, so
+    sum_j dK_j = 0 (per head and dimension; bf16 rounding allowed for)."""
+    w = W.STRESS_256K
+    q, k, v = W.make_qkv(w)
+    do = torch.randn(q.shape, generator=torch.Generator().manual_seed(12)).to(torch.bfloat16)
+    gq, gk, gv = (torch.from_numpy(a) for a in run_bwd(q, k, v, do, w.P, w.layout, w.causal))
+    rng = np.random.default_rng(3)
+    rows = np.unique(np.concatenate([[0, 1, 16383, 16384, 131072, w.N - 1],
+                                     rng.integers(0, w.N, 10)]))
+    for h in (0, w.H - 1):
+        ref = OB.dq_rows(q[0, h].float().numpy(), k[0, h].float().numpy(),
+                         v[0, h].float().numpy(), do[0, h].float().numpy(), w.scale, True, rows)
+        got = gq[0, h, rows].numpy()
+        scale = max(np.abs(ref).max(), 1e-6)
+        assert np.abs(got - ref).max() <= REL_MAX * scale, (h, np.abs(got - ref).max() / scale)
+    sum_dv = gv[0].double().sum(dim=1)                 # [H, d]
+    sum_do = do[0].double().sum(dim=1)
+    abs_dv = gv[0].double().abs().sum(dim=1)
+    assert torch.all((sum_dv - sum_do).abs() <= 2.0 ** -7 * abs_dv + 1e-3)
+    sum_dk = gk[0].double().sum(dim=1)
+    abs_dk = gk[0].double().abs().sum(dim=1)
+    assert torch.all(sum_dk.abs() <= 2.0 ** -7 * abs_dk + 1e-3)

@@ -69,3 +69,14 @@ def test_D_is_rowsum_of_P_times_dP():
     s = np.where(np.triu(np.ones((10, 10), bool), 1), -np.inf, q @ k.T * 0.4)
     p = np.exp(s - lse[:, None])
     np.testing.assert_allclose(d_row, np.sum(p * (do @ v.T), axis=1), atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_dq_rows_equal_full_backward(causal):
+    """The per-row dQ equals the full backward's rows (same definition)."""
+    g = np.random.default_rng(8)
+    n, d = 40, 8
+    q, k, v, do = (g.standard_normal((n, d)) for _ in range(4))
+    dq, _, _, _ = OB.attention_backward(q, k, v, do, 0.3, causal)
+    rows = [0, 1, 17, 39]
+    np.testing.assert_allclose(OB.dq_rows(q, k, v, do, 0.3, causal, rows), dq[rows], atol=1e-12)
