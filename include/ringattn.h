@@ -20,13 +20,19 @@
  *     (token t on device t mod P), GetMask 函数 (block masks), 分块与分瓦片
  *     (skip fully masked tiles), 位置编码处理 (position ids striped alike).
  *   - 1cademy, "Computing Attention Weights in Sequence Parallelism": the
- *     softmax denominator as a sum of per-node partial sums (lse merge).
+ *     softmax denominator as a sum of per-node partial sums (lse merge, the
+ *     per-round partials of the ring).
+ *   - aiunderstanding.org, "Parallélisme de séquence et attention en
+ *     anneau": L'avenir (zigzag named as a causal rebalancing variant beside
+ *     striping; the layout's definition here is a reading, see RA_ZIGZAG).
  *
  * Conventions for every entry point:
  *   - All pointers marked "device" are CUDA device pointers on the current
  *     device; the caller allocates and owns every buffer (including the
- *     backward's workspace).  The library never allocates device memory and
- *     keeps no pointer after a call returns.
+ *     backward's workspace and ra_attn_fwd_host's staging workspace).  The
+ *     library never allocates device memory at run time (its only device
+ *     data are static: a 4-byte fault word and ra_attn_bwd_noalloc's 4 MiB
+ *     scratch) and keeps no pointer after a call returns.
  *   - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL =
  *     the legacy default stream).  A return of RA_OK means the work was
  *     validated and enqueued, not that it finished.
@@ -35,8 +41,10 @@
  *     point aborts, prints, or traps on the device.
  *   - Tensors are dense row-major.  [B, H, N, d] bf16 means element
  *     (b, h, n, i) at ((b*H + h)*N + n)*d + i, two bytes each.
- *   - Thread safety: calls may be made from several host threads; each call
- *     only reads its arguments.
+ *   - Thread safety: calls may be made from several host threads.  The
+ *     exceptions share library state: ra_attn_bwd_noalloc's scratch (calls
+ *     must not overlap on the GPU) and ra_attn_fwd_host's copy streams
+ *     (calls on one device are enqueued one at a time).
  */
 #ifndef RINGATTN_H_
 #define RINGATTN_H_
