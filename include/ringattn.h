@@ -80,8 +80,8 @@ typedef int ra_status;
 #define RA_STRIPED 1         /* shard j = tokens j, j+P, j+2P, ...  (Striped)  */
 #define RA_ZIGZAG 2          /* shard j = chunks j and 2P-1-j of 2P chunks      */
                              /* (a reading: the pages only name "zigzag";      */
-                             /* needs N/P even; attention needs N/P % 512 == 0, */
-                             /* forward paths only)                             */
+                             /* needs N/P even; attention needs N/P % 512 == 0; */
+                             /* not for ra_attn_fwd_block / ra_tile_census)     */
 
 /* Optional scheduling flag for ra_attn_fwd, OR-ed into `layout`.
  * Default ("owner" schedule): each virtual shard j is served by its own fixed

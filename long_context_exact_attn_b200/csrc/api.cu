@@ -239,9 +239,10 @@ ra_status ra_attn_bwd(const void* q, const void* k, const void* v, const void* o
                       float* workspace, int64_t B, int64_t H, int64_t N, int64_t d, int P,
                       int layout, int causal, float scale, void* stream) {
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return RA_ERR_NULL;
-  if (layout != RA_CONTIGUOUS && layout != RA_STRIPED) return RA_ERR_LAYOUT;
+  if (layout != RA_CONTIGUOUS && layout != RA_STRIPED && layout != RA_ZIGZAG) return RA_ERR_LAYOUT;
   if (d != 64 && d != 128) return RA_ERR_HEADDIM;
   if (B < 1 || H < 1 || N < 1 || P < 1 || N % P != 0) return RA_ERR_SHAPE;
+  if (layout == RA_ZIGZAG && (N / P) % 512 != 0) return RA_ERR_SHAPE;
   if (B * H * N >= ((int64_t)1 << 31) || N / P > ((int64_t)1 << 30) / 128) return RA_ERR_SHAPE;
   if (B * H * P * ((N / P + 127) / 128) >= ((int64_t)1 << 31)) return RA_ERR_SHAPE;
   if (!(scale > 0.f) || !isfinite(scale)) return RA_ERR_SCALE;
@@ -270,6 +271,7 @@ ra_status ra_attn_bwd(const void* q, const void* k, const void* v, const void* o
   a.dq = dq; a.dk = dk; a.dv = dv; a.workspace = workspace;
   a.BH = B * H; a.N = N; a.d = d; a.P = P;
   a.striped = layout == RA_STRIPED;
+  a.zigzag = layout == RA_ZIGZAG;
   a.causal = causal != 0;
   a.scale = scale;
   a.device = dev;
@@ -283,9 +285,10 @@ ra_status ra_attn_bwd_noalloc(const void* q, const void* k, const void* v, const
                               int64_t B, int64_t H, int64_t N, int64_t d, int P, int layout,
                               int causal, float scale, void* stream) {
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return RA_ERR_NULL;
-  if (layout != RA_CONTIGUOUS && layout != RA_STRIPED) return RA_ERR_LAYOUT;
+  if (layout != RA_CONTIGUOUS && layout != RA_STRIPED && layout != RA_ZIGZAG) return RA_ERR_LAYOUT;
   if (d != 64 && d != 128) return RA_ERR_HEADDIM;
   if (B < 1 || H < 1 || N < 1 || P < 1 || N % P != 0) return RA_ERR_SHAPE;
+  if (layout == RA_ZIGZAG && (N / P) % 512 != 0) return RA_ERR_SHAPE;
   if (B * H * N >= ((int64_t)1 << 31) || N / P > ((int64_t)1 << 30) / 128) return RA_ERR_SHAPE;
   if (B * H * N > kNoAllocScratchFloats) return RA_ERR_SCRATCH;
   if (!(scale > 0.f) || !isfinite(scale)) return RA_ERR_SCALE;
@@ -311,6 +314,7 @@ ra_status ra_attn_bwd_noalloc(const void* q, const void* k, const void* v, const
   a.dq = dq; a.dk = dk; a.dv = dv; a.workspace = nullptr;
   a.BH = B * H; a.N = N; a.d = d; a.P = P;
   a.striped = layout == RA_STRIPED;
+  a.zigzag = layout == RA_ZIGZAG;
   a.causal = causal != 0;
   a.scale = scale;
   a.device = dev;

@@ -42,7 +42,7 @@ struct BwdParams {
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
-  int BH, N, c, P, T, striped, causal;
+  int BH, N, c, P, T, striped, zigzag, causal;
   float c2;               // scale * log2(e)
   float scale;
   unsigned long long timeout_ns;
@@ -265,25 +265,49 @@ __device__ __forceinline__ bool smem_base_ok(const uint8_t* smem, const BwdParam
 // order is free).  On a diagonal block, query tiles before kt - 1 cannot see
 // key tile kt (a query tile qt reaches keys up to (qt + 1) * 128 - 1 + e),
 // so the walk starts there.
+template <bool ZZ>
 struct QCursor {
   int j, qt, P, T, c, kb, striped, causal, y0;
   BlockMask m;
+  int qh, xo, yo;           // zigzag: query chunk half, chunk offsets (query, key)
+  int ktl;                  // key tile index inside its chunk (zigzag) or block
+  // Mask coordinates of the current tile: query row x and key row y of the
+  // shards are x - xo and y - yo in a block (or chunk pair) of length mc().
+  __device__ __forceinline__ int mc() const { return ZZ ? (c >> 1) : c; }
   __device__ void init(const BwdParams& p, int kb_, int y0_) {
     j = 0; qt = -1; P = p.P; T = p.T; c = p.c; kb = kb_; striped = p.striped; causal = p.causal;
     y0 = y0_;
+    qh = 0; xo = 0;
+    const int h = c >> 1;
+    yo = (ZZ && y0 >= h) ? h : 0;
+    ktl = (y0 - yo) / kBN;
   }
   __device__ bool next(int& oj, int& oqt) {
+    const int Tq = ZZ ? (T >> 1) : T;         // query tiles per (chunk or block)
     while (j < P) {
       if (qt < 0) {
-        m = block_mask(j, kb, striped, causal);
-        if (m.all_hidden) { ++j; continue; }
-        const int kt = y0 / kBN;
-        qt = (m.use_diag && kt > 0) ? kt - 1 : 0;
+        if (ZZ) {
+          const int h = c >> 1;
+          m = chunk_mask(qh ? 2 * P - 1 - j : j, zz_chunk(kb, y0, h, P), causal);
+          xo = qh * h;
+        } else {
+          m = block_mask(j, kb, striped, causal);
+        }
+        if (m.all_hidden) {
+          qt = -1;
+          if (!ZZ || qh == 1) { qh = 0; ++j; } else { qh = 1; }
+          continue;
+        }
+        qt = (m.use_diag && ktl > 0) ? ktl - 1 : 0;
       }
-      if (qt >= T) { qt = -1; ++j; continue; }
-      const int k = tile_kind(m, qt * kBM, y0, c);
+      if (qt >= Tq) {
+        qt = -1;
+        if (!ZZ || qh == 1) { qh = 0; ++j; } else { qh = 1; }
+        continue;
+      }
+      const int k = tile_kind(m, qt * kBM, y0 - yo, mc());
       ++qt;
-      if (k != TILE_SKIP) { oj = j; oqt = qt - 1; return true; }
+      if (k != TILE_SKIP) { oj = j; oqt = (ZZ ? qh * Tq : 0) + qt - 1; return true; }
     }
     return false;
   }
@@ -301,7 +325,7 @@ __device__ __forceinline__ void dkdv_item(const BwdParams& p, int idx, int& bh, 
   else { kt = r / p.P; kb = r % p.P; }
 }
 
-template <int D>
+template <int D, bool ZZ>
 __global__ void __launch_bounds__(320, 1)
 bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -329,7 +353,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       load_tile<D>(sb + C::kFixed0, &tmK, bar + kBarFixed, y0, kb, bh);
       load_tile<D>(sb + C::kFixed1, &tmV, bar + kBarFixed, y0, kb, bh);
     }
-    QCursor cur;
+    QCursor<ZZ> cur;
     cur.init(p, kb, y0);
     uint32_t na = 0, nb = 0;   // tiles issued into ring A / ring B
     int j, qt;
@@ -389,7 +413,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     // of P_i right after the MMA that reads them (tcgen05 MMAs of one CTA
     // run in issue order), so the tensor core computes the next scores while
     // the element-wise warps finish dS_i and start on P_{i+1}.
-    QCursor cur;
+    QCursor<ZZ> cur;
     cur.init(p, kb, y0);
     int j, qt;
     bool ok = warp_wait(bar + kBarFixed, 0, abort_flag, p.timeout_ns);
@@ -455,16 +479,18 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t myS = tS + lane_off + 64 * wg, mydP = tdP + lane_off + 64 * wg;
     const uint64_t c2x2 = pk2(p.c2, p.c2);
-    QCursor cur;
+    QCursor<ZZ> cur;
     cur.init(p, kb, y0);
     int j, qt;
     uint32_t i = 0;
     bool ok = true;
     while (cur.next(j, qt)) {
       const uint32_t b = i & 1;
-      int lo = 0, hi = p.c - qt * kBM;          // visible query columns [lo, hi)
+      // visible query columns [lo, hi), in the block's (chunk pair's) rows
+      const int qx0 = qt * kBM - cur.xo, yl = y - cur.yo;
+      int lo = 0, hi = cur.mc() - qx0;
       if (cur.m.use_diag) {
-        const int l2 = y + 1 - cur.m.e - qt * kBM;   // query x sees key y iff y < x + e
+        const int l2 = yl + 1 - cur.m.e - qx0;   // query x sees key y iff y < x + e
         lo = l2 > 0 ? l2 : 0;
       }
       if (y >= p.c) hi = 0;
@@ -574,24 +600,40 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 // Work item: query tile qt of shard j of (b, h); key tiles of every block
 // that is not hidden, blocks in ascending order (the same order in every
 // CTA, for L2 reuse; the gradient is a sum), skipped tiles left out.
+template <bool ZZ>
 struct KCursor {
   int kb, kt, kend, P, c, j, striped, causal, x0;
   BlockMask bm;
   TileSpan sp;
+  int r, xo, yo, kt_off;    // zigzag: sub-round, chunk offsets, key tile offset
+  __device__ __forceinline__ int mc() const { return ZZ ? (c >> 1) : c; }
   __device__ void init(const BwdParams& p, int j_, int x0_) {
     kb = -1; kt = 0; kend = 0; P = p.P; c = p.c; j = j_; striped = p.striped; causal = p.causal;
     x0 = x0_;
+    r = -1; xo = 0; yo = 0; kt_off = 0;
   }
   __device__ bool next(int& okb, int& oy0, int& kind, BlockMask& m) {
     while (kt >= kend) {
-      if (++kb >= P) return false;
-      bm = block_mask(j, kb, striped, causal);
-      sp = tile_span(bm, x0, c);
+      if (ZZ) {
+        // sub-round r = 2 * block + chunk half of the key block
+        if (++r >= 2 * P) return false;
+        kb = r >> 1;
+        const int h = c >> 1, hk = r & 1;
+        xo = x0 < h ? 0 : h;
+        yo = hk * h;
+        bm = chunk_mask(zz_chunk(j, x0, h, P), hk ? 2 * P - 1 - kb : kb, causal);
+        sp = tile_span(bm, x0 - xo, h);
+        kt_off = hk * (h / kBN);
+      } else {
+        if (++kb >= P) return false;
+        bm = block_mask(j, kb, striped, causal);
+        sp = tile_span(bm, x0, c);
+      }
       kend = sp.part_end;
       kt = 0;
     }
     okb = kb;
-    oy0 = kt * kBN;
+    oy0 = ((ZZ ? kt_off : 0) + kt) * kBN;
     kind = tile_kind_at(sp, kt);
     m = bm;
     ++kt;
@@ -610,7 +652,7 @@ __device__ __forceinline__ void dq_item(const BwdParams& p, int idx, int& bh, in
   else { qt = p.T - 1 - r / p.P; j = r % p.P; }
 }
 
-template <int D>
+template <int D, bool ZZ>
 __global__ void __launch_bounds__(320, 1)
 bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -635,7 +677,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       mbar_arrive_expect_tx(bar + kBarFixed, 2 * C::kTile);
       load_tile<D>(sb + C::kFixed0, &tmQ, bar + kBarFixed, x0, j, bh);
       load_tile<D>(sb + C::kFixed1, &tmdO, bar + kBarFixed, x0, j, bh);
-      KCursor cur;
+      KCursor<ZZ> cur;
       cur.init(p, j, x0);
       uint32_t na = 0, nb = 0;
       int kb, y0, kind;
@@ -669,7 +711,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     // Order per key tile i: S_{i+1} = Q K_{i+1}^T as soon as the element-wise
     // warps have read S_i; dQ += dS_i K_i; dP_{i+1} = dO V_{i+1}^T into the
     // columns of dS_i right after the MMA that reads them.
-    KCursor cur;
+    KCursor<ZZ> cur;
     cur.init(p, j, x0);
     int kb, y0, kind;
     BlockMask bm;
@@ -738,7 +780,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const uint64_t c2x2 = pk2(p.c2, p.c2), nl2 = pk2(-lse2, -lse2), d2 = pk2(drow, drow);
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t myS = tS + lane_off + 64 * wg, mydP = tdP + lane_off + 64 * wg;
-    KCursor cur;
+    KCursor<ZZ> cur;
     cur.init(p, j, x0);
     int kb, y0, kind;
     BlockMask bm;
@@ -746,7 +788,8 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     bool ok = true;
     while (cur.next(kb, y0, kind, bm)) {
       const int lim =
-          (xvalid ? ((kind == TILE_PARTIAL) ? row_limit(bm, x, y0, p.c) : kBN) : 0) - 64 * wg;
+          (xvalid ? ((kind == TILE_PARTIAL) ? row_limit(bm, x - cur.xo, y0 - cur.yo, cur.mc()) : kBN)
+                  : 0) - 64 * wg;
       const bool all_vis = __all_sync(0xffffffffu, lim >= 64) != 0;
       if (!warp_wait(bar + kBarS, i & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
       tc_fence_after();
@@ -829,7 +872,7 @@ static bool encode_map(CUtensorMap* map, const void* base, int64_t BH, int64_t N
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D>
+template <int D, bool ZZ>
 static ra_status launch_bwd(const BwdLaunch& a) {
   using C = BwdCfg<D>;
   const int64_t c = a.N / a.P;
@@ -839,9 +882,9 @@ static ra_status launch_bwd(const BwdLaunch& a) {
     return RA_ERR_CUDA;
   static int attr_set[64] = {0};
   if (a.device < 64 && !attr_set[a.device]) {
-    if (cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(bwd_dkdv_kernel<D, ZZ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmem) != cudaSuccess ||
-        cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(bwd_dq_kernel<D, ZZ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmem) != cudaSuccess)
       return RA_ERR_CUDA;
     attr_set[a.device] = 1;
@@ -860,6 +903,7 @@ static ra_status launch_bwd(const BwdLaunch& a) {
   p.P = a.P;
   p.T = (int)((c + kBM - 1) / kBM);
   p.striped = a.striped;
+  p.zigzag = a.zigzag;
   p.causal = a.causal;
   p.c2 = (float)((double)a.scale * 1.4426950408889634074);
   p.scale = a.scale;
@@ -872,14 +916,19 @@ static ra_status launch_bwd(const BwdLaunch& a) {
   if (blocks > (long long)a.num_sms * 16) blocks = (long long)a.num_sms * 16;
   bwd_rowdot_kernel<D><<<(int)blocks, 256, 0, st>>>(p.o, p.dout, p.dvec, rows);
   const long long items = (long long)p.BH * p.P * p.T;
-  bwd_dkdv_kernel<D><<<(unsigned)items, C::kThreads, C::kSmem, st>>>(tq, tk, tv, tdo, p);
-  bwd_dq_kernel<D><<<(unsigned)items, C::kThreads, C::kSmem, st>>>(tq, tk, tv, tdo, p);
+  bwd_dkdv_kernel<D, ZZ><<<(unsigned)items, C::kThreads, C::kSmem, st>>>(tq, tk, tv, tdo, p);
+  bwd_dq_kernel<D, ZZ><<<(unsigned)items, C::kThreads, C::kSmem, st>>>(tq, tk, tv, tdo, p);
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
 ra_status attn_bwd_launch(const BwdLaunch& a) {
-  if (a.d == 128) return launch_bwd<128>(a);
-  if (a.d == 64) return launch_bwd<64>(a);
+  if (a.zigzag) {
+    if (a.d == 128) return launch_bwd<128, true>(a);
+    if (a.d == 64) return launch_bwd<64, true>(a);
+  } else {
+    if (a.d == 128) return launch_bwd<128, false>(a);
+    if (a.d == 64) return launch_bwd<64, false>(a);
+  }
   return RA_ERR_HEADDIM;
 }
 

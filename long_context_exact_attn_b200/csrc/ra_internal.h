@@ -52,6 +52,7 @@ struct BwdLaunch {
   float scale;
   int device, num_sms;
   void* stream;
+  int zigzag = 0;                // zigzag layout (striped == 0)
 };
 
 ra_status attn_bwd_launch(const BwdLaunch& a);

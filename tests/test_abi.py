@@ -208,7 +208,7 @@ def test_host_workspace_formula(L):
 @pytest.mark.parametrize("fn,kw,code", [
     ("fwd", dict(layout=2, N=1024, P=4), 3),          # c = 256: not a multiple of 512
     ("fwd", dict(layout=2, N=2048, P=4), None),       # valid sizes: passes validation
-    ("bwd", dict(layout=2), 5),                        # backward: contiguous / striped only
+    ("bwd", dict(layout=2), 3),                        # zigzag backward: c = 256 too short
 ])
 def test_zigzag_validation(L, fn, kw, code):
     if fn == "fwd":

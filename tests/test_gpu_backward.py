@@ -33,12 +33,12 @@ def _lib():
 
 def run_bwd(q, k, v, do, P, layout, causal):
     dev = [t.cuda() for t in (q, k, v, do)]
-    if layout == W.STRIPED:
+    if layout != W.CONTIGUOUS:
         dev = [ops.partition(t, P, layout) for t in dev]
     dq_, dk_, dv_, ddo = dev
     o, lse = ops.attn_fwd(dq_, dk_, dv_, P, layout, causal)
     gq, gk, gv = ops.attn_bwd(dq_, dk_, dv_, o, ddo, lse, P, layout, causal)
-    if layout == W.STRIPED:
+    if layout != W.CONTIGUOUS:
         gq, gk, gv = (ops.partition(t, P, layout, inverse=True) for t in (gq, gk, gv))
     torch.cuda.synchronize()
     assert ops.device_fault() == 0
@@ -66,11 +66,14 @@ CASES = [
     (1, 1, 4096, 128, 8, W.STRIPED, True, 3.0),       # 4 key tiles per shard
     (1, 1, 4096, 128, 4, W.CONTIGUOUS, True, 1.0),
     (1, 1, 3000, 64, 3, W.CONTIGUOUS, False, 1.0),    # ragged, non-causal
+    (1, 2, 4096, 128, 4, W.ZIGZAG, True, 1.0),         # zigzag: chunks j and 2P-1-j
+    (2, 1, 2048, 64, 2, W.ZIGZAG, True, 3.0),
+    (1, 1, 4096, 128, 8, W.ZIGZAG, False, 1.0),
 ]
 
 
 @pytest.mark.parametrize("case", CASES, ids=lambda c: "B{}H{}N{}d{}P{}{}{}x{}".format(
-    c[0], c[1], c[2], c[3], c[4], "s" if c[5] else "c", "C" if c[6] else "F", c[7]))
+    c[0], c[1], c[2], c[3], c[4], "csz"[c[5]], "C" if c[6] else "F", c[7]))
 def test_backward_parity(case):
     B, H, N, d, P, layout, causal, up = case
     w = W.Workload("bwd", B, H, N, d, P, layout, causal, seed=N + 7 * P, qk_scale_up=up)
