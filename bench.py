@@ -257,18 +257,37 @@ def job_value(flops_per_rank, ms_max, world):
     return flops_per_rank * world / (ms_max * 1e-3) / 1e12
 
 
-def timed(fn, steps, world):
+L2_BYTES = 126 * 2 ** 20
+
+
+def timed(fn, steps, world, flush=None):
+    """Mean device time of fn over `steps` runs, max over ranks.  With
+    `flush`, L2 is overwritten before every run and each run is timed on its
+    own, so the flush stays outside the timed windows."""
     barrier(world)
     torch.cuda.synchronize()
     s = torch.cuda.current_stream()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(s)
-    for _ in range(steps):
-        fn()
-    e1.record(s)
-    torch.cuda.synchronize()
+    if flush is None:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for _ in range(steps):
+            fn()
+        e1.record(s)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+    else:
+        evs = []
+        for _ in range(steps):
+            flush()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            fn()
+            e1.record(s)
+            evs.append((e0, e1))
+        torch.cuda.synchronize()
+        ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
     barrier(world)
-    return max_over_ranks(e0.elapsed_time(e1) / steps, world)
+    return max_over_ranks(ms, world)
 
 
 def main():
@@ -319,6 +338,17 @@ def main():
 
     q, k, v = W.make_qkv(w)
     path = Path(ops, w, q, k, v, sched_free=(args.sched == "free"))
+    # Inputs smaller than a few L2s: overwrite L2 before every timed step.
+    in_bytes = 3 * q.numel() * q.element_size()
+    flush = None
+    if in_bytes < 4 * L2_BYTES:
+        flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+        flush = flush_buf.zero_
+        l2_note = (f"inputs ({in_bytes / 2 ** 20:.0f} MiB) not much larger than L2: a "
+                   f"{2 * L2_BYTES / 2 ** 20:.0f} MiB buffer is written before every timed step, "
+                   f"outside the timed window")
+    else:
+        l2_note = f"inputs ({in_bytes / 2 ** 30:.1f} GiB) larger than L2; no flush"
 
     for _ in range(args.warmup):
         path.step()
@@ -328,7 +358,7 @@ def main():
 
     sampler = ClockSampler(local)
     sampler.start()
-    ms = timed(lambda: path.step(time_attn=True), args.steps, world)
+    ms = timed(lambda: path.step(time_attn=True), args.steps, world, flush=flush)
     clocks = sampler.stop()
     attn_ts = path.attn_ms()
     if ops.device_fault():
@@ -384,6 +414,8 @@ def main():
                     torch.cuda.synchronize()
                 n = 3
                 for _ in range(n):
+                    if flush is not None:
+                        flush()
                     pth.step(time_attn=True)
                 t = statistics.median(pth.attn_ms())
                 t = max_over_ranks(t, world)
@@ -416,7 +448,7 @@ def main():
 
         bwd_step()
         torch.cuda.synchronize()
-        bms = timed(bwd_step, max(1, min(args.steps, 3)), world)
+        bms = timed(bwd_step, max(1, min(args.steps, 3)), world, flush=flush)
         if ops.device_fault():
             raise RuntimeError("device fault during the backward pass")
         # useful: 10 d FLOP per visible pair (the five products of the
@@ -493,7 +525,7 @@ def main():
             ops.partition_rope(path.q, w.P, w.layout, 10000.0, ops.ROPE_HALF, out=dst)
 
         rope_step()
-        rms = timed(rope_step, 5, world)
+        rms = timed(rope_step, 5, world, flush=flush)
         hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
         moved = 2 * path.q.numel() * path.q.element_size()   # read + write
         rope = {"kernel": "partition_rope_kernel<1>", "ms": rms, "bytes": moved,
@@ -522,6 +554,7 @@ def main():
                                                                  FALLBACK_PEAKS["bf16_tflops"])),
                 "frac_of_spec_2250": achieved / SPEC_BF16_TFLOPS,
                 "attn_ms_per_launch": attn_ms,
+                "attn_ms_median": statistics.median(attn_ts), "attn_ms_min": min(attn_ts),
                 "useful_flops_per_launch": flops}
 
     line = {
@@ -532,7 +565,7 @@ def main():
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "P": w.P,
                    "layout": w.layout_name, "causal": w.causal, "schedule": args.sched,
                    "step": "partition q,k,v -> attention -> unpartition o,lse",
-                   "l2": "inputs (3 GiB) larger than L2; no flush",
+                   "l2": l2_note,
                    "parallelism": f"replicas x{world}"},
         "tokens_per_s": tokens_s,
         "frac_of_peak": value / world / peak,
