@@ -92,6 +92,11 @@ typedef int ra_status;
  * load-balanced schedule; same results, same tile skipping). */
 #define RA_SCHED_FREE 0x100
 
+/* Optional output flag for ra_attn_fwd, OR-ed into `layout`: O is written as
+ * float32 [B, H, N, d] (o must hold 4 bytes per element) instead of bf16,
+ * e.g. for callers that merge partial results or want O before rounding. */
+#define RA_O_F32 0x200
+
 /* Rotation pairs of ra_partition_rope. */
 #define RA_ROPE_INTERLEAVED 0 /* pair i = dimensions (2i, 2i+1)                */
 #define RA_ROPE_HALF 1        /* pair i = dimensions (i, i + d/2)              */
@@ -171,19 +176,20 @@ ra_status ra_partition_rope(const void* src, void* dst, int64_t B, int64_t H, in
  *
  *   q, k, v  device, [B, H, N, d] bf16, rows already in LAYOUT order (see
  *            ra_partition), 16-byte aligned.
- *   o        device, [B, H, N, d] bf16 output, layout order, 16-byte aligned.
- *            Must not overlap q, k, v.
+ *   o        device, [B, H, N, d] bf16 output (float32 with RA_O_F32),
+ *            layout order, 16-byte aligned.  Must not overlap q, k, v.
  *   lse      device, [B, H, N] float32 output, layout order, 16-byte aligned.
  *   d        64 or 128.
  *   N, P     1 <= P, N % P == 0, c = N / P <= 2^30 / 128; any c (a ragged
  *            last tile of a shard is masked).  B*H*N < 2^31.
- *   layout   RA_CONTIGUOUS or RA_STRIPED, optionally | RA_SCHED_FREE.
+ *   layout   RA_CONTIGUOUS, RA_STRIPED or RA_ZIGZAG (N/P a multiple of
+ *            512), optionally | RA_SCHED_FREE and/or | RA_O_F32.
  *   causal   0: no mask (the layout then only permutes rows); else causal in
  *            original token order.
  *   scale    > 0 and finite; 1/sqrt(d) is the usual value.
  * Arithmetic: bf16 operands, fp32 accumulation of Q K^T and P V on the
  * tensor cores, fp32 softmax statistics, probabilities rounded to bf16 for
- * the P V product, O rounded to bf16 once at the end.
+ * the P V product, O rounded to bf16 once at the end (not with RA_O_F32).
  */
 ra_status ra_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                       int64_t B, int64_t H, int64_t N, int64_t d, int P, int layout,

@@ -199,7 +199,7 @@ ra_status ra_attn_fwd(const void* q, const void* k, const void* v, void* o, floa
                       int64_t B, int64_t H, int64_t N, int64_t d, int P, int layout, int causal,
                       float scale, void* stream) {
   if (!q || !k || !v || !o || !lse) return RA_ERR_NULL;
-  if (layout & ~(0xff | RA_SCHED_FREE)) return RA_ERR_LAYOUT;
+  if (layout & ~(0xff | RA_SCHED_FREE | RA_O_F32)) return RA_ERR_LAYOUT;
   const int base = layout & 0xff;
   if (base != RA_CONTIGUOUS && base != RA_STRIPED && base != RA_ZIGZAG) return RA_ERR_LAYOUT;
   if (d != 64 && d != 128) return RA_ERR_HEADDIM;
@@ -211,10 +211,11 @@ ra_status ra_attn_fwd(const void* q, const void* k, const void* v, void* o, floa
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
       !aligned(lse, 16))
     return RA_ERR_ALIGN;
-  const int64_t tb = B * H * N * d * 2, lb = B * H * N * 4;
-  if (overlap(o, tb, q, tb) || overlap(o, tb, k, tb) || overlap(o, tb, v, tb) ||
+  const bool o_f32 = (layout & RA_O_F32) != 0;
+  const int64_t tb = B * H * N * d * 2, ob = o_f32 ? 2 * tb : tb, lb = B * H * N * 4;
+  if (overlap(o, ob, q, tb) || overlap(o, ob, k, tb) || overlap(o, ob, v, tb) ||
       overlap(lse, lb, q, tb) || overlap(lse, lb, k, tb) || overlap(lse, lb, v, tb) ||
-      overlap(lse, lb, o, tb))
+      overlap(lse, lb, o, ob))
     return RA_ERR_ALIAS;
   int dev;
   DevInfo info;
@@ -227,6 +228,7 @@ ra_status ra_attn_fwd(const void* q, const void* k, const void* v, void* o, floa
   a.zigzag = base == RA_ZIGZAG;
   a.causal = causal != 0;
   a.sched_free = (layout & RA_SCHED_FREE) != 0;
+  a.o_f32 = o_f32;
   a.scale = scale;
   a.device = dev;
   a.num_sms = info.num_sms;

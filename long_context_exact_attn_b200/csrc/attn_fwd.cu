@@ -45,6 +45,7 @@ __device__ unsigned int g_device_fault = 0;
 struct AttnParams {
   __nv_bfloat16* o;
   float* lse;
+  int o_f32;          // O written as float32 (o then points to float rows)
   int BH;             // B * H
   int N;              // sequence length
   int c;              // shard length N / P
@@ -692,7 +693,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
           for (int i = 0; i < 32; ++i) orow[i] = 0u;
         }
-        if (valid) {
+        if (valid && p.o_f32) {
+          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.o) + grow * D + q * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(__uint_as_float(orow[4 * i]) * inv_l,
+                                 __uint_as_float(orow[4 * i + 1]) * inv_l,
+                                 __uint_as_float(orow[4 * i + 2]) * inv_l,
+                                 __uint_as_float(orow[4 * i + 3]) * inv_l);
+        } else if (valid) {
           uint32_t w[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
@@ -754,6 +763,7 @@ static ra_status launch(const AttnLaunch& a) {
   }
   AttnParams p;
   p.o = reinterpret_cast<__nv_bfloat16*>(a.o);
+  p.o_f32 = a.o_f32;
   p.lse = a.lse;
   p.BH = (int)a.BH;
   p.N = (int)a.N;

@@ -19,6 +19,7 @@ CONTIGUOUS = 0
 STRIPED = 1
 ZIGZAG = 2
 SCHED_FREE = 0x100
+O_F32 = 0x200
 
 BF16 = 0
 F32 = 1
@@ -132,10 +133,11 @@ def partition(x, P, layout, inverse=False, out=None):
     return out
 
 
-def attn_fwd(q, k, v, P, layout, causal=True, scale=None, sched_free=False, out=None, lse=None):
+def attn_fwd(q, k, v, P, layout, causal=True, scale=None, sched_free=False, out=None, lse=None,
+             o_f32=False):
     """Exact blockwise attention forward; q, k, v: [B, H, N, d] bf16 CUDA
-    tensors in LAYOUT order.  Returns (o [B, H, N, d] bf16, lse [B, H, N]
-    float32), both in layout order."""
+    tensors in LAYOUT order.  Returns (o [B, H, N, d] bf16, or float32 with
+    ``o_f32``, lse [B, H, N] float32), both in layout order."""
     for n, t in (("q", q), ("k", k), ("v", v)):
         _cuda_contig(t, n)
         if t.dtype != torch.bfloat16:
@@ -145,17 +147,18 @@ def attn_fwd(q, k, v, P, layout, causal=True, scale=None, sched_free=False, out=
     B, H, N, d = q.shape
     if scale is None:
         scale = d ** -0.5
+    odt = torch.float32 if o_f32 else torch.bfloat16
     if out is None:
-        out = torch.empty_like(q)
+        out = torch.empty(q.shape, dtype=odt, device=q.device)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    if out.shape != q.shape or out.dtype != torch.bfloat16:
-        raise ValueError("out must be bf16 of q's shape")
+    if out.shape != q.shape or out.dtype != odt:
+        raise ValueError(f"out must be {odt} of q's shape")
     if lse.shape != (B, H, N) or lse.dtype != torch.float32:
         raise ValueError("lse must be float32 [B, H, N]")
     _cuda_contig(out, "out")
     _cuda_contig(lse, "lse")
-    lay = int(layout) | (SCHED_FREE if sched_free else 0)
+    lay = int(layout) | (SCHED_FREE if sched_free else 0) | (O_F32 if o_f32 else 0)
     _check(lib().ra_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, d, int(P),
                              lay, int(bool(causal)), float(scale), _stream(q)), "ra_attn_fwd")
     return out, lse

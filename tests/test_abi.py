@@ -68,7 +68,7 @@ def attn(L, q=A, k=Bp, v=Cp, o=Op, lse=Lp, B=1, H=2, N=1024, d=128, P=4, layout=
     (dict(q=A + 8), 2), (dict(o=Op + 2), 2), (dict(lse=Lp + 4), 2),
     (dict(N=1000, P=3), 3), (dict(P=0), 3), (dict(N=0), 3), (dict(B=0), 3),
     (dict(d=96), 4), (dict(d=256), 4),
-    (dict(layout=3), 5), (dict(layout=0x400), 5),
+    (dict(layout=3), 5), (dict(layout=0x400), 5), (dict(layout=0x1201), 5),
     (dict(scale=0.0), 6), (dict(scale=float("inf")), 6), (dict(scale=float("nan")), 6),
     (dict(scale=-1.0), 6),
     (dict(o=A), 8), (dict(lse=Op + 64), 8),
@@ -223,3 +223,10 @@ def test_zigzag_validation(L, fn, kw, code):
 
 def test_zigzag_partition_needs_even_shards(L):
     assert L.ra_partition(vp(A), vp(Bp), 1, 1, 600, 8, 200, 2, 0, 0, None) == 3   # c = 3
+
+
+def test_o_f32_flag_validation(L):
+    # float32 O is twice the size: an o that overlaps q only in its second half
+    tb = 2 * 1024 * 128 * 2
+    assert attn(L, o=A - tb - tb // 2, layout=0x201) == 8
+    assert attn(L, o=A - tb - tb // 2, layout=0x001) != 8

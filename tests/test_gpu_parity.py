@@ -329,3 +329,24 @@ def test_lse_merge_of_split_keys_equals_full_attention():
                                                   k[0, h].double().numpy(),
                                                   v[0, h].double().numpy(), w.scale, False)
     assert_close(om.float().cpu().numpy(), lm.cpu().numpy(), o_ref, lse_ref, "merged halves")
+
+
+@pytest.mark.parametrize("layout", [W.STRIPED, W.CONTIGUOUS])
+def test_o_f32_output_rounds_to_the_bf16_output(layout):
+    """RA_O_F32 writes the same O before its final rounding: rounding it to
+    bf16 (nearest even) gives the bf16 output bit for bit, lse identical, and
+    it is at least as close to the oracle."""
+    w = W.Workload("of32", 1, 2, 2048, 128, 4, layout, True, 13, qk_scale_up=3.0)
+    q, k, v = W.make_qkv(w)
+    dq, dk, dv = (t.cuda() for t in (q, k, v))
+    o16, l16 = ops.attn_fwd(dq, dk, dv, w.P, layout, True)
+    o32, l32 = ops.attn_fwd(dq, dk, dv, w.P, layout, True, o_f32=True)
+    torch.cuda.synchronize()
+    assert o32.dtype == torch.float32
+    assert torch.equal(o32.to(torch.bfloat16), o16)
+    assert torch.equal(l32, l16)
+    perm = OP.slot_to_token(w.N, w.P, LAYOUT[layout])
+    o_ref, _ = oracle_full(q, k, v, True, w.scale)
+    e32 = np.abs(o32.cpu().numpy()[:, :, np.argsort(perm)] - o_ref).mean()
+    e16 = np.abs(o16.float().cpu().numpy()[:, :, np.argsort(perm)] - o_ref).mean()
+    assert e32 <= e16
