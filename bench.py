@@ -398,6 +398,24 @@ def main():
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "api": "ra_attn_fwd_host (pinned host buffers)", "heads_per_chunk": g}
 
+    # ---- the same step with the layout's permutation applied inside the
+    # attention kernel (RA_TOKEN_ORDER: one launch, token order in and out)
+    fused = None
+    if not args.no_compare and path.layout != W.CONTIGUOUS:
+        fo, fl = torch.empty_like(path.o), torch.empty_like(path.lse)
+
+        def fused_step():
+            ops.attn_fwd(path.q, path.k, path.v, w.P, path.layout, w.causal,
+                         sched_free=path.sched_free, out=fo, lse=fl, token_order=True)
+
+        fused_step()
+        fms = timed(fused_step, max(1, min(args.steps, 5)), world, flush=flush)
+        fused = {"ms_per_step": fms, "useful_tflops": flops * world / (fms * 1e-3) / 1e12,
+                 "launches_per_step": 1,
+                 "note": "partition and un-partition folded into the kernel's TMA "
+                         "coordinates and epilogue rows (bit-identical results)"}
+        del fo, fl
+
     # ---- the layout/schedule comparison at equal shapes (attention only)
     compare = None
     if not args.no_compare:
@@ -575,6 +593,7 @@ def main():
         "cpu_baseline": cpu,
         "e2e": e2e,
         "layout_compare": compare,
+        "token_order_step": fused,
         "backward": backward,
         "rope_partition": rope,
         "ring_emulation": ring,

@@ -97,6 +97,14 @@ typedef int ra_status;
  * e.g. for callers that merge partial results or want O before rounding. */
 #define RA_O_F32 0x200
 
+/* Optional flag for ra_attn_fwd, OR-ed into `layout`: q, k, v, o and lse
+ * are in TOKEN order.  The layout's permutation is then applied inside the
+ * kernel (the TMA loads address shard j's rows where the tokens live, the
+ * epilogue writes each row to its token position), so no ra_partition pass
+ * is needed before or after; results equal the partition / attention /
+ * inverse-partition sequence bit for bit. */
+#define RA_TOKEN_ORDER 0x400
+
 /* Rotation pairs of ra_partition_rope. */
 #define RA_ROPE_INTERLEAVED 0 /* pair i = dimensions (2i, 2i+1)                */
 #define RA_ROPE_HALF 1        /* pair i = dimensions (i, i + d/2)              */
@@ -183,7 +191,8 @@ ra_status ra_partition_rope(const void* src, void* dst, int64_t B, int64_t H, in
  *   N, P     1 <= P, N % P == 0, c = N / P <= 2^30 / 128; any c (a ragged
  *            last tile of a shard is masked).  B*H*N < 2^31.
  *   layout   RA_CONTIGUOUS, RA_STRIPED or RA_ZIGZAG (N/P a multiple of
- *            512), optionally | RA_SCHED_FREE and/or | RA_O_F32.
+ *            512), optionally | RA_SCHED_FREE, | RA_O_F32, | RA_TOKEN_ORDER
+ *            (then q, k, v, o, lse are in token order).
  *   causal   0: no mask (the layout then only permutes rows); else causal in
  *            original token order.
  *   scale    > 0 and finite; 1/sqrt(d) is the usual value.
@@ -254,7 +263,9 @@ ra_status ra_attn_bwd_noalloc(const void* q, const void* k, const void* v, const
  * Same computation and results as ra_partition + ra_attn_fwd + ra_partition
  * (inverse) on device copies (bit-identical: every (b, h) is computed alone).
  * The heads are processed in chunks through two staging slots of the
- * caller's device workspace: the host-to-device copy of chunk i+1 and the
+ * caller's device workspace (each chunk runs the attention with
+ * RA_TOKEN_ORDER, so only q, k, v, o, lse are staged): the host-to-device
+ * copy of chunk i+1 and the
  * device-to-host copy of chunk i-1 run on the library's own copy streams
  * while chunk i computes on `stream`.  Host buffers should be page-locked
  * (pinned) for the copies to overlap.

@@ -64,23 +64,21 @@ bool overlap(const void* a, int64_t na, const void* b, int64_t nb) {
 
 // ------------------------------------------------------------ host path
 // Device staging of ra_attn_fwd_host: two slots, each holding a chunk of G
-// heads: q, k, v (token order), for the striped layout also qp, kp, vp, op
-// (layout order) and lsep, then o and lse (token order).
+// heads: q, k, v, o and lse, all in token order (the attention applies the
+// layout's permutation in its own addressing).
 struct HostPlan {
   int64_t tok;      // bytes of one [N, d] bf16 head
   int64_t lsz;      // bytes of one [N] float32 head
   int64_t per_head; // staging bytes per head per slot (256-byte rounded parts)
-  bool striped;
 };
 
 int64_t round256(int64_t x) { return (x + 255) / 256 * 256; }
 
-HostPlan host_plan(int64_t N, int64_t d, bool striped) {
+HostPlan host_plan(int64_t N, int64_t d) {
   HostPlan h;
   h.tok = N * d * 2;
   h.lsz = N * 4;
-  h.striped = striped;
-  h.per_head = (striped ? 8 : 4) * round256(h.tok) + (striped ? 2 : 1) * round256(h.lsz);
+  h.per_head = 4 * round256(h.tok) + round256(h.lsz);
   return h;
 }
 
@@ -199,7 +197,7 @@ ra_status ra_attn_fwd(const void* q, const void* k, const void* v, void* o, floa
                       int64_t B, int64_t H, int64_t N, int64_t d, int P, int layout, int causal,
                       float scale, void* stream) {
   if (!q || !k || !v || !o || !lse) return RA_ERR_NULL;
-  if (layout & ~(0xff | RA_SCHED_FREE | RA_O_F32)) return RA_ERR_LAYOUT;
+  if (layout & ~(0xff | RA_SCHED_FREE | RA_O_F32 | RA_TOKEN_ORDER)) return RA_ERR_LAYOUT;
   const int base = layout & 0xff;
   if (base != RA_CONTIGUOUS && base != RA_STRIPED && base != RA_ZIGZAG) return RA_ERR_LAYOUT;
   if (d != 64 && d != 128) return RA_ERR_HEADDIM;
@@ -229,6 +227,7 @@ ra_status ra_attn_fwd(const void* q, const void* k, const void* v, void* o, floa
   a.causal = causal != 0;
   a.sched_free = (layout & RA_SCHED_FREE) != 0;
   a.o_f32 = o_f32;
+  a.tok = (layout & RA_TOKEN_ORDER) != 0;
   a.scale = scale;
   a.device = dev;
   a.num_sms = info.num_sms;
@@ -397,7 +396,8 @@ ra_status ra_lse_merge_acc(float* o_acc, float* lse_acc, const void* o_b, const 
 
 int64_t ra_attn_fwd_host_workspace(int64_t N, int64_t d, int layout, int64_t heads_per_chunk) {
   if (N < 1 || d < 1 || heads_per_chunk < 1) return -1;
-  const HostPlan h = host_plan(N, d, (layout & 0xff) != RA_CONTIGUOUS);
+  (void)layout;
+  const HostPlan h = host_plan(N, d);
   return 2 * heads_per_chunk * h.per_head;
 }
 
@@ -415,8 +415,7 @@ ra_status ra_attn_fwd_host(const void* q, const void* k, const void* v, void* o,
   if (B * H * N >= ((int64_t)1 << 31) || N / P > ((int64_t)1 << 30) / 128) return RA_ERR_SHAPE;
   if (!(scale > 0.f) || !isfinite(scale)) return RA_ERR_SCALE;
   if (!aligned(workspace, 256)) return RA_ERR_ALIGN;
-  const bool striped = base != RA_CONTIGUOUS;   // a permuted layout: stage both orders
-  const HostPlan hp = host_plan(N, d, striped);
+  const HostPlan hp = host_plan(N, d);
   const int64_t BH = B * H;
   int64_t G = workspace_bytes / (2 * hp.per_head);
   if (G < 1) return RA_ERR_WORKSPACE;
@@ -438,23 +437,15 @@ ra_status ra_attn_fwd_host(const void* q, const void* k, const void* v, void* o,
       !chk(cudaStreamWaitEvent(hs->out, hs->entry, 0)))
     return RA_ERR_CUDA;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const int64_t T = round256(hp.tok) * G, L = round256(hp.lsz) * G;
+  const int64_t T = round256(hp.tok) * G;
   const int64_t nch = (BH + G - 1) / G;
   for (int64_t i = 0; i < nch; ++i) {
     const int s = (int)(i & 1);
     const int64_t h0 = i * G, g = (BH - h0 < G) ? BH - h0 : G;
     const int64_t tb = g * hp.tok, lb = g * hp.lsz;
     uint8_t* slot = ws + s * G * hp.per_head;
-    uint8_t *dq = slot, *dk = dq + T, *dv = dk + T, *dqp = nullptr, *dkp = nullptr, *dvp = nullptr,
-            *dop = nullptr, *dlp = nullptr;
-    uint8_t* cur = dv + T;
-    if (striped) {
-      dqp = cur; dkp = dqp + T; dvp = dkp + T; dop = dvp + T; cur = dop + T;
-    }
-    uint8_t* dout = cur;
-    cur += T;
-    if (striped) { dlp = cur; cur += L; }
-    float* dl = reinterpret_cast<float*>(cur);
+    uint8_t *dq = slot, *dk = dq + T, *dv = dk + T, *dout = dv + T;
+    float* dl = reinterpret_cast<float*>(dout + T);
     // inputs of chunk i (the slot's previous chunk has been read back)
     if (i >= 2 && !chk(cudaStreamWaitEvent(hs->in, hs->d2h[s], 0))) return RA_ERR_CUDA;
     const uint8_t* hq = static_cast<const uint8_t*>(q) + h0 * hp.tok;
@@ -477,21 +468,9 @@ ra_status ra_attn_fwd_host(const void* q, const void* k, const void* v, void* o,
     a.device = dev;
     a.num_sms = info.num_sms;
     a.stream = stream;
-    const int64_t row = d * 2;
-    if (striped) {
-      if ((st = partition_launch(dq, dqp, g, N, P, row, base, 0, stream)) ||
-          (st = partition_launch(dk, dkp, g, N, P, row, base, 0, stream)) ||
-          (st = partition_launch(dv, dvp, g, N, P, row, base, 0, stream)))
-        return st;
-      a.q = dqp; a.k = dkp; a.v = dvp; a.o = dop; a.lse = reinterpret_cast<float*>(dlp);
-      if ((st = attn_fwd_launch(a))) return st;
-      if ((st = partition_launch(dop, dout, g, N, P, row, base, 1, stream)) ||
-          (st = partition_launch(dlp, dl, g, N, P, 4, base, 1, stream)))
-        return st;
-    } else {
-      a.q = dq; a.k = dk; a.v = dv; a.o = dout; a.lse = dl;
-      if ((st = attn_fwd_launch(a))) return st;
-    }
+    a.q = dq; a.k = dk; a.v = dv; a.o = dout; a.lse = dl;
+    a.tok = 1;
+    if ((st = attn_fwd_launch(a))) return st;
     if (!chk(cudaEventRecord(hs->comp[s], cs))) return RA_ERR_CUDA;
     // results of chunk i back to the host
     if (!chk(cudaStreamWaitEvent(hs->out, hs->comp[s], 0)) ||

@@ -46,6 +46,8 @@ struct AttnParams {
   __nv_bfloat16* o;
   float* lse;
   int o_f32;          // O written as float32 (o then points to float rows)
+  int tok;            // q, k, v, o, lse in token order: the layout's permutation
+                      // is applied in the TMA coordinates and the epilogue
   int BH;             // B * H
   int N;              // sequence length
   int c;              // shard length N / P
@@ -315,6 +317,46 @@ __device__ __forceinline__ void mma_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_
 #endif
 constexpr int kPolyEvery = RA_POLY_EVERY;
 
+// TMA coordinates (second, third) of the 128-row tile of shard `shard`
+// starting at local row x0.  Layout order: (x0, shard) of a [BH, P, c, d]
+// map.  Token order: striped rows are token x*P + shard, read through a
+// [BH, c, P, d] map as (shard, x0); zigzag rows lie in chunk shard or
+// 2P-1-shard of a [BH, 2P, h, d] map; contiguous token order is layout order.
+template <bool ZZ>
+__device__ __forceinline__ void tile_coord(const AttnParams& p, int shard, int x0, int& c1,
+                                           int& c2) {
+  c1 = x0;
+  c2 = shard;
+  if (!p.tok) return;
+  if (p.striped) {
+    c1 = shard;
+    c2 = x0;
+  } else if (ZZ) {
+    const int h = p.c >> 1;
+    if (x0 >= h) {
+      c1 = x0 - h;
+      c2 = 2 * p.P - 1 - shard;
+    }
+  }
+}
+
+// Row of (shard j, local row x) in the output tensors' order.
+template <bool ZZ>
+__device__ __forceinline__ size_t out_row(const AttnParams& p, int bh, int j, int x) {
+  size_t t;
+  if (!p.tok) {
+    t = (size_t)j * p.c + x;
+  } else if (p.striped) {
+    t = (size_t)x * p.P + j;
+  } else if (ZZ) {
+    const int h = p.c >> 1;
+    t = x < h ? (size_t)j * h + x : (size_t)(2 * p.P - 1 - j) * h + (x - h);
+  } else {
+    t = (size_t)j * p.c + x;
+  }
+  return (size_t)bh * p.N + t;
+}
+
 template <int D, bool ZZ>
 __global__ void __launch_bounds__(320, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -385,10 +427,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (!mbar_wait(bar_q_empty, (k & 1) ^ 1, abort_flag, p.timeout_ns)) { ok = false; break; }
         mbar_arrive_expect_tx(bar_q_full, 2 * C::kTileBytes);
         const int x0 = it.pair * 2 * kBM;
-        for (int t = 0; t < 2; ++t)
+        for (int t = 0; t < 2; ++t) {
+          int c1, c2;
+          tile_coord<ZZ>(p, it.j, x0 + t * kBM, c1, c2);
           for (int ch = 0; ch < C::kChunks; ++ch)
-            tma_load_4d(sQ + t * C::kTileBytes + ch * 16384, &tmQ, bar_q_full, ch * 64,
-                        x0 + t * kBM, it.j, it.bh);
+            tma_load_4d(sQ + t * C::kTileBytes + ch * 16384, &tmQ, bar_q_full, ch * 64, c1, c2,
+                        it.bh);
+        }
         TileSeq<ZZ> seq;
         seq.init(p, it);
         int kb, y0, k0, k1;
@@ -400,9 +445,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             if (!mbar_wait(bar_empty(s), ph ^ 1, abort_flag, p.timeout_ns)) { ok = false; break; }
             mbar_arrive_expect_tx(bar_full(s), C::kTileBytes);
             const CUtensorMap* tm = kv ? &tmV : &tmK;
+            int c1, c2;
+            tile_coord<ZZ>(p, kb, y0, c1, c2);
             for (int ch = 0; ch < C::kChunks; ++ch)
-              tma_load_4d(sRing + s * C::kTileBytes + ch * 16384, tm, bar_full(s), ch * 64, y0,
-                          kb, it.bh);
+              tma_load_4d(sRing + s * C::kTileBytes + ch * 16384, tm, bar_full(s), ch * 64, c1,
+                          c2, it.bh);
             ++n_loads;
           }
           if (!ok) break;
@@ -682,7 +729,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       // a row that saw no key (possible only for a single block) gets O = 0
       // and lse = -inf; its O columns in TMEM were never written
       const float inv_l = (acc && l > 0.f) ? 1.f / l : 0.f;
-      const size_t grow = (size_t)it.bh * p.N + (size_t)it.j * p.c + (size_t)(valid ? x : 0);
+      const size_t grow = out_row<ZZ>(p, it.bh, it.j, valid ? x : 0);
       __nv_bfloat16* orow_g = p.o + grow * D;
 #pragma unroll 1
       for (int q = 0; q < D / 32; ++q) {
@@ -730,13 +777,27 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 }
 
 // ------------------------------------------------------------------ host
+// mode 0: [BH, P, c, d] (layout order, or token order of the contiguous
+// layout); mode 1: striped token order as [BH, c, P, d] (box over c);
+// mode 2: zigzag token order as [BH, 2P, c/2, d].
 static bool encode_qkv_map(CUtensorMap* map, const void* base, int64_t BH, int64_t N, int64_t c,
-                           int P, int d) {
+                           int P, int d, int mode = 0) {
   PFN_encodeTiled enc = get_encode_tiled();
   if (!enc) return false;
   cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)c, (cuuint64_t)P, (cuuint64_t)BH};
   cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)c * d * 2, (cuuint64_t)N * d * 2};
   cuuint32_t box[4] = {64, (cuuint32_t)kBM, 1, 1};
+  if (mode == 1) {
+    dims[1] = (cuuint64_t)P;
+    dims[2] = (cuuint64_t)c;
+    strides[1] = (cuuint64_t)P * d * 2;
+    box[1] = 1;
+    box[2] = (cuuint32_t)kBM;
+  } else if (mode == 2) {
+    dims[1] = (cuuint64_t)(c / 2);
+    dims[2] = (cuuint64_t)(2 * P);
+    strides[1] = (cuuint64_t)(c / 2) * d * 2;
+  }
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -750,9 +811,10 @@ static ra_status launch(const AttnLaunch& a) {
   using C = Cfg<D>;
   CUtensorMap tq, tk, tv;
   const int64_t c = a.N / a.P;
-  if (!encode_qkv_map(&tq, a.q, a.BH, a.N, c, a.P, D) ||
-      !encode_qkv_map(&tk, a.k, a.BH, a.N, c, a.P, D) ||
-      !encode_qkv_map(&tv, a.v, a.BH, a.N, c, a.P, D))
+  const int mode = !a.tok ? 0 : a.striped ? 1 : a.zigzag ? 2 : 0;
+  if (!encode_qkv_map(&tq, a.q, a.BH, a.N, c, a.P, D, mode) ||
+      !encode_qkv_map(&tk, a.k, a.BH, a.N, c, a.P, D, mode) ||
+      !encode_qkv_map(&tv, a.v, a.BH, a.N, c, a.P, D, mode))
     return RA_ERR_CUDA;
   static int attr_set[64] = {0};
   if (a.device < 64 && !attr_set[a.device]) {
@@ -764,6 +826,7 @@ static ra_status launch(const AttnLaunch& a) {
   AttnParams p;
   p.o = reinterpret_cast<__nv_bfloat16*>(a.o);
   p.o_f32 = a.o_f32;
+  p.tok = a.tok;
   p.lse = a.lse;
   p.BH = (int)a.BH;
   p.N = (int)a.N;

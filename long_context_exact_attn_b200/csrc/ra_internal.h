@@ -32,6 +32,7 @@ struct AttnLaunch {
   int blk_j = -1, blk_kb = -1;   // single-block mode when blk_kb >= 0 (P = 1)
   int zigzag = 0;                // zigzag layout (striped == 0)
   int o_f32 = 0;                 // write O as float32
+  int tok = 0;                   // q, k, v, o, lse in token order
 };
 
 ra_status attn_fwd_launch(const AttnLaunch& a);

@@ -20,6 +20,7 @@ STRIPED = 1
 ZIGZAG = 2
 SCHED_FREE = 0x100
 O_F32 = 0x200
+TOKEN_ORDER = 0x400
 
 BF16 = 0
 F32 = 1
@@ -134,10 +135,12 @@ def partition(x, P, layout, inverse=False, out=None):
 
 
 def attn_fwd(q, k, v, P, layout, causal=True, scale=None, sched_free=False, out=None, lse=None,
-             o_f32=False):
+             o_f32=False, token_order=False):
     """Exact blockwise attention forward; q, k, v: [B, H, N, d] bf16 CUDA
-    tensors in LAYOUT order.  Returns (o [B, H, N, d] bf16, or float32 with
-    ``o_f32``, lse [B, H, N] float32), both in layout order."""
+    tensors in LAYOUT order (in token order with ``token_order``: the
+    kernel applies the layout's permutation itself).  Returns (o [B, H, N, d]
+    bf16, or float32 with ``o_f32``, lse [B, H, N] float32), in the same
+    order as the inputs."""
     for n, t in (("q", q), ("k", k), ("v", v)):
         _cuda_contig(t, n)
         if t.dtype != torch.bfloat16:
@@ -158,7 +161,8 @@ def attn_fwd(q, k, v, P, layout, causal=True, scale=None, sched_free=False, out=
         raise ValueError("lse must be float32 [B, H, N]")
     _cuda_contig(out, "out")
     _cuda_contig(lse, "lse")
-    lay = int(layout) | (SCHED_FREE if sched_free else 0) | (O_F32 if o_f32 else 0)
+    lay = (int(layout) | (SCHED_FREE if sched_free else 0) | (O_F32 if o_f32 else 0)
+           | (TOKEN_ORDER if token_order else 0))
     _check(lib().ra_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, d, int(P),
                              lay, int(bool(causal)), float(scale), _stream(q)), "ra_attn_fwd")
     return out, lse

@@ -68,7 +68,7 @@ def attn(L, q=A, k=Bp, v=Cp, o=Op, lse=Lp, B=1, H=2, N=1024, d=128, P=4, layout=
     (dict(q=A + 8), 2), (dict(o=Op + 2), 2), (dict(lse=Lp + 4), 2),
     (dict(N=1000, P=3), 3), (dict(P=0), 3), (dict(N=0), 3), (dict(B=0), 3),
     (dict(d=96), 4), (dict(d=256), 4),
-    (dict(layout=3), 5), (dict(layout=0x400), 5), (dict(layout=0x1201), 5),
+    (dict(layout=3), 5), (dict(layout=0x800), 5), (dict(layout=0x1201), 5),
     (dict(scale=0.0), 6), (dict(scale=float("inf")), 6), (dict(scale=float("nan")), 6),
     (dict(scale=-1.0), 6),
     (dict(o=A), 8), (dict(lse=Op + 64), 8),
@@ -189,7 +189,7 @@ def host(L, q=A, k=Bp, v=Cp, o=Op, lse=Lp, B=1, H=2, N=1024, d=128, P=4, layout=
 
 @pytest.mark.parametrize("kw,code", [
     (dict(ws=0), 1), (dict(o=0), 1), (dict(ws=(6 << 40) + 128), 2), (dict(N=1000, P=3), 3),
-    (dict(d=96), 4), (dict(layout=3), 5), (dict(scale=-1.0), 6), (dict(wsb=4210687), 14),
+    (dict(d=96), 4), (dict(layout=3), 5), (dict(scale=-1.0), 6), (dict(wsb=2105343), 14),
     (dict(wsb=0), 14),
 ])
 def test_attn_fwd_host_rejects_invalid_arguments(L, kw, code):
@@ -197,11 +197,11 @@ def test_attn_fwd_host_rejects_invalid_arguments(L, kw, code):
 
 
 def test_host_workspace_formula(L):
-    # per head and slot: striped 8 bf16 [N, d] buffers + 2 float32 [N];
-    # contiguous 4 + 1; two slots
-    assert L.ra_attn_fwd_host_workspace(1024, 128, 1, 1) == 2 * (8 * 262144 + 2 * 4096)
+    # per head and slot: q, k, v, o ([N, d] bf16) and lse ([N] float32), all
+    # in token order whatever the layout; two slots
+    assert L.ra_attn_fwd_host_workspace(1024, 128, 1, 1) == 2 * (4 * 262144 + 4096)
     assert L.ra_attn_fwd_host_workspace(1024, 128, 0, 3) == 2 * 3 * (4 * 262144 + 4096)
-    assert L.ra_attn_fwd_host_workspace(1000, 64, 1, 1) == 2 * (8 * 128000 + 2 * 4096)
+    assert L.ra_attn_fwd_host_workspace(1000, 64, 2, 1) == 2 * (4 * 128000 + 4096)
     assert L.ra_attn_fwd_host_workspace(0, 64, 1, 1) == -1
 
 

@@ -350,3 +350,39 @@ def test_o_f32_output_rounds_to_the_bf16_output(layout):
     e32 = np.abs(o32.cpu().numpy()[:, :, np.argsort(perm)] - o_ref).mean()
     e16 = np.abs(o16.float().cpu().numpy()[:, :, np.argsort(perm)] - o_ref).mean()
     assert e32 <= e16
+
+
+TOKEN_CASES = [
+    # (B, H, N, d, P, layout, causal)
+    (1, 2, 2048, 128, 4, W.STRIPED, True),
+    (2, 3, 600, 128, 3, W.STRIPED, True),        # c = 200: ragged tiles
+    (1, 2, 1500, 64, 5, W.STRIPED, False),
+    (1, 2, 1024, 128, 4, W.CONTIGUOUS, True),
+    (1, 2, 4096, 128, 4, W.ZIGZAG, True),
+    (1, 1, 262144, 128, 16, W.STRIPED, True),    # stress shape, one head
+]
+
+
+@pytest.mark.parametrize("case", TOKEN_CASES, ids=lambda c: "B{}H{}N{}d{}P{}{}{}".format(
+    c[0], c[1], c[2], c[3], c[4], "csz"[c[5]], "C" if c[6] else "F"))
+def test_token_order_is_bit_identical_to_partitioned_path(case):
+    """RA_TOKEN_ORDER (the stripe applied in the TMA addressing and the
+    epilogue) gives exactly the partition / attention / inverse-partition
+    result."""
+    B, H, N, d, P, layout, causal = case
+    w = W.Workload("tok", B, H, N, d, P, layout, causal, seed=N + P, qk_scale_up=3.0)
+    q, k, v = (t.cuda() for t in W.make_qkv(w))
+    o_t, l_t = ops.attn_fwd(q, k, v, P, layout, causal, token_order=True)
+    if layout == W.CONTIGUOUS:
+        o_r, l_r = ops.attn_fwd(q, k, v, P, layout, causal)
+    else:
+        qp, kp, vp = (ops.partition(t, P, layout) for t in (q, k, v))
+        o_p, l_p = ops.attn_fwd(qp, kp, vp, P, layout, causal)
+        o_r = ops.partition(o_p, P, layout, inverse=True)
+        l_r = ops.partition(l_p, P, layout, inverse=True)
+    o32, _ = ops.attn_fwd(q, k, v, P, layout, causal, token_order=True, o_f32=True)
+    torch.cuda.synchronize()
+    assert ops.device_fault() == 0
+    assert torch.equal(o_t, o_r)
+    assert torch.equal(l_t, l_r)
+    assert torch.equal(o32.to(torch.bfloat16), o_t)
