@@ -54,16 +54,40 @@ def load_peaks():
 
 
 # The sources the forward kernel is compiled from (its file and what it
-# includes): a recorded ncu traffic figure is valid while these are unchanged.
+# includes): a recorded ncu traffic figure is valid while their code (not
+# their comments) is unchanged.
 FWD_SOURCES = ("attn_fwd.cu", "exp2_poly.h", "ra_internal.h", "ra_ptx.cuh", "ra_tiles.cuh")
+
+
+def _strip_comments(text):
+    """C/C++ source without comments and blank-space runs (comment edits do
+    not change the compiled kernel, so they must not invalidate a record)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        if text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        elif text[i] == '"':
+            j = i + 1
+            while j < n and text[j] != '"':
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        else:
+            out.append(text[i])
+            i += 1
+    return " ".join("".join(out).split())
 
 
 def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "long_context_exact_attn_b200", "csrc")
     for name in FWD_SOURCES:
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update(name.encode() + _strip_comments(f.read()).encode())
     return h.hexdigest()[:16]
 
 

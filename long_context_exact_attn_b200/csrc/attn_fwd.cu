@@ -14,7 +14,13 @@
 //   warps 4-7  softmax warpgroup for query tile 1
 //   warp  8    TMA producer: Q tile pair once per work item, then K and V
 //              tiles into a ring of shared-memory slots
-//   warp  9    tcgen05 issuer (one thread) + TMEM owner
+//   warp  9    tcgen05 issuer (warp-uniform, one elected lane issues) and
+//              TMEM owner
+// Variants of the same kernel: the zigzag layout (template parameter ZZ:
+// each key block walked as its two chunks), token-order addressing (the
+// layout's permutation applied in the TMA coordinates and the epilogue's
+// rows), float32 output, and a single-block mode (one query shard against
+// one key block, the per-round step of a physical ring).
 // Tensor memory (512 columns x 128 lanes x 32 bit):
 //   [0,128)  S0 = Q0 K^T (fp32), later overwritten in place by P0 (bf16x2,
 //            columns [0,64)) which is the A operand of P0 V
