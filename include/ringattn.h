@@ -220,8 +220,9 @@ ra_status ra_attn_fwd(const void* q, const void* k, const void* v, void* o, floa
  *                     not overlap each other or any input.
  *   workspace         device, float32[B * H * N] scratch the call overwrites
  *                     (holds D); owned by the caller, no overlap with others.
- *   All pointers 16-byte aligned.  d, N, P, layout (no scheduling flag),
- *   causal and scale as for ra_attn_fwd.
+ *   All pointers 16-byte aligned.  d, N, P, layout, causal and scale as for
+ *   ra_attn_fwd; of the flags only RA_TOKEN_ORDER (every tensor, lse
+ *   included, in token order).
  * Arithmetic: bf16 operands, fp32 accumulation on the tensor cores, P and dS
  * rounded to bf16 for their products, outputs rounded to bf16 once.
  */

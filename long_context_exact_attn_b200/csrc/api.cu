@@ -240,6 +240,8 @@ ra_status ra_attn_bwd(const void* q, const void* k, const void* v, const void* o
                       float* workspace, int64_t B, int64_t H, int64_t N, int64_t d, int P,
                       int layout, int causal, float scale, void* stream) {
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return RA_ERR_NULL;
+  const int tok = (layout & RA_TOKEN_ORDER) != 0;
+  layout &= ~RA_TOKEN_ORDER;
   if (layout != RA_CONTIGUOUS && layout != RA_STRIPED && layout != RA_ZIGZAG) return RA_ERR_LAYOUT;
   if (d != 64 && d != 128) return RA_ERR_HEADDIM;
   if (B < 1 || H < 1 || N < 1 || P < 1 || N % P != 0) return RA_ERR_SHAPE;
@@ -273,6 +275,7 @@ ra_status ra_attn_bwd(const void* q, const void* k, const void* v, const void* o
   a.BH = B * H; a.N = N; a.d = d; a.P = P;
   a.striped = layout == RA_STRIPED;
   a.zigzag = layout == RA_ZIGZAG;
+  a.tok = tok;
   a.causal = causal != 0;
   a.scale = scale;
   a.device = dev;
@@ -286,6 +289,8 @@ ra_status ra_attn_bwd_noalloc(const void* q, const void* k, const void* v, const
                               int64_t B, int64_t H, int64_t N, int64_t d, int P, int layout,
                               int causal, float scale, void* stream) {
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return RA_ERR_NULL;
+  const int tok = (layout & RA_TOKEN_ORDER) != 0;
+  layout &= ~RA_TOKEN_ORDER;
   if (layout != RA_CONTIGUOUS && layout != RA_STRIPED && layout != RA_ZIGZAG) return RA_ERR_LAYOUT;
   if (d != 64 && d != 128) return RA_ERR_HEADDIM;
   if (B < 1 || H < 1 || N < 1 || P < 1 || N % P != 0) return RA_ERR_SHAPE;
@@ -316,6 +321,7 @@ ra_status ra_attn_bwd_noalloc(const void* q, const void* k, const void* v, const
   a.BH = B * H; a.N = N; a.d = d; a.P = P;
   a.striped = layout == RA_STRIPED;
   a.zigzag = layout == RA_ZIGZAG;
+  a.tok = tok;
   a.causal = causal != 0;
   a.scale = scale;
   a.device = dev;

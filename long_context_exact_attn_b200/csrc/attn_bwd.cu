@@ -43,6 +43,8 @@ struct BwdParams {
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   int BH, N, c, P, T, striped, zigzag, causal;
+  int tok;                // all tensors in token order (the layout applied in
+                          // the TMA coordinates and the row indices)
   float c2;               // scale * log2(e)
   float scale;
   unsigned long long timeout_ns;
@@ -136,12 +138,51 @@ enum : uint32_t {
   kAbort = 140
 };
 
-// TMA: one 128 x D tile of a [BH, P, c, D] tensor at (shard, row0, bh).
-template <int D>
-__device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* tm, uint32_t bar,
-                                          int row0, int shard, int bh) {
+// TMA: one 128 x D tile of shard `shard` starting at local row row0.  In
+// layout order the map is [BH, P, c, D] and the coordinates (row0, shard);
+// in token order the striped map is [BH, c, P, D] read as (shard, row0)
+// (shard j's rows are tokens x*P + j), the zigzag map [BH, 2P, c/2, D]
+// read as (row in chunk, chunk), and contiguous token order is layout order.
+template <bool ZZ>
+__device__ __forceinline__ void tile_coord(const BwdParams& p, int shard, int row0, int& c1,
+                                           int& c2) {
+  c1 = row0;
+  c2 = shard;
+  if (!p.tok) return;
+  if (p.striped) {
+    c1 = shard;
+    c2 = row0;
+  } else if (ZZ) {
+    const int h = p.c >> 1;
+    if (row0 >= h) {
+      c1 = row0 - h;
+      c2 = 2 * p.P - 1 - shard;
+    }
+  }
+}
+
+template <int D, bool ZZ>
+__device__ __forceinline__ void load_tile(const BwdParams& p, uint32_t dst, const CUtensorMap* tm,
+                                          uint32_t bar, int row0, int shard, int bh) {
+  int c1, c2;
+  tile_coord<ZZ>(p, shard, row0, c1, c2);
 #pragma unroll
-  for (int ch = 0; ch < D / 64; ++ch) tma_load_4d(dst + ch * 16384, tm, bar, ch * 64, row0, shard, bh);
+  for (int ch = 0; ch < D / 64; ++ch) tma_load_4d(dst + ch * 16384, tm, bar, ch * 64, c1, c2, bh);
+}
+
+// Row (in the tensors' order) of local row x of shard j.
+template <bool ZZ>
+__device__ __forceinline__ size_t bwd_row(const BwdParams& p, int bh, int j, int x) {
+  size_t t = (size_t)j * p.c + x;
+  if (p.tok) {
+    if (p.striped) {
+      t = (size_t)x * p.P + j;
+    } else if (ZZ) {
+      const int h = p.c >> 1;
+      t = x < h ? (size_t)j * h + x : (size_t)(2 * p.P - 1 - j) * h + (x - h);
+    }
+  }
+  return (size_t)bh * p.N + t;
 }
 
 // Whole-warp bounded wait (same result in every lane).
@@ -350,8 +391,8 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       mbar_arrive_expect_tx(bar + kBarFixed, 2 * C::kTile);
-      load_tile<D>(sb + C::kFixed0, &tmK, bar + kBarFixed, y0, kb, bh);
-      load_tile<D>(sb + C::kFixed1, &tmV, bar + kBarFixed, y0, kb, bh);
+      load_tile<D, ZZ>(p, sb + C::kFixed0, &tmK, bar + kBarFixed, y0, kb, bh);
+      load_tile<D, ZZ>(p, sb + C::kFixed1, &tmV, bar + kBarFixed, y0, kb, bh);
     }
     QCursor<ZZ> cur;
     cur.init(p, kb, y0);
@@ -365,7 +406,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       for (int u = 0; u < 4; ++u) {
         const int x = qt * kBM + lane + 32 * u;
         const bool valid = x < p.c;
-        const size_t row = (size_t)bh * p.N + (size_t)j * p.c + (size_t)(valid ? x : 0);
+        const size_t row = bwd_row<ZZ>(p, bh, j, valid ? x : 0);
         lv[u] = valid ? p.lse[row] * 1.4426950408889634f : INFINITY;
         dv[u] = valid ? p.dvec[row] : 0.f;
       }
@@ -375,7 +416,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         break;
       if (lane == 0) {
         mbar_arrive_expect_tx(bar + kBarFullA + 8 * a, C::kTile);
-        load_tile<D>(ringA + a * C::kTile, &tmQ, bar + kBarFullA + 8 * a, qt * kBM, j, bh);
+        load_tile<D, ZZ>(p, ringA + a * C::kTile, &tmQ, bar + kBarFullA + 8 * a, qt * kBM, j, bh);
       }
       ++na;
       const uint32_t b = nb & 1;
@@ -389,7 +430,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
       if (lane == 0) {
         mbar_arrive_expect_tx(bar + kBarFullB + 8 * b, C::kTile);
-        load_tile<D>(ringB + b * C::kTile, &tmdO, bar + kBarFullB + 8 * b, qt * kBM, j, bh);
+        load_tile<D, ZZ>(p, ringB + b * C::kTile, &tmdO, bar + kBarFullB + 8 * b, qt * kBM, j, bh);
       } else {
         mbar_arrive(bar + kBarFullB + 8 * b);
       }
@@ -572,7 +613,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     if (ok && (i == 0 || warp_wait(bar + kBarAcc, 0, abort_flag, p.timeout_ns))) {
       tc_fence_after();
       const bool valid = y < p.c;
-      const size_t row = (size_t)bh * p.N + (size_t)kb * p.c + (size_t)(valid ? y : 0);
+      const size_t row = bwd_row<ZZ>(p, bh, kb, valid ? y : 0);
 #pragma unroll 1
       for (int q = 0; q < D / 64; ++q) {
         const int col = wg * (D / 2) + q * 32;
@@ -675,8 +716,8 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       mbar_arrive_expect_tx(bar + kBarFixed, 2 * C::kTile);
-      load_tile<D>(sb + C::kFixed0, &tmQ, bar + kBarFixed, x0, j, bh);
-      load_tile<D>(sb + C::kFixed1, &tmdO, bar + kBarFixed, x0, j, bh);
+      load_tile<D, ZZ>(p, sb + C::kFixed0, &tmQ, bar + kBarFixed, x0, j, bh);
+      load_tile<D, ZZ>(p, sb + C::kFixed1, &tmdO, bar + kBarFixed, x0, j, bh);
       KCursor<ZZ> cur;
       cur.init(p, j, x0);
       uint32_t na = 0, nb = 0;
@@ -688,13 +729,13 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             !mbar_wait(bar + kBarEmptyA + 8 * a, (na / C::kSlotsA - 1) & 1, abort_flag, p.timeout_ns))
           break;
         mbar_arrive_expect_tx(bar + kBarFullA + 8 * a, C::kTile);
-        load_tile<D>(ringA + a * C::kTile, &tmK, bar + kBarFullA + 8 * a, y0, kb, bh);
+        load_tile<D, ZZ>(p, ringA + a * C::kTile, &tmK, bar + kBarFullA + 8 * a, y0, kb, bh);
         ++na;
         const uint32_t b = nb & 1;
         if (nb >= 2 && !mbar_wait(bar + kBarEmptyB + 8 * b, ((nb >> 1) - 1) & 1, abort_flag, p.timeout_ns))
           break;
         mbar_arrive_expect_tx(bar + kBarFullB + 8 * b, C::kTile);
-        load_tile<D>(ringB + b * C::kTile, &tmV, bar + kBarFullB + 8 * b, y0, kb, bh);
+        load_tile<D, ZZ>(p, ringB + b * C::kTile, &tmV, bar + kBarFullB + 8 * b, y0, kb, bh);
         ++nb;
       }
       volatile int no_abort = 0;
@@ -774,7 +815,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const int wg = warp / 4, wq = warp % 4;
     const int x = x0 + wq * 32 + lane;
     const bool xvalid = x < p.c;
-    const size_t xrow = (size_t)bh * p.N + (size_t)j * p.c + (size_t)(xvalid ? x : 0);
+    const size_t xrow = bwd_row<ZZ>(p, bh, j, xvalid ? x : 0);
     const float lse2 = xvalid ? p.lse[xrow] * 1.4426950408889634f : INFINITY;
     const float drow = xvalid ? p.dvec[xrow] : 0.f;
     const uint64_t c2x2 = pk2(p.c2, p.c2), nl2 = pk2(-lse2, -lse2), d2 = pk2(drow, drow);
@@ -859,13 +900,26 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 }
 
 // ------------------------------------------------------------------ host
+// mode 0: [BH, P, c, d]; 1: striped token order [BH, c, P, d] (box over c);
+// 2: zigzag token order [BH, 2P, c/2, d].
 static bool encode_map(CUtensorMap* map, const void* base, int64_t BH, int64_t N, int64_t c, int P,
-                       int d) {
+                       int d, int mode) {
   PFN_encodeTiled enc = get_encode_tiled();
   if (!enc) return false;
   cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)c, (cuuint64_t)P, (cuuint64_t)BH};
   cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)c * d * 2, (cuuint64_t)N * d * 2};
   cuuint32_t box[4] = {64, (cuuint32_t)kBM, 1, 1};
+  if (mode == 1) {
+    dims[1] = (cuuint64_t)P;
+    dims[2] = (cuuint64_t)c;
+    strides[1] = (cuuint64_t)P * d * 2;
+    box[1] = 1;
+    box[2] = (cuuint32_t)kBM;
+  } else if (mode == 2) {
+    dims[1] = (cuuint64_t)(c / 2);
+    dims[2] = (cuuint64_t)(2 * P);
+    strides[1] = (cuuint64_t)(c / 2) * d * 2;
+  }
   cuuint32_t estr[4] = {1, 1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -877,8 +931,11 @@ static ra_status launch_bwd(const BwdLaunch& a) {
   using C = BwdCfg<D>;
   const int64_t c = a.N / a.P;
   CUtensorMap tq, tk, tv, tdo;
-  if (!encode_map(&tq, a.q, a.BH, a.N, c, a.P, D) || !encode_map(&tk, a.k, a.BH, a.N, c, a.P, D) ||
-      !encode_map(&tv, a.v, a.BH, a.N, c, a.P, D) || !encode_map(&tdo, a.dout, a.BH, a.N, c, a.P, D))
+  const int mode = !a.tok ? 0 : a.striped ? 1 : a.zigzag ? 2 : 0;
+  if (!encode_map(&tq, a.q, a.BH, a.N, c, a.P, D, mode) ||
+      !encode_map(&tk, a.k, a.BH, a.N, c, a.P, D, mode) ||
+      !encode_map(&tv, a.v, a.BH, a.N, c, a.P, D, mode) ||
+      !encode_map(&tdo, a.dout, a.BH, a.N, c, a.P, D, mode))
     return RA_ERR_CUDA;
   static int attr_set[64] = {0};
   if (a.device < 64 && !attr_set[a.device]) {
@@ -904,6 +961,7 @@ static ra_status launch_bwd(const BwdLaunch& a) {
   p.T = (int)((c + kBM - 1) / kBM);
   p.striped = a.striped;
   p.zigzag = a.zigzag;
+  p.tok = a.tok;
   p.causal = a.causal;
   p.c2 = (float)((double)a.scale * 1.4426950408889634074);
   p.scale = a.scale;

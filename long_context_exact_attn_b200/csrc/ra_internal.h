@@ -55,6 +55,7 @@ struct BwdLaunch {
   int device, num_sms;
   void* stream;
   int zigzag = 0;                // zigzag layout (striped == 0)
+  int tok = 0;                   // all tensors in token order
 };
 
 ra_status attn_bwd_launch(const BwdLaunch& a);

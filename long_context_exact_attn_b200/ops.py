@@ -169,9 +169,9 @@ def attn_fwd(q, k, v, P, layout, causal=True, scale=None, sched_free=False, out=
 
 
 def attn_bwd(q, k, v, o, dout, lse, P, layout, causal=True, scale=None, workspace=None,
-             dq=None, dk=None, dv=None):
-    """Gradients (dq, dk, dv) of attn_fwd; all tensors in LAYOUT order, as
-    returned by attn_fwd on the same q, k, v.  ``workspace``: float32 with
+             dq=None, dk=None, dv=None, token_order=False):
+    """Gradients (dq, dk, dv) of attn_fwd; all tensors in LAYOUT order (token
+    order with ``token_order``), as returned by attn_fwd on the same q, k, v.  ``workspace``: float32 with
     B*H*N elements (allocated here if not given)."""
     for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
         _cuda_contig(t, n)
@@ -194,8 +194,9 @@ def attn_bwd(q, k, v, o, dout, lse, P, layout, causal=True, scale=None, workspac
     dv = torch.empty_like(q) if dv is None else dv
     for n, t in (("dq", dq), ("dk", dk), ("dv", dv), ("workspace", workspace)):
         _cuda_contig(t, n)
+    lay = int(layout) | (TOKEN_ORDER if token_order else 0)
     _check(lib().ra_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
-                             _ptr(dk), _ptr(dv), _ptr(workspace), B, H, N, d, int(P), int(layout),
+                             _ptr(dk), _ptr(dv), _ptr(workspace), B, H, N, d, int(P), lay,
                              int(bool(causal)), float(scale), _stream(q)), "ra_attn_bwd")
     return dq, dk, dv
 

@@ -117,8 +117,8 @@ def bwd(L, q=A, k=Bp, v=Cp, o=Op, do=6 << 40, lse=Lp, dq=7 << 40, dk=8 << 40, dv
 
 @pytest.mark.parametrize("kw,code", [
     (dict(ws=0), 1), (dict(do=0), 1), (dict(dq=(7 << 40) + 8), 2), (dict(ws=(10 << 40) + 4), 2),
-    (dict(N=1000, P=3), 3), (dict(d=32), 4), (dict(layout=0x101), 5), (dict(scale=0.0), 6),
-    (dict(dq=A), 8), (dict(dk=7 << 40), 8), (dict(ws=Lp), 8),
+    (dict(N=1000, P=3), 3), (dict(d=32), 4), (dict(layout=0x101), 5), (dict(layout=0x201), 5),
+    (dict(scale=0.0), 6), (dict(dq=A), 8), (dict(dk=7 << 40), 8), (dict(ws=Lp), 8),
 ])
 def test_attn_bwd_rejects_invalid_arguments(L, kw, code):
     assert bwd(L, **kw) == code

@@ -128,3 +128,25 @@ def test_backward_full_stress_size():
     sum_dk = gk[0].double().sum(dim=1)
     abs_dk = gk[0].double().abs().sum(dim=1)
     assert torch.all(sum_dk.abs() <= 2.0 ** -7 * abs_dk + 1e-3)
+
+
+@pytest.mark.parametrize("layout,N,P", [(W.STRIPED, 2048, 4), (W.ZIGZAG, 4096, 4),
+                                        (W.CONTIGUOUS, 1024, 4), (W.STRIPED, 600, 3)])
+def test_backward_token_order_is_bit_identical(layout, N, P):
+    """RA_TOKEN_ORDER forward + backward on token-order tensors equals the
+    partitioned forward + backward, gradients un-partitioned, bit for bit."""
+    w = W.Workload("bwd_tok", 1, 2, N, 128, P, layout, True, N + 3, qk_scale_up=3.0)
+    q, k, v = (t.cuda() for t in W.make_qkv(w))
+    do = torch.randn(q.shape, generator=torch.Generator().manual_seed(N)).to(torch.bfloat16).cuda()
+    o_t, l_t = ops.attn_fwd(q, k, v, P, layout, True, token_order=True)
+    g_t = ops.attn_bwd(q, k, v, o_t, do, l_t, P, layout, True, token_order=True)
+    part = (lambda t: ops.partition(t, P, layout)) if layout != W.CONTIGUOUS else (lambda t: t)
+    unpart = ((lambda t: ops.partition(t, P, layout, inverse=True))
+              if layout != W.CONTIGUOUS else (lambda t: t))
+    qp, kp, vp, dop = (part(t) for t in (q, k, v, do))
+    o_p, l_p = ops.attn_fwd(qp, kp, vp, P, layout, True)
+    g_p = [unpart(g) for g in ops.attn_bwd(qp, kp, vp, o_p, dop, l_p, P, layout, True)]
+    torch.cuda.synchronize()
+    assert ops.device_fault() == 0
+    for a, b in zip(g_t, g_p):
+        assert torch.equal(a, b)
