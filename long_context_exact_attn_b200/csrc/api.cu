@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "ra_internal.h"
+#include "ra_bwd.h"
 
 namespace ra {
 

@@ -29,6 +29,7 @@
 #include <mutex>
 
 #include "ra_internal.h"
+#include "ra_bwd.h"
 #include "ra_ptx.cuh"
 #include "ra_tiles.cuh"
 

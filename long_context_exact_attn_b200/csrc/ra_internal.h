@@ -37,32 +37,6 @@ struct AttnLaunch {
 
 ra_status attn_fwd_launch(const AttnLaunch& a);
 
-struct BwdLaunch {
-  const void* q;
-  const void* k;
-  const void* v;
-  const void* o;
-  const void* dout;
-  const float* lse;
-  void* dq;
-  void* dk;
-  void* dv;
-  float* workspace;
-  int64_t BH, N, d;
-  int P;
-  int striped, causal;
-  float scale;
-  int device, num_sms;
-  void* stream;
-  int zigzag = 0;                // zigzag layout (striped == 0)
-  int tok = 0;                   // all tensors in token order
-};
-
-ra_status attn_bwd_launch(const BwdLaunch& a);
-
-// Capacity (floats) of the fixed scratch used by ra_attn_bwd_noalloc.
-constexpr long long kNoAllocScratchFloats = 1LL << 20;
-ra_status attn_bwd_noalloc_launch(BwdLaunch a);
 ra_status read_device_fault(int* code);
 unsigned int* device_fault_word();
 ra_status wait_selftest_launch(int64_t limit_ns, void* stream);
