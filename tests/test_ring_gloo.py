@@ -40,7 +40,7 @@ def _worker(rank, world, port, layout, causal, out):
         c = N // P
         g = np.random.default_rng(11)
         q, k, v = (g.standard_normal((N, d)) * s for s in (3.0, 3.0, 1.0))
-        lay = OP.STRIPED if layout else OP.CONTIGUOUS
+        lay = {0: OP.CONTIGUOUS, 1: OP.STRIPED, 2: OP.ZIGZAG}[layout]
         qp, kp, vp = (OP.partition(a, P, lay, axis=0) for a in (q, k, v))
         shard = lambda a, j: torch.from_numpy(np.ascontiguousarray(a[j * c:(j + 1) * c]))[None, None]
         seen = []
@@ -73,8 +73,9 @@ def _worker(rank, world, port, layout, causal, out):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 4])
-@pytest.mark.parametrize("layout,causal", [(1, True), (0, True), (1, False)])
+@pytest.mark.parametrize("world,layout,causal", [
+    (2, 1, True), (2, 0, True), (2, 1, False), (4, 1, True), (4, 0, True), (4, 1, False),
+    (3, 1, True), (2, 2, True), (4, 2, True)])
 def test_process_ring_equals_definition(world, layout, causal):
     from oracle import attention as OA
     from oracle import partition as OP
@@ -93,7 +94,7 @@ def test_process_ring_equals_definition(world, layout, causal):
     N, d, P = 6 * world, 8, world
     g = np.random.default_rng(11)
     q, k, v = (g.standard_normal((N, d)) * s for s in (3.0, 3.0, 1.0))
-    lay = OP.STRIPED if layout else OP.CONTIGUOUS
+    lay = {0: OP.CONTIGUOUS, 1: OP.STRIPED, 2: OP.ZIGZAG}[layout]
     o_ref, lse_ref = OA.attention(q, k, v, d ** -0.5, causal)
     o = np.concatenate([res[r][0] for r in range(P)])
     lse = np.concatenate([res[r][1] for r in range(P)])
