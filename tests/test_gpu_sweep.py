@@ -1,7 +1,7 @@
 """A seeded sweep of shapes against the oracle: shard lengths from 1 to
 several tiles (ragged ones included), P from 1 to N, d 64 and 128, all three
 layouts (zigzag where N/P is a multiple of 512), causal and not, q,k x1 and
-x3.  Per case: the forward (partitioned path) within the forward tolerances,
+x3, one or two batch entries.  Per case: the forward (partitioned path) within the forward tolerances,
 the token-order path bit-identical to it, and for every third case the
 backward within its tolerances."""
 
@@ -17,7 +17,7 @@ from tests.test_gpu_parity import assert_close, oracle_full, run_path
 pytestmark = pytest.mark.gpu
 
 
-def _cases(n=24, seed=2024):
+def _cases(n=40, seed=2024):
     rng = np.random.default_rng(seed)
     out = []
     for i in range(n):
@@ -32,7 +32,8 @@ def _cases(n=24, seed=2024):
         causal = bool(rng.random() < 0.8)
         up = float(rng.choice([1.0, 3.0]))
         H = int(rng.choice([1, 2]))
-        out.append((i, H, N, d, P, layout, causal, up))
+        B = int(rng.choice([1, 2])) if N <= 4096 else 1
+        out.append((i, B, H, N, d, P, layout, causal, up))
     return out
 
 
@@ -44,11 +45,11 @@ def _lib():
     ops.device_fault()
 
 
-@pytest.mark.parametrize("case", _cases(), ids=lambda c: "i{}H{}N{}d{}P{}{}{}x{}".format(
-    c[0], c[1], c[2], c[3], c[4], "csz"[c[5]], "C" if c[6] else "F", c[7]))
+@pytest.mark.parametrize("case", _cases(), ids=lambda c: "i{}B{}H{}N{}d{}P{}{}{}x{}".format(
+    c[0], c[1], c[2], c[3], c[4], c[5], "csz"[c[6]], "C" if c[7] else "F", c[8]))
 def test_sweep(case):
-    i, H, N, d, P, layout, causal, up = case
-    w = W.Workload("sweep", 1, H, N, d, P, layout, causal, seed=1000 + i, qk_scale_up=up)
+    i, B, H, N, d, P, layout, causal, up = case
+    w = W.Workload("sweep", B, H, N, d, P, layout, causal, seed=1000 + i, qk_scale_up=up)
     q, k, v = W.make_qkv(w)
     o, lse = run_path(q, k, v, P, layout, causal)
     o_ref, lse_ref = oracle_full(q, k, v, causal, w.scale)
@@ -63,12 +64,12 @@ def test_sweep(case):
         grads = ops.attn_bwd(qd, kd, vd, o_t, do.cuda(), l_t, P, layout, causal, token_order=True)
         torch.cuda.synchronize()
         assert ops.device_fault() == 0
-        for h in range(H):
-            ref = OB.attention_backward(q[0, h].double().numpy(), k[0, h].double().numpy(),
-                                        v[0, h].double().numpy(), do[0, h].double().numpy(),
+        for b, h in ((b, h) for b in range(B) for h in range(H)):
+            ref = OB.attention_backward(q[b, h].double().numpy(), k[b, h].double().numpy(),
+                                        v[b, h].double().numpy(), do[b, h].double().numpy(),
                                         w.scale, causal)[:3]
             for name, g, r in zip(("dq", "dk", "dv"), grads, ref):
-                g = g[0, h].float().cpu().numpy()
+                g = g[b, h].float().cpu().numpy()
                 scale = max(np.abs(r).max(), 1e-6)
                 err = np.abs(g - r)
                 assert err.max() <= 2e-2 * scale, (case, name, err.max() / scale)
