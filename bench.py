@@ -589,7 +589,8 @@ def main():
     peak = float(peaks.get(peak_key, FALLBACK_PEAKS[peak_key]))
     achieved = flops / (attn_ms * 1e-3) / 1e12
     traffic = recorded_traffic(w.name)
-    roofline = {"bound": "tensor", "kernel": "attn_fwd_kernel<128>", "achieved": achieved,
+    kname = f"attn_fwd_kernel<{w.d}, {'true' if w.layout == W.ZIGZAG else 'false'}>"
+    roofline = {"bound": "tensor", "kernel": kname, "achieved": achieved,
                 "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                 "peak_source": f"{peaks_src} {peak_key}",
                 "frac_of_burst_peak": achieved / float(peaks.get("bf16_tflops",
