@@ -97,8 +97,8 @@ typedef int ra_status;
  * e.g. for callers that merge partial results or want O before rounding. */
 #define RA_O_F32 0x200
 
-/* Optional flag for ra_attn_fwd, OR-ed into `layout`: q, k, v, o and lse
- * are in TOKEN order.  The layout's permutation is then applied inside the
+/* Optional flag for ra_attn_fwd and ra_attn_bwd, OR-ed into `layout`: all
+ * their tensors (q, k, v, o, lse; dO and the gradients) are in TOKEN order.  The layout's permutation is then applied inside the
  * kernel (the TMA loads address shard j's rows where the tokens live, the
  * epilogue writes each row to its token position), so no ra_partition pass
  * is needed before or after; results equal the partition / attention /
@@ -125,8 +125,10 @@ int ra_version(void);
  *
  * Defined by the placements of "Striped Attention" review 分区策略对比 and
  * Ring Attention explainer ステップ1: with c = N/P, layout slot s = j*c + x
- * (shard j, local index x) holds token t = x*P + j (RA_STRIPED) or
- * t = j*c + x (RA_CONTIGUOUS).  Position ids are moved the same way
+ * (shard j, local index x) holds token t = x*P + j (RA_STRIPED),
+ * t = j*c + x (RA_CONTIGUOUS), or, with h = c/2, t = j*h + x for x < h and
+ * t = (2P-1-j)*h + (x - h) otherwise (RA_ZIGZAG, a reading of the layout the
+ * pages only name).  Position ids are moved the same way
  * (Striped review, 位置编码处理): pass the int32 ids as [1, 1, N, 1] RA_I32.
  *
  *   src, dst  device, [B, H, N, d] of `dtype` (bf16 = 2 bytes, f32/i32 = 4).

@@ -145,7 +145,7 @@ const char* ra_status_string(ra_status s) {
   }
 }
 
-int ra_version(void) { return 100; }
+int ra_version(void) { return 200; }
 
 ra_status ra_partition(const void* src, void* dst, int64_t B, int64_t H, int64_t N, int64_t d,
                        int P, int layout, int inverse, int dtype, void* stream) {
