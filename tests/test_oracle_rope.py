@@ -78,7 +78,7 @@ def test_scores_depend_on_relative_position_only(pairing):
              @ rope.rope(k, [25 + shift], 10000.0, pairing).T)
         np.testing.assert_allclose(s, base, rtol=1e-9, atol=1e-9)
     other = rope.rope(q, [41], 10000.0, pairing) @ rope.rope(k, [25], 10000.0, pairing).T
-    assert abs(float(other - base)) > 1e-6
+    assert abs((other - base).item()) > 1e-6
 
 
 @pytest.mark.parametrize("pairing", [INTERLEAVED, HALF])
