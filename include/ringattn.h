@@ -292,7 +292,9 @@ ra_status ra_attn_fwd_host(const void* q, const void* k, const void* v, void* o,
                            void* stream);
 
 /* Device workspace bytes for ra_attn_fwd_host with `heads_per_chunk` heads
- * per chunk (two staging slots); -1 for invalid sizes. */
+ * per chunk (two staging slots); -1 for invalid sizes (N outside
+ * [1, 2^31), d outside [1, 1024], heads_per_chunk < 1, or a byte count that
+ * does not fit int64_t). */
 int64_t ra_attn_fwd_host_workspace(int64_t N, int64_t d, int layout, int64_t heads_per_chunk);
 
 /*
@@ -334,7 +336,8 @@ ra_status ra_attn_fwd_block(const void* q, const void* k, const void* v, void* o
  *   o_b, lse_b       device bf16 [rows, d] and float32 [rows]: the partial.
  *   o_final          device bf16 [rows, d], written when mode has
  *                    RA_MERGE_FINAL (may be NULL otherwise).
- *   d                a multiple of 8.
+ *   rows, d          0 <= rows < 2^31; d a multiple of 8, 8 <= d <= 2^20
+ *                    (else RA_ERR_SHAPE).
  * No buffer may overlap another (RA_ERR_ALIAS); o_acc, o_b, o_final 16-byte
  * aligned.  Unknown mode bits: RA_ERR_LAYOUT.  Empty sides (lse = -inf)
  * contribute nothing; both empty give o = 0, lse = -inf.
@@ -355,7 +358,8 @@ ra_status ra_lse_merge_acc(float* o_acc, float* lse_acc, const void* o_b, const 
  *   lse_a, lse_b, lse_out device, [rows] float32.
  *   o_out may alias o_a (and lse_out lse_a): each element is read before it
  *   is written by the same thread.
- *   rows >= 0 (0 is a no-op), 1 <= d, d % 8 == 0.
+ *   0 <= rows < 2^40 (0 is a no-op); d % 8 == 0, 8 <= d <= 2^20 (else
+ *   RA_ERR_SHAPE).
  * Arithmetic in fp32, o_out rounded to bf16.
  */
 ra_status ra_lse_merge(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,

@@ -58,6 +58,13 @@ ra_status current_device(int* dev, DevInfo* info) {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// a * b * c < 2^31 for positive factors, decided without overflowing int64
+// (each factor and the partial product are bounded before the next multiply).
+bool rows_fit(int64_t a, int64_t b, int64_t c) {
+  const int64_t lim = (int64_t)1 << 31;
+  return a < lim && b < lim && c < lim && a * b < lim && a * b * c < lim;
+}
+
 bool overlap(const void* a, int64_t na, const void* b, int64_t nb) {
   const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
   return x < y + (uintptr_t)nb && y < x + (uintptr_t)na;
@@ -159,7 +166,7 @@ ra_status ra_partition(const void* src, void* dst, int64_t B, int64_t H, int64_t
   }
   if (B < 1 || H < 1 || N < 1 || d < 1 || P < 1 || N % P != 0) return RA_ERR_SHAPE;
   if (layout == RA_ZIGZAG && (N / P) % 2 != 0) return RA_ERR_SHAPE;
-  if (B * H * N >= ((int64_t)1 << 31) || d * esz >= ((int64_t)1 << 30)) return RA_ERR_SHAPE;
+  if (!rows_fit(B, H, N) || d >= ((int64_t)1 << 30) / esz) return RA_ERR_SHAPE;
   const int64_t row_bytes = d * esz;
   const uintptr_t need = (row_bytes % 16 == 0) ? 16 : (esz == 2 ? 2 : 4);
   if (!aligned(src, need) || !aligned(dst, need)) return RA_ERR_ALIGN;
@@ -179,7 +186,7 @@ ra_status ra_partition_rope(const void* src, void* dst, int64_t B, int64_t H, in
   if (d < 16 || d > 512 || d % 16 != 0) return RA_ERR_HEADDIM;
   if (B < 1 || H < 1 || N < 1 || P < 1 || N % P != 0) return RA_ERR_SHAPE;
   if (layout == RA_ZIGZAG && (N / P) % 2 != 0) return RA_ERR_SHAPE;
-  if (B * H * N >= ((int64_t)1 << 31)) return RA_ERR_SHAPE;
+  if (!rows_fit(B, H, N)) return RA_ERR_SHAPE;
   if (pairing != RA_ROPE_INTERLEAVED && pairing != RA_ROPE_HALF) return RA_ERR_ROPE;
   if (!(base > 1.f) || !isfinite(base)) return RA_ERR_ROPE;
   if (!aligned(src, 16) || !aligned(dst, 16)) return RA_ERR_ALIGN;
@@ -204,7 +211,7 @@ ra_status ra_attn_fwd(const void* q, const void* k, const void* v, void* o, floa
   if (d != 64 && d != 128) return RA_ERR_HEADDIM;
   if (B < 1 || H < 1 || N < 1 || P < 1 || N % P != 0) return RA_ERR_SHAPE;
   if (base == RA_ZIGZAG && (N / P) % 512 != 0) return RA_ERR_SHAPE;
-  if (B * H * N >= ((int64_t)1 << 31) || B * H >= ((int64_t)1 << 31)) return RA_ERR_SHAPE;
+  if (!rows_fit(B, H, N)) return RA_ERR_SHAPE;
   if (N / P > ((int64_t)1 << 30) / 128) return RA_ERR_SHAPE;
   if (!(scale > 0.f) || !isfinite(scale)) return RA_ERR_SCALE;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
@@ -247,7 +254,7 @@ ra_status ra_attn_bwd(const void* q, const void* k, const void* v, const void* o
   if (d != 64 && d != 128) return RA_ERR_HEADDIM;
   if (B < 1 || H < 1 || N < 1 || P < 1 || N % P != 0) return RA_ERR_SHAPE;
   if (layout == RA_ZIGZAG && (N / P) % 512 != 0) return RA_ERR_SHAPE;
-  if (B * H * N >= ((int64_t)1 << 31) || N / P > ((int64_t)1 << 30) / 128) return RA_ERR_SHAPE;
+  if (!rows_fit(B, H, N) || N / P > ((int64_t)1 << 30) / 128) return RA_ERR_SHAPE;
   if (B * H * P * ((N / P + 127) / 128) >= ((int64_t)1 << 31)) return RA_ERR_SHAPE;
   if (!(scale > 0.f) || !isfinite(scale)) return RA_ERR_SCALE;
   const void* all[] = {q, k, v, o, dout, lse, dq, dk, dv, workspace};
@@ -296,7 +303,7 @@ ra_status ra_attn_bwd_noalloc(const void* q, const void* k, const void* v, const
   if (d != 64 && d != 128) return RA_ERR_HEADDIM;
   if (B < 1 || H < 1 || N < 1 || P < 1 || N % P != 0) return RA_ERR_SHAPE;
   if (layout == RA_ZIGZAG && (N / P) % 512 != 0) return RA_ERR_SHAPE;
-  if (B * H * N >= ((int64_t)1 << 31) || N / P > ((int64_t)1 << 30) / 128) return RA_ERR_SHAPE;
+  if (!rows_fit(B, H, N) || N / P > ((int64_t)1 << 30) / 128) return RA_ERR_SHAPE;
   if (B * H * N > kNoAllocScratchFloats) return RA_ERR_SCRATCH;
   if (!(scale > 0.f) || !isfinite(scale)) return RA_ERR_SCALE;
   const void* all[] = {q, k, v, o, dout, lse, dq, dk, dv};
@@ -339,8 +346,7 @@ ra_status ra_attn_fwd_block(const void* q, const void* k, const void* v, void* o
   if (d != 64 && d != 128) return RA_ERR_HEADDIM;
   if (B < 1 || H < 1 || c < 1 || P < 1 || j < 0 || j >= P || kb < 0 || kb >= P)
     return RA_ERR_SHAPE;
-  if (B * H * c >= ((int64_t)1 << 31) || c > ((int64_t)1 << 30) / 128 ||
-      c * (int64_t)P >= ((int64_t)1 << 31))
+  if (!rows_fit(B, H, c) || c > ((int64_t)1 << 30) / 128 || c * (int64_t)P >= ((int64_t)1 << 31))
     return RA_ERR_SHAPE;
   if (!(scale > 0.f) || !isfinite(scale)) return RA_ERR_SCALE;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
@@ -382,7 +388,8 @@ ra_status ra_lse_merge_acc(float* o_acc, float* lse_acc, const void* o_b, const 
   if ((mode & ~3) != 0) return RA_ERR_LAYOUT;
   const int first = mode & RA_MERGE_FIRST, final_ = (mode & RA_MERGE_FINAL) != 0;
   if (final_ && !o_final) return RA_ERR_NULL;
-  if (rows < 0 || d < 8 || d % 8 != 0 || rows >= ((int64_t)1 << 31)) return RA_ERR_SHAPE;
+  if (rows < 0 || d < 8 || d % 8 != 0 || d > (1 << 20) || rows >= ((int64_t)1 << 31))
+    return RA_ERR_SHAPE;
   if (!aligned(o_acc, 16) || !aligned(o_b, 16) || !aligned(lse_acc, 4) || !aligned(lse_b, 4) ||
       (final_ && !aligned(o_final, 16)))
     return RA_ERR_ALIGN;
@@ -403,8 +410,10 @@ ra_status ra_lse_merge_acc(float* o_acc, float* lse_acc, const void* o_b, const 
 
 int64_t ra_attn_fwd_host_workspace(int64_t N, int64_t d, int layout, int64_t heads_per_chunk) {
   if (N < 1 || d < 1 || heads_per_chunk < 1) return -1;
+  if (N >= ((int64_t)1 << 31) || d > 1024) return -1;
   (void)layout;
   const HostPlan h = host_plan(N, d);
+  if (heads_per_chunk > INT64_MAX / (2 * h.per_head)) return -1;
   return 2 * heads_per_chunk * h.per_head;
 }
 
@@ -419,7 +428,7 @@ ra_status ra_attn_fwd_host(const void* q, const void* k, const void* v, void* o,
   if (d != 64 && d != 128) return RA_ERR_HEADDIM;
   if (B < 1 || H < 1 || N < 1 || P < 1 || N % P != 0) return RA_ERR_SHAPE;
   if (base == RA_ZIGZAG && (N / P) % 512 != 0) return RA_ERR_SHAPE;
-  if (B * H * N >= ((int64_t)1 << 31) || N / P > ((int64_t)1 << 30) / 128) return RA_ERR_SHAPE;
+  if (!rows_fit(B, H, N) || N / P > ((int64_t)1 << 30) / 128) return RA_ERR_SHAPE;
   if (!(scale > 0.f) || !isfinite(scale)) return RA_ERR_SCALE;
   if (!aligned(workspace, 256)) return RA_ERR_ALIGN;
   const HostPlan hp = host_plan(N, d);

@@ -230,3 +230,30 @@ def test_o_f32_flag_validation(L):
     tb = 2 * 1024 * 128 * 2
     assert attn(L, o=A - tb - tb // 2, layout=0x201) == 8
     assert attn(L, o=A - tb - tb // 2, layout=0x001) != 8
+
+
+BIG = 1 << 33    # with two more such factors B*H*N wraps around int64
+
+
+@pytest.mark.parametrize("call", [
+    lambda L: attn(L, B=BIG, H=BIG, N=BIG, P=1),
+    lambda L: attn(L, B=1 << 21, H=1 << 21, N=1024),
+    lambda L: host(L, B=BIG, H=BIG, N=BIG, P=1),
+    lambda L: bwd(L, B=BIG, H=BIG, N=BIG, P=1),
+    lambda L: bwd_noalloc(L, B=BIG, H=BIG, N=BIG, P=1),
+    lambda L: blk(L, B=BIG, H=BIG, c=256),
+    lambda L: L.ra_partition(vp(A), vp(Bp), BIG, BIG, BIG, 8, 1, 0, 0, 0, None),
+    lambda L: L.ra_partition(vp(A), vp(Bp), 1, 1, 16, 1 << 62, 4, 0, 0, 0, None),
+    lambda L: prope(L, B=BIG, H=BIG, N=BIG, P=1),
+    lambda L: macc(L, d=1 << 40),
+])
+def test_sizes_that_overflow_int64_are_refused(L, call):
+    # the product of the sizes is checked factor by factor, never computed
+    # past 2^62
+    assert call(L) == 3
+
+
+def test_host_workspace_overflow_is_refused(L):
+    assert L.ra_attn_fwd_host_workspace(1 << 31, 128, 1, 1) == -1
+    assert L.ra_attn_fwd_host_workspace(1024, 2048, 1, 1) == -1
+    assert L.ra_attn_fwd_host_workspace(1 << 30, 128, 1, 1 << 40) == -1
