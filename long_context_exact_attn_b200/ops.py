@@ -108,6 +108,31 @@ def _cuda_contig(t, name):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _like(t, name, shape, dtype, device):
+    """A caller-provided output: CUDA, contiguous, of the expected shape and
+    dtype, on the inputs' device (the library writes exactly that many bytes)."""
+    _cuda_contig(t, name)
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype} of shape {tuple(shape)}")
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}")
+    return t
+
+
+def _same_device(*named):
+    dev = named[0][1].device
+    for n, t in named[1:]:
+        if t.device != dev:
+            raise ValueError(f"{n} is on {t.device}, expected {dev}")
+
+
+def _launch(where, t, fn, *args):
+    """One C entry point, called with t's device current (the library works on
+    the current device); raises on a non-zero status."""
+    with torch.cuda.device(t.device):
+        _check(fn(*args), where)
+
+
 def partition(x, P, layout, inverse=False, out=None):
     """Token order -> layout order (or back, ``inverse=True``) along dim -2 of
     a [B, H, N, d] tensor, or along the only dim of an [N] tensor (position
@@ -124,13 +149,9 @@ def partition(x, P, layout, inverse=False, out=None):
         d = 1
     else:
         raise ValueError("expected [N], [B, H, N] or [B, H, N, d]")
-    if out is None:
-        out = torch.empty_like(x)
-    if out.shape != x.shape or out.dtype != x.dtype:
-        raise ValueError("out must match x in shape and dtype")
-    _cuda_contig(out, "out")
-    _check(lib().ra_partition(_ptr(x), _ptr(out), B, H, N, d, int(P), int(layout), int(bool(inverse)),
-                              _DTYPE_CODE[x.dtype], _stream(x)), "ra_partition")
+    out = torch.empty_like(x) if out is None else _like(out, "out", x.shape, x.dtype, x.device)
+    _launch("ra_partition", x, lib().ra_partition, _ptr(x), _ptr(out), B, H, N, d, int(P),
+            int(layout), int(bool(inverse)), _DTYPE_CODE[x.dtype], _stream(x))
     return out
 
 
@@ -147,24 +168,19 @@ def attn_fwd(q, k, v, P, layout, causal=True, scale=None, sched_free=False, out=
             raise ValueError(f"{n} must be bfloat16")
     if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
         raise ValueError("q, k, v must all be [B, H, N, d] of the same shape")
+    _same_device(("q", q), ("k", k), ("v", v))
     B, H, N, d = q.shape
     if scale is None:
         scale = d ** -0.5
     odt = torch.float32 if o_f32 else torch.bfloat16
-    if out is None:
-        out = torch.empty(q.shape, dtype=odt, device=q.device)
-    if lse is None:
-        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    if out.shape != q.shape or out.dtype != odt:
-        raise ValueError(f"out must be {odt} of q's shape")
-    if lse.shape != (B, H, N) or lse.dtype != torch.float32:
-        raise ValueError("lse must be float32 [B, H, N]")
-    _cuda_contig(out, "out")
-    _cuda_contig(lse, "lse")
+    out = (torch.empty(q.shape, dtype=odt, device=q.device) if out is None
+           else _like(out, "out", q.shape, odt, q.device))
+    lse = (torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None
+           else _like(lse, "lse", (B, H, N), torch.float32, q.device))
     lay = (int(layout) | (SCHED_FREE if sched_free else 0) | (O_F32 if o_f32 else 0)
            | (TOKEN_ORDER if token_order else 0))
-    _check(lib().ra_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, d, int(P),
-                             lay, int(bool(causal)), float(scale), _stream(q)), "ra_attn_fwd")
+    _launch("ra_attn_fwd", q, lib().ra_attn_fwd, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+            B, H, N, d, int(P), lay, int(bool(causal)), float(scale), _stream(q))
     return out, lse
 
 
@@ -180,24 +196,23 @@ def attn_bwd(q, k, v, o, dout, lse, P, layout, causal=True, scale=None, workspac
     if q.dim() != 4:
         raise ValueError("expected [B, H, N, d]")
     B, H, N, d = q.shape
-    _cuda_contig(lse, "lse")
-    if lse.shape != (B, H, N) or lse.dtype != torch.float32:
-        raise ValueError("lse must be float32 [B, H, N]")
+    _like(lse, "lse", (B, H, N), torch.float32, q.device)
+    _same_device(("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout))
     if scale is None:
         scale = d ** -0.5
     if workspace is None:
         workspace = torch.empty(B * H * N, dtype=torch.float32, device=q.device)
-    if workspace.numel() < B * H * N or workspace.dtype != torch.float32:
-        raise ValueError("workspace must hold B*H*N float32")
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(q) if dk is None else dk
-    dv = torch.empty_like(q) if dv is None else dv
-    for n, t in (("dq", dq), ("dk", dk), ("dv", dv), ("workspace", workspace)):
-        _cuda_contig(t, n)
+    _cuda_contig(workspace, "workspace")
+    if workspace.numel() < B * H * N or workspace.dtype != torch.float32 or \
+            workspace.device != q.device:
+        raise ValueError(f"workspace must hold B*H*N float32 on {q.device}")
+    dq = torch.empty_like(q) if dq is None else _like(dq, "dq", q.shape, q.dtype, q.device)
+    dk = torch.empty_like(q) if dk is None else _like(dk, "dk", q.shape, q.dtype, q.device)
+    dv = torch.empty_like(q) if dv is None else _like(dv, "dv", q.shape, q.dtype, q.device)
     lay = int(layout) | (TOKEN_ORDER if token_order else 0)
-    _check(lib().ra_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
-                             _ptr(dk), _ptr(dv), _ptr(workspace), B, H, N, d, int(P), lay,
-                             int(bool(causal)), float(scale), _stream(q)), "ra_attn_bwd")
+    _launch("ra_attn_bwd", q, lib().ra_attn_bwd, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout),
+            _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), B, H, N, d, int(P), lay,
+            int(bool(causal)), float(scale), _stream(q))
     return dq, dk, dv
 
 
@@ -221,16 +236,20 @@ def attn_fwd_host(q, k, v, P, layout, causal=True, scale=None, workspace=None, o
     B, H, N, d = q.shape
     if scale is None:
         scale = d ** -0.5
-    if workspace is None or not workspace.is_cuda:
+    if workspace is None:
         raise ValueError("workspace must be a CUDA tensor")
+    _cuda_contig(workspace, "workspace")
     o = torch.empty(q.shape, dtype=q.dtype, pin_memory=True) if out is None else out
     lse = torch.empty((B, H, N), dtype=torch.float32, pin_memory=True) if lse is None else lse
+    for n, t, shape, dt in (("out", o, q.shape, q.dtype), ("lse", lse, (B, H, N), torch.float32)):
+        if t.is_cuda or not t.is_contiguous() or tuple(t.shape) != tuple(shape) or t.dtype != dt:
+            raise ValueError(f"{n} must be a contiguous host {dt} tensor of shape {tuple(shape)}")
     lay = int(layout) | (SCHED_FREE if sched_free else 0)
     st = torch.cuda.current_stream(workspace.device) if stream is None else stream
-    _check(lib().ra_attn_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
-                                  int(P), lay, int(bool(causal)), float(scale), _ptr(workspace),
-                                  workspace.numel() * workspace.element_size(),
-                                  ctypes.c_void_p(st.cuda_stream)), "ra_attn_fwd_host")
+    _launch("ra_attn_fwd_host", workspace, lib().ra_attn_fwd_host, _ptr(q), _ptr(k), _ptr(v),
+            _ptr(o), _ptr(lse), B, H, N, d, int(P), lay, int(bool(causal)), float(scale),
+            _ptr(workspace), workspace.numel() * workspace.element_size(),
+            ctypes.c_void_p(st.cuda_stream))
     return o, lse
 
 
@@ -242,16 +261,16 @@ def attn_fwd_block(q, k, v, j, kb, P, layout, causal=True, scale=None, out=None,
         _cuda_contig(t, n)
         if t.dtype != torch.bfloat16 or t.dim() != 4 or t.shape != q.shape:
             raise ValueError(f"{n} must be bfloat16 [B, H, c, d] like q")
+    _same_device(("q", q), ("k", k), ("v", v))
     B, H, c, d = q.shape
     if scale is None:
         scale = d ** -0.5
-    o = torch.empty_like(q) if out is None else out
-    lse = torch.empty(B, H, c, dtype=torch.float32, device=q.device) if lse is None else lse
-    _cuda_contig(o, "out")
-    _cuda_contig(lse, "lse")
-    _check(lib().ra_attn_fwd_block(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, c, d,
-                                   int(j), int(kb), int(P), int(layout), int(bool(causal)),
-                                   float(scale), _stream(q)), "ra_attn_fwd_block")
+    o = torch.empty_like(q) if out is None else _like(out, "out", q.shape, q.dtype, q.device)
+    lse = (torch.empty(B, H, c, dtype=torch.float32, device=q.device) if lse is None
+           else _like(lse, "lse", (B, H, c), torch.float32, q.device))
+    _launch("ra_attn_fwd_block", q, lib().ra_attn_fwd_block, _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+            _ptr(lse), B, H, c, d, int(j), int(kb), int(P), int(layout), int(bool(causal)),
+            float(scale), _stream(q))
     return o, lse
 
 
@@ -271,13 +290,13 @@ def lse_merge_acc(o_acc, lse_acc, o_b, lse_b, first=False, final_out=None):
         raise ValueError("lse_acc, lse_b: float32 with one value per row")
     for n, t in (("o_acc", o_acc), ("lse_acc", lse_acc), ("o_b", o_b), ("lse_b", lse_b)):
         _cuda_contig(t, n)
+    _same_device(("o_b", o_b), ("o_acc", o_acc), ("lse_acc", lse_acc), ("lse_b", lse_b))
     mode = (MERGE_FIRST if first else 0) | (MERGE_FINAL if final_out is not None else 0)
     fin = None
     if final_out is not None:
-        _cuda_contig(final_out, "final_out")
-        fin = _ptr(final_out)
-    _check(lib().ra_lse_merge_acc(_ptr(o_acc), _ptr(lse_acc), _ptr(o_b), _ptr(lse_b), fin, rows,
-                                  d, mode, _stream(o_b)), "ra_lse_merge_acc")
+        fin = _ptr(_like(final_out, "final_out", o_b.shape, torch.bfloat16, o_b.device))
+    _launch("ra_lse_merge_acc", o_b, lib().ra_lse_merge_acc, _ptr(o_acc), _ptr(lse_acc),
+            _ptr(o_b), _ptr(lse_b), fin, rows, d, mode, _stream(o_b))
     return o_acc, lse_acc
 
 
@@ -291,10 +310,9 @@ def partition_rope(x, P, layout, base=10000.0, pairing=ROPE_INTERLEAVED, out=Non
     if x.dim() != 4 or x.dtype != torch.bfloat16:
         raise ValueError("x must be bfloat16 [B, H, N, d]")
     B, H, N, d = x.shape
-    out = torch.empty_like(x) if out is None else out
-    _cuda_contig(out, "out")
-    _check(lib().ra_partition_rope(_ptr(x), _ptr(out), B, H, N, d, int(P), int(layout),
-                                   int(pairing), float(base), _stream(x)), "ra_partition_rope")
+    out = torch.empty_like(x) if out is None else _like(out, "out", x.shape, x.dtype, x.device)
+    _launch("ra_partition_rope", x, lib().ra_partition_rope, _ptr(x), _ptr(out), B, H, N, d,
+            int(P), int(layout), int(pairing), float(base), _stream(x))
     return out
 
 
@@ -311,13 +329,12 @@ def attn_bwd_noalloc(q, k, v, o, dout, lse, P, layout, causal, scale, dq, dk, dv
     if q.dim() != 4:
         raise ValueError("expected [B, H, N, d]")
     B, H, N, d = q.shape
-    _cuda_contig(lse, "lse")
-    if lse.shape != (B, H, N) or lse.dtype != torch.float32:
-        raise ValueError("lse must be float32 [B, H, N]")
-    _check(lib().ra_attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
-                                     _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, int(P),
-                                     int(layout), int(bool(causal)), float(scale), _stream(q)),
-           "ra_attn_bwd_noalloc")
+    _like(lse, "lse", (B, H, N), torch.float32, q.device)
+    _same_device(("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout), ("dq", dq), ("dk", dk),
+                 ("dv", dv))
+    _launch("ra_attn_bwd_noalloc", q, lib().ra_attn_bwd_noalloc, _ptr(q), _ptr(k), _ptr(v),
+            _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, int(P),
+            int(layout), int(bool(causal)), float(scale), _stream(q))
     return dq, dk, dv
 
 
@@ -332,15 +349,15 @@ def lse_merge(o_a, lse_a, o_b, lse_b, out=None, lse_out=None):
         raise ValueError("lse_a, lse_b must be float32")
     d = o_a.shape[-1]
     rows = o_a.numel() // d
-    if out is None:
-        out = torch.empty_like(o_a)
-    if lse_out is None:
-        lse_out = torch.empty_like(lse_a)
-    for n, t in (("o_a", o_a), ("lse_a", lse_a), ("o_b", o_b), ("lse_b", lse_b), ("out", out),
-                 ("lse_out", lse_out)):
+    for n, t in (("o_a", o_a), ("lse_a", lse_a), ("o_b", o_b), ("lse_b", lse_b)):
         _cuda_contig(t, n)
-    _check(lib().ra_lse_merge(_ptr(o_a), _ptr(lse_a), _ptr(o_b), _ptr(lse_b), _ptr(out),
-                              _ptr(lse_out), rows, d, _stream(o_a)), "ra_lse_merge")
+    _same_device(("o_a", o_a), ("lse_a", lse_a), ("o_b", o_b), ("lse_b", lse_b))
+    out = (torch.empty_like(o_a) if out is None
+           else _like(out, "out", o_a.shape, torch.bfloat16, o_a.device))
+    lse_out = (torch.empty_like(lse_a) if lse_out is None
+               else _like(lse_out, "lse_out", lse_a.shape, torch.float32, o_a.device))
+    _launch("ra_lse_merge", o_a, lib().ra_lse_merge, _ptr(o_a), _ptr(lse_a), _ptr(o_b),
+            _ptr(lse_b), _ptr(out), _ptr(lse_out), rows, d, _stream(o_a))
     return out, lse_out
 
 
@@ -348,8 +365,8 @@ def tile_census(N, P, layout, causal, device="cuda"):
     """int64 [P, P, 4]: per (query shard j, round r): skipped / full /
     masked tiles and visible pairs, from the attention kernel's classifier."""
     out = torch.empty((P, P, 4), dtype=torch.int64, device=device)
-    _check(lib().ra_tile_census(int(N), int(P), int(layout), int(bool(causal)), _ptr(out),
-                                _stream(out)), "ra_tile_census")
+    _launch("ra_tile_census", out, lib().ra_tile_census, int(N), int(P), int(layout),
+            int(bool(causal)), _ptr(out), _stream(out))
     return out
 
 
@@ -357,7 +374,8 @@ def wait_selftest(limit_ns=100_000_000, device="cuda"):
     """Launch the bounded-wait self-test (a wait that nothing completes)."""
     dev = torch.device(device)
     stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
-    _check(lib().ra_wait_selftest(int(limit_ns), stream), "ra_wait_selftest")
+    with torch.cuda.device(dev):
+        _check(lib().ra_wait_selftest(int(limit_ns), stream), "ra_wait_selftest")
 
 
 def device_fault():
