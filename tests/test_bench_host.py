@@ -25,3 +25,53 @@ def test_recorded_traffic_matches_current_forward_sources():
     assert e["kernel_hash"] == bench.kernel_source_hash()
     assert bench.recorded_traffic("striped_causal_N262144_H16_d128_P16_qk3x") == \
         e["dram_bytes_per_launch"]
+
+
+def _run_bench(args, env_extra=None, timeout=300):
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ)
+    env.update(env_extra or {})
+    return subprocess.run([sys.executable, os.path.join(bench.ROOT, "bench.py")] + args,
+                          capture_output=True, text=True, timeout=timeout, env=env,
+                          cwd=bench.ROOT)
+
+
+def test_reference_arm_prints_one_contract_line():
+    import json
+    r = _run_bench(["--impl", "reference", "--steps", "2", "--warmup", "3", "--ref-budget",
+                    "0.2", "--workload", "striped_causal_N8192_H16_d128_P8"])
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["unit"] == "TFLOP/s"
+    assert line["steps"] == 2 and line["warmup"] == 3 and line["higher_is_better"] is True
+    assert line["config"]["workload"] == "striped_causal_N8192_H16_d128_P8"
+    assert line["value"] > 0 and line["cpu_baseline"]["value"] == line["value"]
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"] == {"value": line["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    # ms_per_step is the whole workload's useful work at the measured rate
+    from long_context_exact_attn_b200 import workloads as W
+    w = W.BY_NAME["striped_causal_N8192_H16_d128_P8"]
+    assert abs(line["ms_per_step"] - w.useful_flops() / (line["value"] * 1e12) * 1e3) < 1e-6 * \
+        line["ms_per_step"]
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    r = _run_bench(["--impl", "reference", "--steps", "1", "--warmup", "3", "--ref-budget",
+                    "0.1", "--workload", "tiny_noncausal_N256_d64_P4"],
+                   env_extra={"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == ""
+
+
+def test_warmup_below_three_is_refused():
+    r = _run_bench(["--impl", "reference", "--steps", "1", "--warmup", "2"])
+    assert r.returncode != 0
