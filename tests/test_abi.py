@@ -257,3 +257,38 @@ def test_host_workspace_overflow_is_refused(L):
     assert L.ra_attn_fwd_host_workspace(1 << 31, 128, 1, 1) == -1
     assert L.ra_attn_fwd_host_workspace(1024, 2048, 1, 1) == -1
     assert L.ra_attn_fwd_host_workspace(1 << 30, 128, 1, 1 << 40) == -1
+
+
+C_CALLER = r"""
+#include "ringattn.h"
+#include <stdio.h>
+int main(void) {
+  if (ra_version() < 100) return 2;
+  if (ra_attn_fwd(0, 0, 0, 0, 0, 1, 1, 16, 64, 4, RA_STRIPED, 1, 0.125f, 0) != RA_ERR_NULL)
+    return 3;
+  if (ra_attn_fwd_host_workspace(1024, 128, RA_STRIPED, 1) <= 0) return 4;
+  printf("%s\n", ra_status_string(RA_ERR_SHAPE));
+  return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links(L, tmp_path):
+    # the boundary is a C ABI: the header compiles as strict C11 and a C
+    # program links against the library and calls it
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "caller.c"
+    src.write_text(C_CALLER)
+    exe = tmp_path / "caller"
+    libdir = os.path.dirname(ops.LIB_PATH)
+    r = subprocess.run([gcc, "-std=c11", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                        "-I", os.path.dirname(HEADER), str(src), "-L", libdir, "-lringattn",
+                        "-Wl,-rpath," + libdir, "-o", str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, (r.returncode, r.stderr)
+    assert r.stdout.strip() == ops.status_string(3)
