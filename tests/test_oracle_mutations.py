@@ -219,3 +219,118 @@ def test_zigzag_mutant_fails_example_and_balance(monkeypatch):
     monkeypatch.setattr(partition, "token_of", wrong)
     with pytest.raises(AssertionError):
         TP2.test_zigzag_example_N16_P4()
+
+
+@pytest.mark.parametrize("kind", ["diagonal_inclusive", "order_swapped"])
+def test_ring_getmask_mutants_fail_position_pin(monkeypatch, kind):
+    def wrong(j, k, c):
+        mask = np.zeros((c, c), dtype=bool)
+        hidden = (j > k) if kind == "order_swapped" else (j < k)
+        if hidden:
+            mask[:, :] = True
+        elif j == k:
+            for x in range(c):
+                for y in range(c):
+                    if (y <= x) if kind == "diagonal_inclusive" else (y < x):
+                        mask[x, y] = True
+        return mask
+    monkeypatch.setattr(masks, "getmask_ring", wrong)
+    with pytest.raises(AssertionError):
+        TP.test_getmask_equals_causal_C_over_positions(CONTIGUOUS, 3, 4)
+
+
+def test_zigzag_getmask_mutant_fails_orientation_pin(monkeypatch):
+    """Planted: the mask blocks a key at the query's own position too."""
+    def wrong(j, k, c, P):
+        N = c * P
+        qpos = np.array([partition.token_of(j, y, N, P, partition.ZIGZAG) for y in range(c)])
+        kpos = np.array([partition.token_of(k, x, N, P, partition.ZIGZAG) for x in range(c)])
+        return kpos[:, None] >= qpos[None, :]
+    monkeypatch.setattr(masks, "getmask_zigzag", wrong)
+    with pytest.raises(AssertionError):
+        TP.test_zigzag_mask_orientation_matches_positions()
+
+
+def test_key_block_mutant_fails_ring_pass_pin(monkeypatch):
+    """Planted: the ring turning the other way (block (j + r) mod P)."""
+    monkeypatch.setattr(work, "key_block", lambda j, r, P: (j + r) % P)
+    with pytest.raises(AssertionError):
+        TP.test_key_block_follows_the_ring_pass(3)
+
+
+def _block_attention_mutant(kind):
+    orig = ring.block_attention
+
+    def f(qj, kb_k, kb_v, j, kb, P, layout, causal, scale):
+        if kind == "pair_swapped":
+            return orig(qj, kb_k, kb_v, kb, j, P, layout, causal, scale)
+        o, lse = orig(qj, kb_k, kb_v, j, kb, P, layout, causal, scale)
+        if kind == "empty_lse_zero":
+            lse = np.where(np.isneginf(lse), 0.0, lse)
+        return o, lse
+    return f
+
+
+@pytest.mark.parametrize("kind", ["pair_swapped", "empty_lse_zero"])
+def test_block_attention_mutants_fail_definition_pin(monkeypatch, kind):
+    import tests.test_oracle_attention as TA2
+    monkeypatch.setattr(ring, "block_attention", _block_attention_mutant(kind))
+    with pytest.raises(AssertionError):
+        TA2.test_block_attention_empty_rows_and_positions()
+
+
+def test_ring_by_merge_mutant_fails_exactness_pin(monkeypatch):
+    """Planted: the last round's partial is never merged."""
+    from oracle.merge import lse_merge
+    from oracle.partition import shard_len
+
+    def wrong(q, k, v, P, layout, causal, scale):
+        q = np.asarray(q, dtype=np.float64)
+        N = q.shape[0]
+        c = shard_len(N, P)
+        out, lse_out = np.empty((N, np.asarray(v).shape[1])), np.empty(N)
+        for j in range(P):
+            o_acc = l_acc = None
+            for r in range(max(P - 1, 1)):
+                kb = (j - r) % P
+                o_r, l_r = ring.block_attention(q[j * c:(j + 1) * c], k[kb * c:(kb + 1) * c],
+                                                v[kb * c:(kb + 1) * c], j, kb, P, layout,
+                                                causal, scale)
+                o_acc, l_acc = (o_r, l_r) if o_acc is None else lse_merge(o_acc, l_acc, o_r, l_r)
+            out[j * c:(j + 1) * c], lse_out[j * c:(j + 1) * c] = o_acc, l_acc
+        return out, lse_out
+    monkeypatch.setattr(ring, "ring_by_merge", wrong)
+    with pytest.raises(AssertionError):
+        TA.test_ring_by_merging_round_partials_equals_full_softmax(STRIPED, True, 24, 4)
+
+
+def test_dq_rows_mutant_fails_full_backward_pin(monkeypatch):
+    """Planted: dQ rows without the softmax scale factor."""
+    from oracle import backward as OB
+    orig = OB.dq_rows
+    monkeypatch.setattr(OB, "dq_rows",
+                        lambda q, k, v, do, scale, causal, rows:
+                        orig(q, k, v, do, scale, causal, rows) / scale)
+    import tests.test_oracle_backward as TB
+    with pytest.raises(AssertionError):
+        TB.test_dq_rows_equal_full_backward(True)
+
+
+def test_tile_census_mutant_fails_brute_force_pin(monkeypatch):
+    """Planted: the diagonal tiles counted as full instead of partial."""
+    orig = work.tile_census_closed_form
+
+    def wrong(j, r, c, P, layout, causal, b):
+        skip, full, part = orig(j, r, c, P, layout, causal, b)
+        return skip, full + part, 0
+    monkeypatch.setattr(work, "tile_census_closed_form", wrong)
+    with pytest.raises(AssertionError):
+        TP.test_tile_census_brute_force_equals_closed_form(STRIPED, True, 8, 4, 2)
+
+
+def test_zigzag_work_mutant_fails_brute_force_pin(monkeypatch):
+    """Planted: the second chunk's own triangle dropped from the total."""
+    monkeypatch.setattr(work, "work_zigzag_device_total",
+                        lambda c, P: (c // 2) ** 2 * (2 * P - 1))
+    with pytest.raises(AssertionError):
+        TP.test_zigzag_work_is_equal_on_every_device(16, 4)

@@ -168,3 +168,17 @@ def test_zigzag_mask_orientation_matches_positions():
         for k in range(P):
             assert np.array_equal(masks.getmask(j, k, c, ZIGZAG, P).T,
                                   masks.mask_from_positions(j, k, N, P, ZIGZAG))
+
+
+@pytest.mark.parametrize("P", [1, 2, 3, 4, 7])
+def test_key_block_follows_the_ring_pass(P):
+    """Ring explainer, ステップ2: every device starts with its own K/V block
+    and, each round, hands the block it holds to device j+1 (receiving from
+    j-1).  Simulating that hand-over round by round gives the block each
+    device holds; key_block(j, r, P) must name the same block."""
+    held = list(range(P))                       # round 0: own block
+    for r in range(P):
+        for j in range(P):
+            assert work.key_block(j, r, P) == held[j], (j, r)
+        held = [held[(j - 1) % P] for j in range(P)]   # receive from j-1
+    assert held == list(range(P))               # after P rounds, back home
