@@ -334,3 +334,48 @@ def test_zigzag_work_mutant_fails_brute_force_pin(monkeypatch):
                         lambda c, P: (c // 2) ** 2 * (2 * P - 1))
     with pytest.raises(AssertionError):
         TP.test_zigzag_work_is_equal_on_every_device(16, 4)
+
+
+def test_attention_rows_mutant_fails_full_pin(monkeypatch):
+    """Planted: a causal row that does not see its own key."""
+    orig = att.attention_rows
+
+    def wrong(q, k, v, scale, causal, rows):
+        if not causal:
+            return orig(q, k, v, scale, causal, rows)
+        o = np.empty((len(rows), np.asarray(v).shape[-1]))
+        lse = np.empty(len(rows))
+        for n, i in enumerate(rows):
+            hi = max(int(i), 1)                  # keys 0..i-1 (row 0 keeps key 0)
+            o[n], lse[n] = (a[0] for a in att.attention(np.asarray(q)[i:i + 1],
+                                                          np.asarray(k)[:hi],
+                                                          np.asarray(v)[:hi], scale, False))
+        return o, lse
+    monkeypatch.setattr(att, "attention_rows", wrong)
+    with pytest.raises(AssertionError):
+        TA.test_attention_rows_equals_full(True)
+
+
+def test_negative_control_mutant_fails(monkeypatch):
+    """Planted: a 'local-only' scheme that in fact sees every key (so the
+    negative control would no longer show the flaw)."""
+    monkeypatch.setattr(att, "local_only_attention",
+                        lambda q, k, v, scale, causal, P, shard_of_row, q_pos=None:
+                        att.attention(q, k, v, scale, causal))
+    with pytest.raises(AssertionError):
+        TA.test_negative_control_local_only_is_wrong(True)
+
+
+def test_rope_partition_mutant_fails_position_pin(monkeypatch):
+    """Planted: the rotation applied at the slot index after striping, i.e.
+    position ids not permuted with the tokens (what the Striped review's
+    位置编码处理 warns against)."""
+    import tests.test_oracle_rope as TR
+    from oracle import rope as R
+
+    def wrong(x, P, layout, base=10000.0, pairing=R.INTERLEAVED):
+        xp = partition.partition(x, P, layout)
+        return R.rope(xp, np.arange(x.shape[-2]), base, pairing)
+    monkeypatch.setattr(R, "rope_partition", wrong)
+    with pytest.raises(AssertionError):
+        TR.test_rotate_then_stripe_equals_stripe_positions_then_rotate(STRIPED)
