@@ -98,11 +98,12 @@ typedef int ra_status;
 #define RA_O_F32 0x200
 
 /* Optional flag for ra_attn_fwd and ra_attn_bwd, OR-ed into `layout`: all
- * their tensors (q, k, v, o, lse; dO and the gradients) are in TOKEN order.  The layout's permutation is then applied inside the
- * kernel (the TMA loads address shard j's rows where the tokens live, the
- * epilogue writes each row to its token position), so no ra_partition pass
- * is needed before or after; results equal the partition / attention /
- * inverse-partition sequence bit for bit. */
+ * their tensors (q, k, v, o, lse; dO and the gradients) are in TOKEN order.
+ * The layout's permutation is then applied inside the kernel (the TMA loads
+ * address shard j's rows where the tokens live, the epilogue writes each row
+ * to its token position), so no ra_partition pass is needed before or after;
+ * results equal the partition / attention / inverse-partition sequence bit
+ * for bit. */
 #define RA_TOKEN_ORDER 0x400
 
 /* Rotation pairs of ra_partition_rope. */
@@ -139,7 +140,8 @@ int ra_version(void);
  *             1: layout order -> token order  (dst[.,.,t(s),:] = src[.,.,s,:])
  *   P         number of shards, 1 <= P <= N, N % P == 0.
  *   d         row length in elements (any value >= 1; use d = 1 for lse or
- *             position ids).
+ *             position ids); d * element size < 2^30.
+ *   B, H, N   >= 1 with B*H*N < 2^31 (else RA_ERR_SHAPE).
  * The result is a pure byte permutation (bit-exact).  RA_CONTIGUOUS is the
  * identity and is performed as a copy.
  */
@@ -164,6 +166,7 @@ ra_status ra_partition(const void* src, void* dst, int64_t B, int64_t H, int64_t
  *   src, dst  device bf16 [B, H, N, d], 16-byte aligned, not overlapping
  *             (RA_ERR_ALIAS).
  *   d         a multiple of 16, 16 <= d <= 512 (else RA_ERR_HEADDIM).
+ *   B, H, N, P  as ra_partition (B*H*N < 2^31, N % P == 0).
  *   base      RoPE base (e.g. 10000), finite and > 1 (else RA_ERR_ROPE).
  *   pairing   RA_ROPE_INTERLEAVED or RA_ROPE_HALF (else RA_ERR_ROPE).
  * Angles are evaluated in double precision, the rotation in fp32, and the
