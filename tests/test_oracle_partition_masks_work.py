@@ -182,3 +182,32 @@ def test_key_block_follows_the_ring_pass(P):
             assert work.key_block(j, r, P) == held[j], (j, r)
         held = [held[(j - 1) % P] for j in range(P)]   # receive from j-1
     assert held == list(range(P))               # after P rounds, back home
+
+
+def _ring_time(c, P, layout, brute):
+    """Sum over rounds of the busiest device's unmasked pairs (each round
+    lasts as long as its slowest device: Striped review, 问题定义)."""
+    total = 0
+    for r in range(P):
+        if brute:
+            total += max(work.work_brute_force(j, r, c * P, P, layout) for j in range(P))
+        else:
+            total += max(work.work_exact_closed_form(j, r, c, P, layout) for j in range(P))
+    return total
+
+
+def test_striped_speedup_over_ring_approaches_two():
+    """Striped review, 理论最大加速比: as the block size and the device count
+    grow, Striped over Ring tends to 2x.  Per-round maxima of the exact
+    counts give ring = c(c+1)/2 + (P-1) c^2 and striped = P c(c+1)/2; the
+    ratio grows with c and P and stays below 2."""
+    for c, P in ((1, 2), (3, 4), (8, 3), (6, 6)):
+        ring_t, striped_t = _ring_time(c, P, CONTIGUOUS, True), _ring_time(c, P, STRIPED, True)
+        assert ring_t == c * (c + 1) // 2 + (P - 1) * c * c
+        assert striped_t == P * c * (c + 1) // 2
+    prev = 0.0
+    for c, P in ((4, 2), (16, 4), (64, 8), (256, 16), (1024, 64), (4096, 256)):
+        s = _ring_time(c, P, CONTIGUOUS, False) / _ring_time(c, P, STRIPED, False)
+        assert prev < s < 2.0
+        prev = s
+    assert prev > 1.99
