@@ -24,29 +24,31 @@ import numpy as np
 from .partition import CONTIGUOUS, STRIPED, ZIGZAG, token_of
 
 
+def _key_query_grid(c):
+    """Index grids in the printed orientation: x (key-local) down the rows,
+    y (query-local) along the columns."""
+    return np.arange(c)[:, None], np.arange(c)[None, :]
+
+
 def getmask_ring(j, k, c):
-    """GETMASKRINGATTENTION(j, k): MASK[x (key), y (query)], True = -inf."""
-    mask = np.zeros((c, c), dtype=bool)
-    if j < k:
-        mask[:, :] = True
-    elif j == k:
-        for x in range(c):
-            for y in range(c):
-                if y < x:
-                    mask[x, y] = True
-    return mask
+    """Ring (contiguous) block mask, MASK[x (key), y (query)], True = -inf.
+
+    A later key block (j < k) is hidden entirely, the diagonal block (j = k)
+    hides a key that comes after the query (y < x), an earlier block hides
+    nothing."""
+    x, y = _key_query_grid(c)
+    return np.broadcast_to((j < k) | ((j == k) & (y < x)), (c, c)).copy()
 
 
 def getmask_striped(j, k, c):
-    """GETMASKSTRIPEDATTENTION(j, k): MASK[x (key), y (query)], True = -inf."""
-    mask = np.zeros((c, c), dtype=bool)
-    for x in range(c):
-        for y in range(c):
-            if j < k and y <= x:
-                mask[x, y] = True
-            elif j >= k and y < x:
-                mask[x, y] = True
-    return mask
+    """Striped block mask, MASK[x (key), y (query)], True = -inf.
+
+    Every block pair has the same shape of mask, a triangle whose diagonal is
+    hidden only when the key shard comes after the query shard: hidden where
+    y < x + e, with e = 1 for j < k and e = 0 for j >= k."""
+    x, y = _key_query_grid(c)
+    e = 1 if j < k else 0
+    return y < x + e
 
 
 def getmask_zigzag(j, k, c, P):
