@@ -45,6 +45,10 @@
  *     exceptions share library state: ra_attn_bwd_noalloc's scratch (calls
  *     must not overlap on the GPU) and ra_attn_fwd_host's copy streams
  *     (calls on one device are enqueued one at a time).
+ *   - Per device the library looks up, once, the device addresses of its
+ *     static data (and creates ra_attn_fwd_host's copy streams); it keeps
+ *     them until the process exits, so it must not be used on a device
+ *     after a cudaDeviceReset of that device.
  */
 #ifndef RINGATTN_H_
 #define RINGATTN_H_
@@ -253,8 +257,10 @@ ra_status ra_attn_bwd(const void* q, const void* k, const void* v, const void* o
  *   B * H * N must be <= 1048576, else RA_ERR_SCRATCH (nothing launched).
  *   The first call on a device looks up the array's device address (with
  *   that device current); make that first call before any stream capture.
- *   All calls share the one array: calls whose kernels overlap on the GPU
- *   race on it and give wrong results; order them on one stream.
+ *   All calls on one device share that device's array: calls whose kernels
+ *   overlap on the same GPU race on it and give wrong results; order them on
+ *   one stream.  The looked-up address is kept for the life of the process:
+ *   do not use the library across a cudaDeviceReset of that device.
  */
 ra_status ra_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
                               const void* dout, const float* lse, void* dq, void* dk, void* dv,
@@ -409,6 +415,27 @@ ra_status ra_device_fault(int* code);
  *   limit_ns  1000 <= limit_ns <= 1e10, else RA_ERR_SHAPE.
  */
 ra_status ra_wait_selftest(int64_t limit_ns, void* stream);
+
+/*
+ * ra_attn_abort_selftest -- exercise the attention kernel's own abort path.
+ *
+ * Not an operation of the pages: a diagnostic for the library's failure
+ * detection.  Runs ra_attn_fwd on the given arguments (same meaning, layout,
+ * ownership and validation) with one change: in every CTA the MMA warp
+ * never signals that the first tile's scores are ready, so the softmax warps'
+ * wait for them cannot complete.  The kernel's main-loop waits give up after
+ * limit_ns of wall time; every role of the CTA then stops, the CTA waits for
+ * its own tensor-core operations and TMA loads in flight (those waits keep
+ * the normal 2 s limit), frees its tensor memory, records fault code 1 in the
+ * device fault word and returns.  The outputs are incomplete.  Read the code
+ * with ra_device_fault(); the CUDA context stays usable.
+ *
+ *   limit_ns  1000 <= limit_ns <= 1e10, else RA_ERR_SHAPE.
+ */
+ra_status ra_attn_abort_selftest(const void* q, const void* k, const void* v, void* o,
+                                 float* lse, int64_t B, int64_t H, int64_t N, int64_t d, int P,
+                                 int layout, int causal, float scale, int64_t limit_ns,
+                                 void* stream);
 
 #ifdef __cplusplus
 }

@@ -201,9 +201,10 @@ ra_status ra_partition_rope(const void* src, void* dst, int64_t B, int64_t H, in
                                stream);
 }
 
-ra_status ra_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
-                      int64_t B, int64_t H, int64_t N, int64_t d, int P, int layout, int causal,
-                      float scale, void* stream) {
+// Validates ra_attn_fwd's arguments and fills the launch description.
+static ra_status fwd_prepare(const void* q, const void* k, const void* v, void* o, float* lse,
+                             int64_t B, int64_t H, int64_t N, int64_t d, int P, int layout,
+                             int causal, float scale, void* stream, AttnLaunch* out) {
   if (!q || !k || !v || !o || !lse) return RA_ERR_NULL;
   if (layout & ~(0xff | RA_SCHED_FREE | RA_O_F32 | RA_TOKEN_ORDER)) return RA_ERR_LAYOUT;
   const int base = layout & 0xff;
@@ -240,6 +241,30 @@ ra_status ra_attn_fwd(const void* q, const void* k, const void* v, void* o, floa
   a.device = dev;
   a.num_sms = info.num_sms;
   a.stream = stream;
+  *out = a;
+  return RA_OK;
+}
+
+ra_status ra_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                      int64_t B, int64_t H, int64_t N, int64_t d, int P, int layout, int causal,
+                      float scale, void* stream) {
+  AttnLaunch a;
+  const ra_status st = fwd_prepare(q, k, v, o, lse, B, H, N, d, P, layout, causal, scale, stream,
+                                   &a);
+  return st ? st : attn_fwd_launch(a);
+}
+
+ra_status ra_attn_abort_selftest(const void* q, const void* k, const void* v, void* o,
+                                 float* lse, int64_t B, int64_t H, int64_t N, int64_t d, int P,
+                                 int layout, int causal, float scale, int64_t limit_ns,
+                                 void* stream) {
+  if (limit_ns < 1000 || limit_ns > 10000000000LL) return RA_ERR_SHAPE;
+  AttnLaunch a;
+  const ra_status st = fwd_prepare(q, k, v, o, lse, B, H, N, d, P, layout, causal, scale, stream,
+                                   &a);
+  if (st) return st;
+  a.main_limit_ns = limit_ns;
+  a.withhold_first_s = 1;
   return attn_fwd_launch(a);
 }
 

@@ -65,7 +65,11 @@ struct AttnParams {
   int groups;         // shard groups (owner schedule) or 1 (free schedule)
   int ctas_per_group;
   float c2;           // scale * log2(e)
-  unsigned long long timeout_ns;
+  unsigned long long timeout_ns;        // limit of every main-loop wait
+  unsigned long long drain_timeout_ns;  // limit of the waits that drain the CTA's own
+                                        // MMAs and TMA loads before it exits
+  int withhold_first_s;                 // self-test: the first S-ready signal of every
+                                        // CTA is never sent (the waits must give up)
   // Single-block mode (blk_kb >= 0): Q is one query shard, K/V one key
   // block (both stored as shard 0 of a P = 1 tensor); the mask is the
   // GetMask of the real pair (blk_j, blk_kb).
@@ -241,15 +245,6 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
-}
-
-// acc += bf16 value (mixed-precision add: bf16 operand, fp32 accumulator).
-__device__ __forceinline__ float add_bf16(float acc, unsigned short h) {
-  asm("add.rn.f32.bf16 %0, %1, %0;" : "+f"(acc) : "h"(h));
-  return acc;
-}
-__device__ __forceinline__ void split_bf16x2(uint32_t v, unsigned short& lo, unsigned short& hi) {
-  asm("mov.b32 {%0, %1}, %2;" : "=h"(lo), "=h"(hi) : "r"(v));
 }
 
 // r[i] *= alpha for 32 fp32 values held as raw bits (packed f32x2 multiplies).
@@ -465,7 +460,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       volatile int no_abort = 0;
       const uint32_t first = n_loads > (uint32_t)C::kSlots ? n_loads - C::kSlots : 0;
       for (uint32_t n = first; n < n_loads; ++n)
-        mbar_wait(bar_full(n % C::kSlots), (n / C::kSlots) & 1, &no_abort, p.timeout_ns);
+        mbar_wait(bar_full(n % C::kSlots), (n / C::kSlots) & 1, &no_abort, p.drain_timeout_ns);
     }
     __syncwarp();
   } else if (warp == 9) {
@@ -481,6 +476,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const uint32_t s_full0 = bar_s_full, s_full1 = bar_s_full + 8;
       const uint32_t p_full0 = bar_p_full, p_full1 = bar_p_full + 8;
       const uint32_t p_full2_0 = bar_p_full2, p_full2_1 = bar_p_full2 + 8;
+      bool withhold = p.withhold_first_s != 0;
       const uint32_t o_free0 = bar_o_free, o_free1 = bar_o_free + 8;
       const uint32_t full0 = bars + 2 * 8, empty0 = bars + (2 + C::kSlots) * 8;
       uint32_t slot = 0, phase = 0;       // next K/V tile to consume, in producer order
@@ -518,7 +514,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (!wmbar_wait(full0 + 8 * kslot, phase, abort_flag, p.timeout_ns)) { ok = false; break; }
         tc_fence_after();
         const uint32_t ka0 = sRing + kslot * C::kTileBytes;
-        if (c0 != TILE_SKIP) { mma_qk<D>(tS0, sQ0, ka0); mma_commit_w(s_full0); }
+        if (c0 != TILE_SKIP) {
+          mma_qk<D>(tS0, sQ0, ka0);
+          if (!withhold) mma_commit_w(s_full0);
+          withhold = false;
+        }
         if (c1 != TILE_SKIP) { mma_qk<D>(tS1, sQ1, ka0); mma_commit_w(s_full1); }
         mma_commit_w(empty0 + 8 * kslot);
         if (++slot == C::kSlots) { slot = 0; phase ^= 1; }
@@ -589,7 +589,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       // All MMAs issued by this thread must be complete before TMEM is freed.
       mma_commit_w(bar_drain);
       volatile int no_abort = 0;
-      wmbar_wait(bar_drain, 0, &no_abort, p.timeout_ns);
+      wmbar_wait(bar_drain, 0, &no_abort, p.drain_timeout_ns);
     }
     __syncwarp();
   } else {
@@ -621,7 +621,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       while (seq.next(kb, y0, k0, k1, bm)) {
         const int kind = t ? k1 : k0;
         if (kind == TILE_SKIP) continue;
-        if (!mbar_wait(my_s_full, s_cnt & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+        // warp-uniform: a lane that gives up makes the whole warp give up, so
+        // the warp-collective TMEM accesses and votes below never diverge
+        if (!wmbar_wait(my_s_full, s_cnt & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
         ++s_cnt;
         tc_fence_after();
         uint32_t sr[4][32];
@@ -729,7 +731,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
       if (!ok) break;
       // --------------------------------------------------------- epilogue
-      if (!mbar_wait(my_o_full, k & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+      if (!wmbar_wait(my_o_full, k & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
       tc_fence_after();
       const bool valid = x < p.c;
       // a row that saw no key (possible only for a single block) gets O = 0
@@ -844,7 +846,9 @@ static ra_status launch(const AttnLaunch& a) {
   p.zigzag = a.zigzag;
   p.causal = a.causal;
   p.c2 = (float)((double)a.scale * 1.4426950408889634074);
-  p.timeout_ns = 2000000000ull;
+  p.drain_timeout_ns = 2000000000ull;
+  p.timeout_ns = a.main_limit_ns > 0 ? (unsigned long long)a.main_limit_ns : p.drain_timeout_ns;
+  p.withhold_first_s = a.withhold_first_s;
   p.blk_j = a.blk_j;
   p.blk_kb = a.blk_kb;
   const long long items_total = (long long)p.npairs * a.P * a.BH;

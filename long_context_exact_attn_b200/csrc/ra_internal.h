@@ -33,6 +33,8 @@ struct AttnLaunch {
   int zigzag = 0;                // zigzag layout (striped == 0)
   int o_f32 = 0;                 // write O as float32
   int tok = 0;                   // q, k, v, o, lse in token order
+  int64_t main_limit_ns = 0;     // > 0: limit of the main-loop waits (abort self-test)
+  int withhold_first_s = 0;      // abort self-test: first S-ready signal never sent
 };
 
 ra_status attn_fwd_launch(const AttnLaunch& a);

@@ -78,6 +78,9 @@ def lib():
         L.ra_tile_census.argtypes = [i64, i32, i32, i32, vp, vp]
         L.ra_wait_selftest.restype = i32
         L.ra_wait_selftest.argtypes = [i64, vp]
+        L.ra_attn_abort_selftest.restype = i32
+        L.ra_attn_abort_selftest.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, i32,
+                                             i32, f32, i64, vp]
         L.ra_device_fault.restype = i32
         L.ra_device_fault.argtypes = [ctypes.POINTER(ctypes.c_int)]
         _lib = L
@@ -376,6 +379,26 @@ def wait_selftest(limit_ns=100_000_000, device="cuda"):
     stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
     with torch.cuda.device(dev):
         _check(lib().ra_wait_selftest(int(limit_ns), stream), "ra_wait_selftest")
+
+
+def attn_abort_selftest(q, k, v, P, layout, causal=True, limit_ns=1_000_000, out=None,
+                        lse=None):
+    """Launch the attention kernel with its first S-ready signal withheld in
+    every CTA: the main-loop waits give up after ``limit_ns``, the kernel
+    drains and returns with fault code 1 (read it with ``device_fault``).
+    Same arguments as attn_fwd (layout order)."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _cuda_contig(t, n)
+        if t.dtype != torch.bfloat16 or t.shape != q.shape or t.dim() != 4:
+            raise ValueError(f"{n} must be bfloat16 [B, H, N, d] like q")
+    B, H, N, d = q.shape
+    out = torch.empty_like(q) if out is None else _like(out, "out", q.shape, q.dtype, q.device)
+    lse = (torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None
+           else _like(lse, "lse", (B, H, N), torch.float32, q.device))
+    _launch("ra_attn_abort_selftest", q, lib().ra_attn_abort_selftest, _ptr(q), _ptr(k), _ptr(v),
+            _ptr(out), _ptr(lse), B, H, N, d, int(P), int(layout), int(bool(causal)),
+            float(d ** -0.5), int(limit_ns), _stream(q))
+    return out, lse
 
 
 def device_fault():

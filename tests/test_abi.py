@@ -77,6 +77,19 @@ def test_attn_fwd_rejects_invalid_arguments(L, kw, code):
     assert attn(L, **kw) == code
 
 
+@pytest.mark.parametrize("kw,limit,code", [
+    (dict(q=0), 1_000_000, 1), (dict(d=96), 1_000_000, 4), (dict(layout=3), 1_000_000, 5),
+    (dict(), 10, 3), (dict(), 20_000_000_000, 3),
+])
+def test_abort_selftest_validates_like_attn_fwd(L, kw, limit, code):
+    a = dict(q=A, k=Bp, v=Cp, o=Op, lse=Lp, B=1, H=2, N=1024, d=128, P=4, layout=0, causal=1,
+             scale=0.088)
+    a.update(kw)
+    assert L.ra_attn_abort_selftest(vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["o"]), vp(a["lse"]),
+                                    a["B"], a["H"], a["N"], a["d"], a["P"], a["layout"],
+                                    a["causal"], a["scale"], limit, None) == code
+
+
 def test_partition_rejects_invalid_arguments(L):
     P = L.ra_partition
     assert P(None, vp(Bp), 1, 1, 16, 4, 4, 1, 0, 0, None) == 1
