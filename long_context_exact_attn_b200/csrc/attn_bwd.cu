@@ -995,9 +995,10 @@ ra_status attn_bwd_launch(const BwdLaunch& a) {
 // For callers that must not allocate device memory themselves: the scratch
 // row vector D of the backward lives in this fixed device array instead of a
 // caller workspace.  Every GPU that loads the library reserves it until the
-// process exits.  All calls share it: two calls whose kernels overlap on the
-// GPU (different streams, or devices sharing nothing but this library) race
-// on it.  D is fully rewritten by every call, so nothing has to be cleared.
+// process exits.  All calls on one device share that device's copy: two
+// calls whose kernels overlap on the same GPU (another stream, or another
+// host thread) race on it; calls on different devices use separate copies.
+// D is fully rewritten by every call, so nothing has to be cleared.
 static __device__ __align__(256) float g_bwd_scratch[kNoAllocScratchFloats];
 
 ra_status attn_bwd_noalloc_launch(BwdLaunch a) {

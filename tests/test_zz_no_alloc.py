@@ -4,7 +4,9 @@ Runs on the GPU through the C-ABI and compares the allocation-free entry point
 with ra_attn_bwd (same inputs, caller workspace) on two calls in a row, each
 within the backward tolerance of the parity tests: max |g - g_ref| <= 2e-2 *
 max|g_ref| and mean |g - g_ref| <= 2e-3 * max|g_ref| per tensor.  The two
-paths run the same kernels, so in practice they agree bit for bit.  The
+paths run the same kernels, so in practice they agree bit for bit; each call's
+gradients are therefore also checked against the fp64 oracle's gradients of
+the plain definition, so that an error common to both paths would show.  The
 second call uses other inputs, so stale contents of the shared scratch from
 the first call would show.
 """
@@ -15,6 +17,7 @@ import torch
 
 from long_context_exact_attn_b200 import ops
 from long_context_exact_attn_b200 import workloads as W
+from oracle import backward as OB
 
 pytestmark = pytest.mark.gpu
 
@@ -38,6 +41,21 @@ def _inputs(w, seed):
     return q, k, v, o, do, lse
 
 
+def _oracle_grads(w, do_seed):
+    """The fp64 oracle's dQ, dK, dV of the same token-order inputs."""
+    q, k, v = W.make_qkv(w)
+    do = torch.randn(q.shape, generator=torch.Generator().manual_seed(do_seed)).to(torch.bfloat16)
+    out = [np.empty(q.shape) for _ in range(3)]
+    for b in range(w.B):
+        for h in range(w.H):
+            g = OB.attention_backward(q[b, h].double().numpy(), k[b, h].double().numpy(),
+                                      v[b, h].double().numpy(), do[b, h].double().numpy(),
+                                      w.scale, w.causal)
+            for t in range(3):
+                out[t][b, h] = g[t]
+    return out
+
+
 def _close(got, ref, what):
     for name, g, r in zip(("dq", "dk", "dv"), got, ref):
         g, r = g.float().cpu().numpy(), r.float().cpu().numpy()
@@ -59,6 +77,9 @@ def test_noalloc_matches_workspace_backward_twice():
         torch.cuda.synchronize()
         assert ops.device_fault() == 0
         _close(got, ref, f"call {call} ({w.name})")
+        tok = [ops.partition(g, w.P, w.layout, inverse=True) for g in got]
+        _close(tok, [torch.from_numpy(a) for a in _oracle_grads(w, 100 + call)],
+               f"call {call} ({w.name}) against the oracle")
 
 
 def test_noalloc_rejects_more_rows_than_its_scratch():
