@@ -38,6 +38,7 @@ import torch  # noqa: E402
 
 from long_context_exact_attn_b200 import workloads as W  # noqa: E402
 
+L2_BYTES = 126 * 2 ** 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 SPEC_BF16_TFLOPS = 2250.0
 METRIC = "causal attn fwd useful TFLOP/s & % BF16 tensor peak; tokens/s (1×B200)"
@@ -161,39 +162,103 @@ def oracle_head(w, h):
     return h, q.double().numpy(), k.double().numpy(), v.double().numpy()
 
 
-def cpu_oracle_rate(w, budget_s, seed=0, head=None):
+def structured_rows(w):
+    """Token indices of rows whose handling differs in the kernel: row 0 and
+    the last row, every shard's first and last local row, and the rows on
+    both sides of shard 0's first tile edges (layout terms)."""
+    from oracle import partition as OP
+
+    lay = {W.CONTIGUOUS: OP.CONTIGUOUS, W.STRIPED: OP.STRIPED, W.ZIGZAG: OP.ZIGZAG}[w.layout]
+    slots = {0, w.N - 1}
+    for j in range(w.P):
+        slots.update({j * w.c, j * w.c + w.c - 1})
+    for x in (127, 128, 255, 256):
+        if x < w.c:
+            slots.add(x)
+    return sorted({OP.token_of(s // w.c, s % w.c, w.N, w.P, lay) for s in slots})
+
+
+def cpu_oracle_leg(w, budget_s, seed=0, head=None):
     """Run the oracle's plain definition row by row on a bounded sample of
-    the workload; returns (useful TFLOP/s, description, threads)."""
+    the workload: the structured rows first, then uniformly random rows until
+    the time budget is spent.  Returns (useful TFLOP/s, description, threads,
+    (head, rows, o, lse)) -- the oracle's rows are kept so the caller can
+    compare the GPU's output with them."""
     from threadpoolctl import threadpool_info
 
     from oracle import attention as OA
 
     rng = np.random.default_rng(seed)
     h, qn, kn, vn = head if head is not None else oracle_head(w, int(rng.integers(0, w.H)))
-    rows = np.sort(rng.choice(w.N, size=min(w.N, 4096), replace=False))
-    done, flops = 0, 0
+    first = structured_rows(w)
+    rest = rng.permutation(w.N)[:4096]
+    order = first + [int(i) for i in rest if int(i) not in set(first)]
+    rows, os_, ls_ = [], [], []
+    flops = 0
     t0 = time.perf_counter()
-    for i in rows:
-        OA.attention_rows(qn, kn, vn, w.scale, w.causal, [int(i)])
+    for i in order[:4096]:
+        o, lse = OA.attention_rows(qn, kn, vn, w.scale, w.causal, [int(i)])
+        rows.append(int(i))
+        os_.append(o[0])
+        ls_.append(lse[0])
         flops += 4 * w.d * ((int(i) + 1) if w.causal else w.N)
-        done += 1
         if time.perf_counter() - t0 > budget_s:
             break
     dt = time.perf_counter() - t0
     threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
-    desc = (f"{done} query rows of head {h} (uniform random over the sequence) of {w.name}, "
-            f"each against all its visible keys; fp64 NumPy oracle; {dt:.1f} s")
-    return flops / dt / 1e12, desc, threads
+    desc = (f"{len(rows)} query rows of head {h} of {w.name} ({len(first)} structured: row 0, "
+            f"shard edges, tile edges; the rest uniform random), each against all its visible "
+            f"keys; fp64 NumPy oracle; {dt:.1f} s")
+    return flops / dt / 1e12, desc, threads, (h, rows, np.array(os_), np.array(ls_))
 
 
-def run_reference(args, w, rank):
+O_MAX, O_MEAN, LSE_MAX = 2e-2, 2e-3, 1e-3
+
+
+def parity_of(o_gpu, lse_gpu, v0, ref):
+    """Element-wise errors of the GPU's O and lse (token order, [B, H, N, d]
+    and [B, H, N]) against the oracle rows of one head."""
+    h, rows, o_ref, lse_ref = ref
+    idx = torch.tensor(rows, dtype=torch.long, device=o_gpu.device)
+    o = o_gpu[0, h].index_select(0, idx).double().cpu().numpy()
+    lse = lse_gpu[0, h].index_select(0, idx).double().cpu().numpy()
+    err = np.abs(o - o_ref)
+    lerr = np.abs(lse - lse_ref)
+    row0 = None
+    if 0 in rows and v0 is not None:
+        row0 = bool(np.array_equal(o[rows.index(0)], v0))
+    return {"head": h, "rows": len(rows), "o_max_abs": float(err.max()),
+            "o_mean_abs": float(err.mean()), "lse_max_abs": float(lerr.max()),
+            "tolerance": {"o_max_abs": O_MAX, "o_mean_abs": O_MEAN, "lse_max_abs": LSE_MAX},
+            "within": bool(err.max() <= O_MAX and err.mean() <= O_MEAN and lerr.max() <= LSE_MAX),
+            "row0_equals_v0": row0,
+            "reference": "fp64 oracle, plain definition, same bf16 inputs"}
+
+
+def config_of(w, sched, world):
+    """The line's config object (shared by both arms, so the two lines name
+    the same workload the same way)."""
+    in_bytes = 3 * w.B * w.H * w.N * w.d * 2
+    if in_bytes < 4 * L2_BYTES:
+        l2 = (f"inputs ({in_bytes / 2 ** 20:.0f} MiB) not much larger than L2: a "
+              f"{2 * L2_BYTES / 2 ** 20:.0f} MiB buffer is written before every timed step, "
+              f"outside the timed window")
+    else:
+        l2 = f"inputs ({in_bytes / 2 ** 30:.1f} GiB) larger than L2; no flush"
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "P": w.P,
+            "layout": w.layout_name, "causal": w.causal, "schedule": sched,
+            "step": "partition q,k,v -> attention -> unpartition o,lse", "l2": l2,
+            "parallelism": f"replicas x{world}"}
+
+
+def run_reference(args, w, rank, world):
     if rank != 0:
         return
     vals = []
     desc = threads = None
     head = oracle_head(w, w.H - 1)
     for i in range(args.warmup + args.steps):
-        rate, desc, threads = cpu_oracle_rate(w, args.ref_budget, seed=i, head=head)
+        rate, desc, threads, _ = cpu_oracle_leg(w, args.ref_budget, seed=i, head=head)
         if i >= args.warmup:
             vals.append(rate)
     val = statistics.mean(vals)
@@ -201,9 +266,11 @@ def run_reference(args, w, rank):
         "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": w.useful_flops() / (val * 1e12) * 1e3,
+        "ms_per_step_kind": "extrapolated_from_rows",
+        "ms_per_step_note": "each step runs a bounded row sample of the workload; ms_per_step is "
+                            "the whole workload's useful work at the measured row rate",
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N,
-                                        "d": w.d, "P": w.P, "layout": w.layout_name},
+        "data": "synthetic", "config": config_of(w, args.sched, world),
         "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -281,9 +348,6 @@ def job_value(flops_per_rank, ms_max, world):
     return flops_per_rank * world / (ms_max * 1e-3) / 1e12
 
 
-L2_BYTES = 126 * 2 ** 20
-
-
 def timed(fn, steps, world, flush=None):
     """Mean device time of fn over `steps` runs, max over ranks.  With
     `flush`, L2 is overwritten before every run and each run is timed on its
@@ -314,6 +378,35 @@ def timed(fn, steps, world, flush=None):
     return max_over_ranks(ms, world)
 
 
+def workload_leg(ops, w2, sched, world, steps):
+    """One of the other configurations of the method's evaluation, timed the
+    same way as the headline step (partition -> attention -> un-partition,
+    L2 flushed before every step when the inputs are near L2 size)."""
+    q2, k2, v2 = W.make_qkv(w2)
+    pth = Path(ops, w2, q2, k2, v2, sched_free=(sched == "free"))
+    in_bytes = 3 * q2.numel() * q2.element_size()
+    flush = None
+    if in_bytes < 4 * L2_BYTES:
+        flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+        flush = flush_buf.zero_
+    for _ in range(3):
+        pth.step()
+    torch.cuda.synchronize()
+    ms = timed(lambda: pth.step(time_attn=True), steps, world, flush=flush)
+    attn = pth.attn_ms()
+    am = max_over_ranks(statistics.median(attn), world)
+    fl = w2.useful_flops()
+    out = {"step_ms": round(ms, 4), "attn_ms_median": round(am, 4),
+           "useful_tflops_step": round(fl * world / (ms * 1e-3) / 1e12, 1),
+           "useful_tflops_attn": round(fl / (am * 1e-3) / 1e12, 1),
+           "tokens_per_s": w2.B * w2.N * world / (ms * 1e-3),
+           "layout": w2.layout_name, "schedule": sched, "causal": w2.causal,
+           "l2_flush": flush is not None, "steps": steps}
+    if ops.device_fault():
+        raise RuntimeError(f"device fault in workload {w2.name}")
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -327,14 +420,19 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-chunks", type=int, default=8,
                     help="head chunks of the host-buffer path (copies overlap compute)")
-    ap.add_argument("--ring-emulate", action="store_true",
-                    help="time every (rank, round) block of the physical ring on this GPU")
+    ap.add_argument("--no-ring-emulate", action="store_true",
+                    help="skip timing every (rank, round) block of the physical ring")
     ap.add_argument("--no-rope", action="store_true",
                     help="skip timing the stripe + RoPE partition of q")
-    ap.add_argument("--backward", action="store_true",
-                    help="also time the backward pass (dQ, dK, dV) on the same workload")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip timing the backward pass (dQ, dK, dV) on the same workload")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip timing the other configurations of the evaluation")
     ap.add_argument("--ref-budget", type=float, default=15.0,
                     help="seconds of CPU work per reference step")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override the workload's head count (a reduced case of the same "
+                         "per-head shape, e.g. for counter captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -343,9 +441,11 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     w = W.BY_NAME[args.workload]
+    if args.heads is not None and args.heads != w.H:
+        w = w.with_(H=args.heads, name=f"{w.name}_H{args.heads}")
 
     if args.impl == "reference":
-        run_reference(args, w, rank)
+        run_reference(args, w, rank, world)
         return
 
     from long_context_exact_attn_b200 import ops
@@ -359,6 +459,7 @@ def main():
                                 device_id=torch.device("cuda", local))
     ops.lib()
     peaks, peaks_src = load_peaks()
+    config = config_of(w, args.sched, world)
 
     q, k, v = W.make_qkv(w)
     path = Path(ops, w, q, k, v, sched_free=(args.sched == "free"))
@@ -368,11 +469,6 @@ def main():
     if in_bytes < 4 * L2_BYTES:
         flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
         flush = flush_buf.zero_
-        l2_note = (f"inputs ({in_bytes / 2 ** 20:.0f} MiB) not much larger than L2: a "
-                   f"{2 * L2_BYTES / 2 ** 20:.0f} MiB buffer is written before every timed step, "
-                   f"outside the timed window")
-    else:
-        l2_note = f"inputs ({in_bytes / 2 ** 30:.1f} GiB) larger than L2; no flush"
 
     for _ in range(args.warmup):
         path.step()
@@ -393,13 +489,17 @@ def main():
     flops = w.useful_flops()
     value = job_value(flops, ms, world)
     tokens_s = w.B * w.N * world / (ms * 1e-3)
+    # the timed step's output (token order), kept on the host for the
+    # comparison with the oracle's rows at the end
+    o_step = path.o.cpu()
+    lse_step = path.lse.cpu()
 
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
         # ra_attn_fwd_host: token-order host q, k, v in, host o, lse out; the
-        # heads go through a device workspace in chunks of a quarter of the
-        # heads, copies of neighbouring chunks overlapping the compute
+        # heads go through a device workspace in chunks, copies of
+        # neighbouring chunks overlapping the compute
         hq, hk, hv = (t.pin_memory() for t in (q, k, v))
         ho = torch.empty(path.o.shape, dtype=path.o.dtype).pin_memory()
         hl = torch.empty(path.lse.shape, dtype=path.lse.dtype).pin_memory()
@@ -413,14 +513,53 @@ def main():
 
         e2e_step()
         torch.cuda.synchronize()
-        e2e_ms = timed(e2e_step, max(1, min(args.steps, 5)), world)
+        n_e2e = max(1, min(args.steps, 5))
+        e2e_ms = timed(e2e_step, n_e2e, world)
         del ws
         torch.cuda.empty_cache()
         h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
         d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+        # Its parts, each timed alone: the attention of every head chunk on
+        # device-resident token-order inputs (the kernels the host path runs),
+        # and plain pinned-memory copies of the step's inputs and outputs.
+        parts = None
+        if w.B == 1:
+            fo, fl_ = torch.empty_like(path.o), torch.empty_like(path.lse)
+
+            def chunks():
+                for h0 in range(0, w.H, g):
+                    h1 = min(w.H, h0 + g)
+                    ops.attn_fwd(path.q[:, h0:h1], path.k[:, h0:h1], path.v[:, h0:h1], w.P,
+                                 path.layout, w.causal, sched_free=args.sched == "free",
+                                 out=fo[:, h0:h1], lse=fl_[:, h0:h1], token_order=True)
+
+            chunks()
+            chunk_ms = timed(chunks, n_e2e, world)
+            dq_ = torch.empty_like(path.q)
+
+            def h2d_copy():
+                for t in (hq, hk, hv):
+                    dq_.copy_(t, non_blocking=True)
+
+            def d2h_copy():
+                ho.copy_(fo, non_blocking=True)
+                hl.copy_(fl_, non_blocking=True)
+
+            h2d_copy()
+            h2d_ms = timed(h2d_copy, 3, world)
+            d2h_ms = timed(d2h_copy, 3, world)
+            del fo, fl_, dq_
+            torch.cuda.empty_cache()
+            parts = {"chunk_kernels_ms": chunk_ms, "exposed_copy_ms": e2e_ms - chunk_ms,
+                     "h2d_alone_ms": h2d_ms, "h2d_gbs": h2d / (h2d_ms * 1e-3) / 1e9,
+                     "d2h_alone_ms": d2h_ms, "d2h_gbs": d2h / (d2h_ms * 1e-3) / 1e9,
+                     "note": "chunk_kernels_ms: the same head chunks attended on device-resident "
+                             "token-order tensors, back to back; exposed_copy_ms = e2e - that; "
+                             "copies timed alone from/to pinned host memory"}
         e2e = {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "api": "ra_attn_fwd_host (pinned host buffers)", "heads_per_chunk": g}
+               "api": "ra_attn_fwd_host (pinned host buffers)", "heads_per_chunk": g,
+               "parts": parts}
 
     # ---- the same step with the layout's permutation applied inside the
     # attention kernel (RA_TOKEN_ORDER: one launch, token order in and out)
@@ -471,13 +610,13 @@ def main():
         if ops.device_fault():
             raise RuntimeError("device fault during the layout comparison")
 
-    # ---- backward pass (optional): 10 d FLOP per visible pair (5 GEMMs)
+    # ---- backward pass: 10 d useful FLOP per visible pair (5 products)
     backward = None
-    if args.backward:
+    if not args.no_backward:
         lay = path.layout
-        qq, kk, vv = (path.qp, path.kp, path.vp) if lay == W.STRIPED else (path.q, path.k, path.v)
-        oo = path.op if lay == W.STRIPED else path.o
-        ll = path.lsep if lay == W.STRIPED else path.lse
+        qq, kk, vv = (path.qp, path.kp, path.vp) if lay != W.CONTIGUOUS else (path.q, path.k, path.v)
+        oo = path.op if lay != W.CONTIGUOUS else path.o
+        ll = path.lsep if lay != W.CONTIGUOUS else path.lse
         path.step()
         dout = torch.randn(qq.shape, device=qq.device,
                            generator=torch.Generator(device=qq.device).manual_seed(1)).to(qq.dtype)
@@ -490,19 +629,35 @@ def main():
 
         bwd_step()
         torch.cuda.synchronize()
-        bms = timed(bwd_step, max(1, min(args.steps, 3)), world, flush=flush)
+        n_b = max(1, min(args.steps, 3))
+        bms = timed(bwd_step, n_b, world, flush=flush)
         if ops.device_fault():
             raise RuntimeError("device fault during the backward pass")
+        del dout, ws, grads
+        torch.cuda.empty_cache()
         # useful: 10 d FLOP per visible pair (the five products of the
         # gradient); executed: 14 d (the dQ kernel recomputes S and dP)
-        useful = 2.5 * flops / (bms * 1e-3) / 1e12
-        executed = 3.5 * flops / (bms * 1e-3) / 1e12
-        backward = {"ms": bms, "useful_tflops": useful, "executed_tflops": executed,
+        useful = 2.5 * flops * world / (bms * 1e-3) / 1e12
+        executed = 3.5 * flops * world / (bms * 1e-3) / 1e12
+        backward = {"ms": bms, "steps": n_b, "useful_tflops": useful,
+                    "executed_tflops": executed,
                     "frac_executed_of_sustained_peak":
-                        executed / float(peaks.get("bf16_tflops_sustained",
-                                                   FALLBACK_PEAKS["bf16_tflops_sustained"])),
+                        executed / world / float(peaks.get("bf16_tflops_sustained",
+                                                           FALLBACK_PEAKS["bf16_tflops_sustained"])),
+                    "kernels": "bwd_rowdot_kernel, bwd_dkdv_kernel, bwd_dq_kernel",
                     "flop_convention": "useful 10 d per visible pair (QK^T, dO V^T, dV, dK, dQ); "
                                        "executed 14 d (S and dP recomputed for dQ)"}
+
+    # ---- the other configurations of the evaluation (same step, own inputs)
+    configs = None
+    if not args.no_configs:
+        configs = {}
+        for w2 in (W.RING_8K, W.STRIPED_8K, W.LONG_128K):
+            if w2.name == w.name:
+                continue
+            configs[w2.name] = workload_leg(ops, w2, args.sched, world,
+                                            steps=20 if w2.N <= 8192 else 5)
+            torch.cuda.empty_cache()
 
     # ---- the physical ring, emulated on this GPU: every (rank j, round r)
     # block of ra_attn_fwd_block timed alone; on P devices round r lasts as
@@ -510,18 +665,15 @@ def main():
     # compute time (the K/V exchange, 2 B H c d 2 bytes per rank per round,
     # overlaps it)
     ring = None
-    if args.ring_emulate and rank == 0 and world == 1:
+    if not args.no_ring_emulate and rank == 0 and world == 1:
         ring = {}
         c = w.N // w.P
         for lay in (W.STRIPED, W.CONTIGUOUS):
-            pth = Path(ops, w, q, k, v, layout=lay)
-            src = (pth.q, pth.k, pth.v)
+            src = (path.q, path.k, path.v)
             if lay != W.CONTIGUOUS:
-                for a, b in ((pth.q, pth.qp), (pth.k, pth.kp), (pth.v, pth.vp)):
-                    ops.partition(a, w.P, lay, out=b)
-                src = (pth.qp, pth.kp, pth.vp)
+                src = tuple(ops.partition(t, w.P, lay) for t in src)
             shards = [[t[:, :, j * c:(j + 1) * c].contiguous() for j in range(w.P)] for t in src]
-            del pth
+            del src
             o_blk = torch.empty_like(shards[0][0])
             l_blk = torch.empty(w.B, w.H, c, dtype=torch.float32, device="cuda")
             acc = torch.empty(o_blk.shape, dtype=torch.float32, device="cuda")
@@ -547,14 +699,16 @@ def main():
             per_rank = [sum(t[j]) for j in range(w.P)]
             xfer = 2 * w.B * w.H * c * w.d * 2
             ring[W.LAYOUT_NAMES[lay]] = {
-                "predicted_ring_ms": total,
-                "useful_tflops_on_P_gpus": flops / (total * 1e-3) / 1e12,
+                "predicted_ring_ms": round(total, 3),
+                "useful_tflops_on_P_gpus": round(flops / (total * 1e-3) / 1e12, 1),
                 "round_max_ms": [round(x, 3) for x in round_max],
                 "rank_busy_ms_min_max": [round(min(per_rank), 3), round(max(per_rank), 3)],
                 "kv_bytes_per_rank_per_round": xfer,
-                "kv_ms_per_round_at_770GBs": xfer / 770e9 * 1e3}
+                "kv_ms_per_round_at_770GBs": round(xfer / 770e9 * 1e3, 4)}
         if ops.device_fault():
             raise RuntimeError("device fault during the ring emulation")
+        ring["contiguous_over_striped"] = round(
+            ring["contiguous"]["predicted_ring_ms"] / ring["striped"]["predicted_ring_ms"], 3)
         ring["note"] = ("per-round block + merge kernels of every rank run one at a time on "
                         "this GPU; P GPUs would run each round's ranks concurrently")
 
@@ -578,23 +732,25 @@ def main():
         if ops.device_fault():
             raise RuntimeError("device fault during the RoPE partition")
 
-    # ---- CPU oracle baseline (rank 0, one GPU only)
-    cpu = None
+    # ---- CPU oracle baseline (rank 0, one GPU only), and the timed step's
+    # output compared with the oracle rows it computes
+    cpu = parity = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, desc, threads = cpu_oracle_rate(w, 15.0)
+        rate, desc, threads, ref = cpu_oracle_leg(w, 15.0)
         cpu = {"value": rate, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                "sample": desc}
+        parity = parity_of(o_step, lse_step, v[0, ref[0], 0].double().numpy(), ref)
 
     peak_key = "bf16_tflops_sustained"
     peak = float(peaks.get(peak_key, FALLBACK_PEAKS[peak_key]))
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     achieved = flops / (attn_ms * 1e-3) / 1e12
     traffic = recorded_traffic(w.name)
     kname = f"attn_fwd_kernel<{w.d}, {'true' if w.layout == W.ZIGZAG else 'false'}>"
     roofline = {"bound": "tensor", "kernel": kname, "achieved": achieved,
                 "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
-                "peak_source": f"{peaks_src} {peak_key}",
-                "frac_of_burst_peak": achieved / float(peaks.get("bf16_tflops",
-                                                                 FALLBACK_PEAKS["bf16_tflops"])),
+                "peak_source": f"{peaks_src} {peak_key} (kernel timed inside a seconds-long loop)",
+                "frac_of_burst_peak": achieved / burst,
                 "frac_of_spec_2250": achieved / SPEC_BF16_TFLOPS,
                 "attn_ms_per_launch": attn_ms,
                 "attn_ms_median": statistics.median(attn_ts), "attn_ms_min": min(attn_ts),
@@ -605,21 +761,19 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16; q,k x3 for the stress workload)",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "P": w.P,
-                   "layout": w.layout_name, "causal": w.causal, "schedule": args.sched,
-                   "step": "partition q,k,v -> attention -> unpartition o,lse",
-                   "l2": l2_note,
-                   "parallelism": f"replicas x{world}"},
+        "config": config,
         "tokens_per_s": tokens_s,
         "frac_of_peak": value / world / peak,
         "gpu_launches": path.launches_per_step * args.steps,
         "clocks": clocks,
         "roofline": roofline,
+        "parity": parity,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "layout_compare": compare,
         "token_order_step": fused,
         "backward": backward,
+        "configs": configs,
         "rope_partition": rope,
         "ring_emulation": ring,
     }

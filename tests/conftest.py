@@ -12,6 +12,16 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
 
 
+def pytest_terminal_summary(terminalreporter):
+    from tests import _margins
+
+    lines = _margins.summary_lines()
+    if lines:
+        terminalreporter.section("parity margins against the fp64 oracle")
+        for line in lines:
+            terminalreporter.write_line(line)
+
+
 @pytest.fixture(scope="session")
 def golden_dir():
     return os.path.join(ROOT, "tests", "golden")

@@ -16,6 +16,7 @@ from oracle import attention as OA
 from oracle import merge as OM
 from oracle import partition as OP
 from oracle import work as OW
+from tests import _margins
 
 pytestmark = pytest.mark.gpu
 
@@ -61,9 +62,10 @@ def oracle_full(q, k, v, causal, scale):
 def assert_close(o, lse, o_ref, lse_ref, what=""):
     err = np.abs(o - o_ref)
     assert np.isfinite(o).all() and np.isfinite(lse).all(), what
+    lerr = np.abs(lse - lse_ref)
+    _margins.record(what, err.max(), err.mean(), lerr.max())
     assert err.max() <= O_MAX, f"{what}: O max-abs {err.max():.3e}"
     assert err.mean() <= O_MEAN, f"{what}: O mean-abs {err.mean():.3e}"
-    lerr = np.abs(lse - lse_ref)
     assert lerr.max() <= LSE_MAX, f"{what}: lse max-abs {lerr.max():.3e}"
 
 
