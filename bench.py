@@ -674,7 +674,7 @@ def main():
                 src = tuple(ops.partition(t, w.P, lay) for t in src)
             shards = [[t[:, :, j * c:(j + 1) * c].contiguous() for j in range(w.P)] for t in src]
             del src
-            o_blk = torch.empty_like(shards[0][0])
+            o_blk = torch.empty(shards[0][0].shape, dtype=torch.float32, device="cuda")
             l_blk = torch.empty(w.B, w.H, c, dtype=torch.float32, device="cuda")
             acc = torch.empty(o_blk.shape, dtype=torch.float32, device="cuda")
             lacc = torch.empty_like(l_blk)
@@ -687,7 +687,7 @@ def main():
                         e1 = torch.cuda.Event(enable_timing=True)
                         e0.record()
                         ops.attn_fwd_block(shards[0][j], shards[1][kb], shards[2][kb], j, kb, w.P,
-                                           lay, w.causal, out=o_blk, lse=l_blk)
+                                           lay, w.causal, out=o_blk, lse=l_blk, o_f32=True)
                         ops.lse_merge_acc(acc, lacc, o_blk, l_blk, first=(r == 0))
                         e1.record()
                         e1.synchronize()
@@ -709,8 +709,9 @@ def main():
             raise RuntimeError("device fault during the ring emulation")
         ring["contiguous_over_striped"] = round(
             ring["contiguous"]["predicted_ring_ms"] / ring["striped"]["predicted_ring_ms"], 3)
-        ring["note"] = ("per-round block + merge kernels of every rank run one at a time on "
-                        "this GPU; P GPUs would run each round's ranks concurrently")
+        ring["note"] = ("per-round block (float32 partial) + merge kernels of every rank run "
+                        "one at a time on this GPU; P GPUs would run each round's ranks "
+                        "concurrently")
 
     # ---- stripe + RoPE of q and k (memory-bound side path, not in the step)
     rope = None

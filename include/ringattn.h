@@ -321,10 +321,17 @@ int64_t ra_attn_fwd_host_workspace(int64_t N, int64_t d, int layout, int64_t hea
  *
  *   q         device bf16 [B, H, c, d]: query shard j in layout order.
  *   k, v      device bf16 [B, H, c, d]: key/value block kb in layout order.
- *   o, lse    outputs: bf16 [B, H, c, d] and float32 [B, H, c].  A query row
- *             that sees no key of the block gets o = 0, lse = -inf.
+ *   o, lse    outputs: bf16 [B, H, c, d] (float32 with RA_O_F32 OR-ed into
+ *             layout) and float32 [B, H, c].  A query row that sees no key
+ *             of the block gets o = 0, lse = -inf.
  *   j, kb, P  0 <= j, kb < P: the pair's shard indices (masks only).
  *   d         64 or 128; c = N / P >= 1.
+ *   layout    RA_CONTIGUOUS or RA_STRIPED, optionally | RA_O_F32.  A ring
+ *             that keeps its per-round partials in float32 (RA_O_F32 here,
+ *             RA_MERGE_F32_PARTIAL in ra_lse_merge_acc) rounds O to bf16
+ *             once, at the end; bf16 partials add one more rounding per
+ *             row, which a peaked softmax (one dominant key) does not
+ *             average away.
  * Same tile skipping and precision as ra_attn_fwd.  Errors as ra_attn_fwd.
  */
 ra_status ra_attn_fwd_block(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -334,14 +341,16 @@ ra_status ra_attn_fwd_block(const void* q, const void* k, const void* v, void* o
 /* Modes of ra_lse_merge_acc (OR-ed). */
 #define RA_MERGE_FIRST 1     /* accumulator not yet set: it becomes the partial */
 #define RA_MERGE_FINAL 2     /* also write the merged O as bf16 to o_final      */
+#define RA_MERGE_F32_PARTIAL 4 /* the partial o_b is float32, not bf16          */
 
 /*
- * ra_lse_merge_acc -- fold a bf16 partial result into a float32 accumulator
- * (the same merge as ra_lse_merge; 1cademy page "Computing Attention Weights
- * in Sequence Parallelism"), so that P rounds round to bf16 once.
+ * ra_lse_merge_acc -- fold a partial result into a float32 accumulator (the
+ * same merge as ra_lse_merge; 1cademy page "Computing Attention Weights in
+ * Sequence Parallelism"), so that P rounds round to bf16 once.
  *
  *   o_acc, lse_acc   device float32 [rows, d] and [rows], read and written.
- *   o_b, lse_b       device bf16 [rows, d] and float32 [rows]: the partial.
+ *   o_b, lse_b       device bf16 [rows, d] (float32 with
+ *                    RA_MERGE_F32_PARTIAL) and float32 [rows]: the partial.
  *   o_final          device bf16 [rows, d], written when mode has
  *                    RA_MERGE_FINAL (may be NULL otherwise).
  *   rows, d          0 <= rows < 2^31; d a multiple of 8, 8 <= d <= 2^20

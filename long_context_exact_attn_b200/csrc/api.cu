@@ -367,6 +367,8 @@ ra_status ra_attn_fwd_block(const void* q, const void* k, const void* v, void* o
                             int64_t B, int64_t H, int64_t c, int64_t d, int j, int kb, int P,
                             int layout, int causal, float scale, void* stream) {
   if (!q || !k || !v || !o || !lse) return RA_ERR_NULL;
+  const bool o_f32 = (layout & RA_O_F32) != 0;
+  layout &= ~RA_O_F32;
   if (layout != RA_CONTIGUOUS && layout != RA_STRIPED) return RA_ERR_LAYOUT;
   if (d != 64 && d != 128) return RA_ERR_HEADDIM;
   if (B < 1 || H < 1 || c < 1 || P < 1 || j < 0 || j >= P || kb < 0 || kb >= P)
@@ -377,10 +379,10 @@ ra_status ra_attn_fwd_block(const void* q, const void* k, const void* v, void* o
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
       !aligned(lse, 16))
     return RA_ERR_ALIGN;
-  const int64_t tb = B * H * c * d * 2, lb = B * H * c * 4;
-  if (overlap(o, tb, q, tb) || overlap(o, tb, k, tb) || overlap(o, tb, v, tb) ||
+  const int64_t tb = B * H * c * d * 2, ob = o_f32 ? 2 * tb : tb, lb = B * H * c * 4;
+  if (overlap(o, ob, q, tb) || overlap(o, ob, k, tb) || overlap(o, ob, v, tb) ||
       overlap(lse, lb, q, tb) || overlap(lse, lb, k, tb) || overlap(lse, lb, v, tb) ||
-      overlap(o, tb, lse, lb))
+      overlap(o, ob, lse, lb))
     return RA_ERR_ALIAS;
   int dev;
   DevInfo info;
@@ -389,12 +391,13 @@ ra_status ra_attn_fwd_block(const void* q, const void* k, const void* v, void* o
   // A block that GetMask hides completely (contiguous causal, kb > j): no
   // query row sees a key of it.
   if (causal && layout == RA_CONTIGUOUS && kb > j) {
-    if (cudaMemsetAsync(o, 0, (size_t)tb, (cudaStream_t)stream) != cudaSuccess) return RA_ERR_CUDA;
+    if (cudaMemsetAsync(o, 0, (size_t)ob, (cudaStream_t)stream) != cudaSuccess) return RA_ERR_CUDA;
     return fill_f32_launch(lse, B * H * c, -INFINITY, stream);
   }
   AttnLaunch a;
   a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
   a.BH = B * H; a.N = c; a.d = d; a.P = 1;
+  a.o_f32 = o_f32;
   a.striped = layout == RA_STRIPED;
   a.causal = causal != 0;
   a.sched_free = 1;
@@ -410,27 +413,29 @@ ra_status ra_attn_fwd_block(const void* q, const void* k, const void* v, void* o
 ra_status ra_lse_merge_acc(float* o_acc, float* lse_acc, const void* o_b, const float* lse_b,
                            void* o_final, int64_t rows, int64_t d, int mode, void* stream) {
   if (!o_acc || !lse_acc || !o_b || !lse_b) return RA_ERR_NULL;
-  if ((mode & ~3) != 0) return RA_ERR_LAYOUT;
+  if ((mode & ~7) != 0) return RA_ERR_LAYOUT;
   const int first = mode & RA_MERGE_FIRST, final_ = (mode & RA_MERGE_FINAL) != 0;
+  const int b_f32 = (mode & RA_MERGE_F32_PARTIAL) != 0;
   if (final_ && !o_final) return RA_ERR_NULL;
   if (rows < 0 || d < 8 || d % 8 != 0 || d > (1 << 20) || rows >= ((int64_t)1 << 31))
     return RA_ERR_SHAPE;
   if (!aligned(o_acc, 16) || !aligned(o_b, 16) || !aligned(lse_acc, 4) || !aligned(lse_b, 4) ||
       (final_ && !aligned(o_final, 16)))
     return RA_ERR_ALIGN;
-  const int64_t ab = rows * d * 4, bb = rows * d * 2, lb = rows * 4;
+  const int64_t ab = rows * d * 4, fb = rows * d * 2, bb = b_f32 ? ab : fb, lb = rows * 4;
   if (overlap(o_acc, ab, o_b, bb) || overlap(o_acc, ab, lse_acc, lb) ||
       overlap(o_acc, ab, lse_b, lb) || overlap(lse_acc, lb, o_b, bb) ||
       overlap(lse_acc, lb, lse_b, lb))
     return RA_ERR_ALIAS;
-  if (final_ && (overlap(o_final, bb, o_acc, ab) || overlap(o_final, bb, o_b, bb) ||
-                 overlap(o_final, bb, lse_acc, lb) || overlap(o_final, bb, lse_b, lb)))
+  if (final_ && (overlap(o_final, fb, o_acc, ab) || overlap(o_final, fb, o_b, bb) ||
+                 overlap(o_final, fb, lse_acc, lb) || overlap(o_final, fb, lse_b, lb)))
     return RA_ERR_ALIAS;
   int dev;
   DevInfo info;
   ra_status st = current_device(&dev, &info);
   if (st) return st;
-  return lse_merge_acc_launch(o_acc, lse_acc, o_b, lse_b, o_final, rows, d, first, final_, stream);
+  return lse_merge_acc_launch(o_acc, lse_acc, o_b, lse_b, o_final, rows, d, first, final_, b_f32,
+                              stream);
 }
 
 int64_t ra_attn_fwd_host_workspace(int64_t N, int64_t d, int layout, int64_t heads_per_chunk) {

@@ -245,8 +245,9 @@ ra_status lse_merge_launch(const void* o_a, const float* lse_a, const void* o_b,
 // rounds round to bf16 only once.  first: the accumulator is not yet set
 // (it becomes the partial).  final: also write O_acc as bf16 to o_final.
 // Both sides empty (lse = -inf) give O = 0, lse = -inf.
+template <bool F32B>
 __global__ void lse_merge_acc_kernel(float* __restrict__ oacc, float* __restrict__ lacc,
-                                     const uint4* __restrict__ ob, const float* __restrict__ lb_,
+                                     const void* __restrict__ ob_, const float* __restrict__ lb_,
                                      uint4* __restrict__ ofin, long long rows, int chunks,
                                      int first, int final_) {
   const int lane = threadIdx.x & 31;
@@ -268,16 +269,28 @@ __global__ void lse_merge_acc_kernel(float* __restrict__ oacc, float* __restrict
     __syncwarp();
     for (int ch = lane; ch < chunks; ch += 32) {
       const size_t idx = (size_t)r * chunks + ch;
-      const uint4 b = ob[idx];
-      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+      float2 b0, b1, b2v, b3;   // the partial's 8 values of this chunk
+      if (F32B) {
+        const float4* f = reinterpret_cast<const float4*>(ob_) + idx * 2;
+        const float4 u = f[0], w = f[1];
+        b0 = make_float2(u.x, u.y);
+        b1 = make_float2(u.z, u.w);
+        b2v = make_float2(w.x, w.y);
+        b3 = make_float2(w.z, w.w);
+      } else {
+        const uint4 b = reinterpret_cast<const uint4*>(ob_)[idx];
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+        b0 = __bfloat1622float2(b2[0]);
+        b1 = __bfloat1622float2(b2[1]);
+        b2v = __bfloat1622float2(b2[2]);
+        b3 = __bfloat1622float2(b2[3]);
+      }
       float4* a4 = reinterpret_cast<float4*>(oacc) + idx * 2;
       float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
       if (!first) {
         a0 = a4[0];
         a1 = a4[1];
       }
-      const float2 b0 = __bfloat1622float2(b2[0]), b1 = __bfloat1622float2(b2[1]);
-      const float2 b2v = __bfloat1622float2(b2[2]), b3 = __bfloat1622float2(b2[3]);
       a0 = make_float4(wa * a0.x + wb * b0.x, wa * a0.y + wb * b0.y, wa * a0.z + wb * b1.x,
                        wa * a0.w + wb * b1.y);
       a1 = make_float4(wa * a1.x + wb * b2v.x, wa * a1.y + wb * b2v.y, wa * a1.z + wb * b3.x,
@@ -301,14 +314,19 @@ __global__ void lse_merge_acc_kernel(float* __restrict__ oacc, float* __restrict
 
 ra_status lse_merge_acc_launch(float* o_acc, float* lse_acc, const void* o_b,
                                const float* lse_b, void* o_final, int64_t rows, int64_t d,
-                               int first, int final_, void* stream) {
+                               int first, int final_, int b_f32, void* stream) {
   if (rows == 0) return RA_OK;
   const int chunks = (int)(d / 8);
   long long blocks = (rows + 7) / 8;
   if (blocks > 148LL * 16) blocks = 148LL * 16;
-  lse_merge_acc_kernel<<<(int)blocks, 256, 0, (cudaStream_t)stream>>>(
-      o_acc, lse_acc, reinterpret_cast<const uint4*>(o_b), lse_b, reinterpret_cast<uint4*>(o_final),
-      (long long)rows, chunks, first, final_);
+  if (b_f32)
+    lse_merge_acc_kernel<true><<<(int)blocks, 256, 0, (cudaStream_t)stream>>>(
+        o_acc, lse_acc, o_b, lse_b, reinterpret_cast<uint4*>(o_final), (long long)rows, chunks,
+        first, final_);
+  else
+    lse_merge_acc_kernel<false><<<(int)blocks, 256, 0, (cudaStream_t)stream>>>(
+        o_acc, lse_acc, o_b, lse_b, reinterpret_cast<uint4*>(o_final), (long long)rows, chunks,
+        first, final_);
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 

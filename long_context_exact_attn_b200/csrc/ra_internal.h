@@ -51,7 +51,7 @@ ra_status partition_rope_launch(const void* src, void* dst, int64_t BH, int64_t 
                                 void* stream);
 ra_status lse_merge_acc_launch(float* o_acc, float* lse_acc, const void* o_b,
                                const float* lse_b, void* o_final, int64_t rows, int64_t d,
-                               int first, int final_, void* stream);
+                               int first, int final_, int b_f32, void* stream);
 ra_status fill_f32_launch(float* dst, int64_t n, float value, void* stream);
 ra_status lse_merge_launch(const void* o_a, const float* lse_a, const void* o_b,
                            const float* lse_b, void* o_out, float* lse_out, int64_t rows,

@@ -256,10 +256,12 @@ def attn_fwd_host(q, k, v, P, layout, causal=True, scale=None, workspace=None, o
     return o, lse
 
 
-def attn_fwd_block(q, k, v, j, kb, P, layout, causal=True, scale=None, out=None, lse=None):
+def attn_fwd_block(q, k, v, j, kb, P, layout, causal=True, scale=None, out=None, lse=None,
+                   o_f32=False):
     """One round of the ring on this device: query shard j [B, H, c, d]
     against key/value block kb [B, H, c, d] (layout order), normalised over
-    the block; rows that see no key of it get o = 0, lse = -inf."""
+    the block; rows that see no key of it get o = 0, lse = -inf.  With
+    ``o_f32`` the partial O is float32 (rounded once, later, by the merge)."""
     for n, t in (("q", q), ("k", k), ("v", v)):
         _cuda_contig(t, n)
         if t.dtype != torch.bfloat16 or t.dim() != 4 or t.shape != q.shape:
@@ -268,33 +270,38 @@ def attn_fwd_block(q, k, v, j, kb, P, layout, causal=True, scale=None, out=None,
     B, H, c, d = q.shape
     if scale is None:
         scale = d ** -0.5
-    o = torch.empty_like(q) if out is None else _like(out, "out", q.shape, q.dtype, q.device)
+    odt = torch.float32 if o_f32 else q.dtype
+    o = (torch.empty(q.shape, dtype=odt, device=q.device) if out is None
+         else _like(out, "out", q.shape, odt, q.device))
     lse = (torch.empty(B, H, c, dtype=torch.float32, device=q.device) if lse is None
            else _like(lse, "lse", (B, H, c), torch.float32, q.device))
+    lay = int(layout) | (O_F32 if o_f32 else 0)
     _launch("ra_attn_fwd_block", q, lib().ra_attn_fwd_block, _ptr(q), _ptr(k), _ptr(v), _ptr(o),
-            _ptr(lse), B, H, c, d, int(j), int(kb), int(P), int(layout), int(bool(causal)),
+            _ptr(lse), B, H, c, d, int(j), int(kb), int(P), lay, int(bool(causal)),
             float(scale), _stream(q))
     return o, lse
 
 
-MERGE_FIRST, MERGE_FINAL = 1, 2
+MERGE_FIRST, MERGE_FINAL, MERGE_F32_PARTIAL = 1, 2, 4
 
 
 def lse_merge_acc(o_acc, lse_acc, o_b, lse_b, first=False, final_out=None):
-    """Fold a bf16 partial (o_b, lse_b) into the float32 accumulator
-    (o_acc, lse_acc) in place; with ``final_out`` also write the merged O as
-    bf16 there."""
+    """Fold a partial (o_b bf16 or float32, lse_b) into the float32
+    accumulator (o_acc, lse_acc) in place; with ``final_out`` also write the
+    merged O as bf16 there."""
     d = o_b.shape[-1]
     rows = o_b.numel() // d
-    if o_acc.dtype != torch.float32 or o_acc.shape != o_b.shape or o_b.dtype != torch.bfloat16:
-        raise ValueError("o_acc float32 and o_b bfloat16 of the same shape")
+    if o_acc.dtype != torch.float32 or o_acc.shape != o_b.shape or \
+            o_b.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("o_acc float32 and o_b bfloat16 or float32 of the same shape")
     if lse_acc.dtype != torch.float32 or lse_b.dtype != torch.float32 or \
             lse_acc.numel() != rows or lse_b.numel() != rows:
         raise ValueError("lse_acc, lse_b: float32 with one value per row")
     for n, t in (("o_acc", o_acc), ("lse_acc", lse_acc), ("o_b", o_b), ("lse_b", lse_b)):
         _cuda_contig(t, n)
     _same_device(("o_b", o_b), ("o_acc", o_acc), ("lse_acc", lse_acc), ("lse_b", lse_b))
-    mode = (MERGE_FIRST if first else 0) | (MERGE_FINAL if final_out is not None else 0)
+    mode = ((MERGE_FIRST if first else 0) | (MERGE_FINAL if final_out is not None else 0)
+            | (MERGE_F32_PARTIAL if o_b.dtype == torch.float32 else 0))
     fin = None
     if final_out is not None:
         fin = _ptr(_like(final_out, "final_out", o_b.shape, torch.bfloat16, o_b.device))

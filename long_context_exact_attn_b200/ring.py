@@ -10,7 +10,8 @@ layout (Striped review) rank j holds the tokens j, j+P, j+2P, ... and every
 round's GetMask keeps the work balanced.
 
 On each rank: ``ra_attn_fwd_block`` computes the round's partial result on
-the device, ``ra_lse_merge_acc`` folds it into a float32 accumulator, and
+the device (in float32, so that O is rounded to bf16 only once, at the end),
+``ra_lse_merge_acc`` folds it into a float32 accumulator, and
 the K/V exchange for the next round is posted before the round's compute so
 that the transfer overlaps it (``torch.distributed`` point-to-point
 operations; NCCL over NVLink on GPUs).  Each rank sends one K and one V block
@@ -18,7 +19,10 @@ per round: 2 * B * H * c * d * 2 bytes.
 
 The block and merge steps are parameters so that the exchange logic can be
 exercised on host tensors (gloo) with any implementation of those two steps;
-by default they are this library's kernels.
+by default they are this library's kernels.  A gloo group moves host tensors
+only: with device tensors on such a group the blocks are staged through host
+buffers (copied out before they are sent, copied in on the current stream
+after they arrive), which keeps the device work in stream order.
 """
 
 import torch
@@ -27,11 +31,16 @@ import torch.distributed as dist
 
 def _kernels():
     from . import ops
-    return ops.attn_fwd_block, ops.lse_merge_acc
+
+    def block(q, k, v, j, kb, P, layout, causal, scale):
+        # float32 partials: O is rounded to bf16 once, by the last merge
+        return ops.attn_fwd_block(q, k, v, j, kb, P, layout, causal, scale, o_f32=True)
+
+    return block, ops.lse_merge_acc
 
 
 def ring_attn_fwd(q, k, v, layout, causal=True, scale=None, group=None, block_fn=None,
-                  merge_fn=None):
+                  merge_fn=None, host_staging=None):
     """This rank's share of the ring: q, k, v are the rank's shard
     [B, H, c, d] in layout order (rank j holds shard j of P = world size).
     Returns (o [B, H, c, d] in q's dtype, lse [B, H, c], float32 or wider) of the
@@ -39,7 +48,9 @@ def ring_attn_fwd(q, k, v, layout, causal=True, scale=None, group=None, block_fn
 
     block_fn(q, k, v, j, kb, P, layout, causal, scale) -> (o_r, lse_r) and
     merge_fn(o_acc, lse_acc, o_r, lse_r, first=..., final_out=...) default to
-    the library's ``attn_fwd_block`` and ``lse_merge_acc``.
+    the library's ``attn_fwd_block`` and ``lse_merge_acc``.  host_staging
+    (default: device tensors on a gloo group) sends and receives the K/V
+    blocks through host copies.
     """
     if block_fn is None or merge_fn is None:
         kb_fn, mg_fn = _kernels()
@@ -58,20 +69,33 @@ def ring_attn_fwd(q, k, v, layout, causal=True, scale=None, group=None, block_fn
     o_acc = torch.empty(q.shape, dtype=acc, device=q.device)
     lse_acc = torch.empty((B, H, c), dtype=acc, device=q.device)
     o = torch.empty_like(q)
+    if host_staging is None:
+        host_staging = q.is_cuda and dist.get_backend(group) == "gloo"
     # Two spare K/V pairs: the block being sent is never the one being
     # received into, and the caller's k, v are never written.
     spare = [(torch.empty_like(k), torch.empty_like(v)) for _ in range(2)]
+    if host_staging:
+        # host images of the block being sent and of the one being received
+        h_send = [torch.empty(k.shape, dtype=k.dtype) for _ in range(2)]
+        h_recv = [torch.empty(k.shape, dtype=k.dtype) for _ in range(2)]
     cur_k, cur_v = k, v
     for r in range(P):
         kb = (rank - r) % P
         reqs = []
         if r < P - 1:
             rk, rv = spare[r % 2]
+            if host_staging:
+                # the host copies complete before the sends are posted
+                h_send[0].copy_(cur_k)
+                h_send[1].copy_(cur_v)
+                send_k, send_v, recv_k, recv_v = h_send[0], h_send[1], h_recv[0], h_recv[1]
+            else:
+                send_k, send_v, recv_k, recv_v = cur_k, cur_v, rk, rv
             reqs = dist.batch_isend_irecv([
-                dist.P2POp(dist.isend, cur_k, nxt, group),
-                dist.P2POp(dist.isend, cur_v, nxt, group),
-                dist.P2POp(dist.irecv, rk, prv, group),
-                dist.P2POp(dist.irecv, rv, prv, group),
+                dist.P2POp(dist.isend, send_k, nxt, group),
+                dist.P2POp(dist.isend, send_v, nxt, group),
+                dist.P2POp(dist.irecv, recv_k, prv, group),
+                dist.P2POp(dist.irecv, recv_v, prv, group),
             ])
         o_r, lse_r = block_fn(q, cur_k, cur_v, rank, kb, P, layout, causal, scale)
         merge_fn(o_acc, lse_acc, o_r, lse_r, first=(r == 0),
@@ -79,5 +103,10 @@ def ring_attn_fwd(q, k, v, layout, causal=True, scale=None, group=None, block_fn
         for req in reqs:
             req.wait()
         if r < P - 1:
+            if host_staging:
+                # ordered on the current stream after this round's kernels;
+                # synchronous, so the host buffers are free for the next round
+                rk.copy_(h_recv[0])
+                rv.copy_(h_recv[1])
             cur_k, cur_v = spare[r % 2]
     return o, lse_acc

@@ -175,8 +175,10 @@ def blk(L, q=A, k=Bp, v=Cp, o=Op, lse=Lp, B=1, H=2, c=256, d=128, j=1, kb=0, P=4
 
 @pytest.mark.parametrize("kw,code", [
     (dict(v=0), 1), (dict(o=Op + 8), 2), (dict(j=4), 3), (dict(kb=-1), 3), (dict(c=0), 3),
-    (dict(d=96), 4), (dict(layout=0x101), 5), (dict(scale=0.0), 6), (dict(o=A), 8),
-    (dict(lse=Cp + 64), 8),
+    (dict(d=96), 4), (dict(layout=0x101), 5), (dict(layout=0x202), 5), (dict(scale=0.0), 6),
+    (dict(o=A), 8), (dict(lse=Cp + 64), 8),
+    # a float32 partial (RA_O_F32) is twice as long: just below q it overlaps q
+    (dict(layout=0x201, o=A - 2 * 256 * 128 * 2), 8),
 ])
 def test_attn_fwd_block_rejects_invalid_arguments(L, kw, code):
     assert blk(L, **kw) == code
@@ -187,8 +189,10 @@ def macc(L, oa=A, la=Bp, ob=Cp, lb=Op, of=Lp, rows=256, d=128, mode=2):
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(oa=0), 1), (dict(of=0), 1), (dict(mode=4), 5), (dict(d=12), 3), (dict(rows=-1), 3),
+    (dict(oa=0), 1), (dict(of=0), 1), (dict(mode=8), 5), (dict(d=12), 3), (dict(rows=-1), 3),
     (dict(oa=A + 4), 2), (dict(ob=A + 4096), 8), (dict(of=Cp), 8),
+    # a float32 partial (RA_MERGE_F32_PARTIAL) is twice as long as a bf16 one
+    (dict(mode=6, of=Cp + 256 * 128 * 2), 8),
 ])
 def test_lse_merge_acc_rejects_invalid_arguments(L, kw, code):
     assert macc(L, **kw) == code

@@ -57,7 +57,12 @@ def test_block_parity_all_pairs(case):
     for j in range(P):
         for kb in range(P):
             o, lse = ops.attn_fwd_block(sh(qp, j), sh(kp, kb), sh(vp, kb), j, kb, P, layout, causal)
+            o32, lse32 = ops.attn_fwd_block(sh(qp, j), sh(kp, kb), sh(vp, kb), j, kb, P, layout,
+                                            causal, o_f32=True)
             torch.cuda.synchronize()
+            # the float32 partial is the same O before its rounding
+            assert o32.dtype == torch.float32 and torch.equal(o32.to(torch.bfloat16), o)
+            assert torch.equal(lse32, lse)
             o, lse = o.float().cpu().numpy(), lse.cpu().numpy()
             for h in range(H):
                 ro, rl = OR.block_attention(sh(qp, j)[0, h].double().cpu().numpy(),
@@ -74,12 +79,15 @@ def test_block_parity_all_pairs(case):
     assert ops.device_fault() == 0
 
 
-@pytest.mark.parametrize("layout", [W.STRIPED, W.CONTIGUOUS])
-def test_emulated_ring_equals_fused_forward_and_definition(layout):
+@pytest.mark.parametrize("layout,P", [(W.STRIPED, 8), (W.CONTIGUOUS, 8), (W.CONTIGUOUS, 4),
+                                      (W.STRIPED, 4)])
+def test_emulated_ring_equals_fused_forward_and_definition(layout, P):
     """Each rank j folds block (j - r) mod P in round r (Ring explainer
-    ステップ2) through the float32 accumulator; the result equals the fused
-    single-launch forward and the plain definition."""
-    w = W.Workload("ring_emu", 1, 2, 4096, 128, 8, layout, True, 77, qk_scale_up=3.0)
+    ステップ2) through the float32 accumulator, with float32 partials (O is
+    rounded to bf16 once); the result equals the fused single-launch forward
+    and the plain definition."""
+    w = W.Workload("ring_emu", 1, 2, 4096 if P == 8 else 2048, 128, P, layout, True, 77 + P,
+                   qk_scale_up=3.0)
     qp, kp, vp = _layout_qkv(w)
     P, c = w.P, w.N // w.P
     o_fused, lse_fused = ops.attn_fwd(qp, kp, vp, P, layout, True)
@@ -94,7 +102,7 @@ def test_emulated_ring_equals_fused_forward_and_definition(layout):
             kb = (j - r) % P
             o_r, l_r = ops.attn_fwd_block(q, kp[:, :, kb * c:(kb + 1) * c].contiguous(),
                                           vp[:, :, kb * c:(kb + 1) * c].contiguous(), j, kb, P,
-                                          layout, True)
+                                          layout, True, o_f32=True)
             ops.lse_merge_acc(acc, lacc, o_r, l_r, first=(r == 0),
                               final_out=out if r == P - 1 else None)
         o_ring[:, :, j * c:(j + 1) * c] = out
