@@ -747,7 +747,13 @@ def main():
     burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     achieved = flops / (attn_ms * 1e-3) / 1e12
     traffic = recorded_traffic(w.name)
-    kname = f"attn_fwd_kernel<{w.d}, {'true' if w.layout == W.ZIGZAG else 'false'}>"
+    # the instance the library launches: work lists for small striped causal
+    # problems in the owner schedule (at most 1024 items)
+    npairs = -(-(-(-w.c // 128)) // 2)
+    lists = (args.sched == "owner" and w.causal and w.layout == W.STRIPED
+             and npairs * w.P * w.B * w.H <= 1024)
+    kname = (f"attn_fwd_kernel<{w.d}, {'true' if w.layout == W.ZIGZAG else 'false'}, "
+             f"{'WorkLists' if lists else 'NoLists'}>")
     roofline = {"bound": "tensor", "kernel": kname, "achieved": achieved,
                 "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                 "peak_source": f"{peaks_src} {peak_key} (kernel timed inside a seconds-long loop)",

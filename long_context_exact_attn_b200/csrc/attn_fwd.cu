@@ -39,6 +39,13 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
+#include <cstring>
+#include <map>
+#include <memory>
+#include <mutex>
+#include <vector>
+
 #include "exp2_poly.h"
 #include "ra_internal.h"
 #include "ra_ptx.cuh"
@@ -47,6 +54,15 @@
 namespace ra {
 
 __device__ unsigned int g_device_fault = 0;
+
+// Work lists for small problems (see WorkLists): capacity, and the largest
+// problem (items of all heads and shards) that uses them.  At N = 8192
+// (512 items) the whole K/V fits in L2 and the lists only rebalance work;
+// at N = 131072 (4096 items) they would break the head-major order that
+// keeps the running CTAs in one head's K/V (measured 13 % slower).
+constexpr int kMaxListItems = 1024;
+constexpr int kMaxListCtas = 160;
+constexpr int kListItemsUsed = 1024;
 
 struct AttnParams {
   __nv_bfloat16* o;
@@ -75,6 +91,16 @@ struct AttnParams {
   // GetMask of the real pair (blk_j, blk_kb).
   int blk_j, blk_kb;
 };
+
+// Per-CTA work lists of the owner schedule (the kernel instance that takes
+// them): CTA b processes the items item[start[b] .. start[b+1]) of its
+// group, in that order.  The other instances take NoLists and deal a
+// group's items to its CTAs in snake order.
+struct WorkLists {
+  uint16_t start[kMaxListCtas + 1];
+  uint16_t item[kMaxListItems];
+};
+struct NoLists {};
 
 template <int D>
 struct Cfg {
@@ -124,13 +150,23 @@ __device__ __forceinline__ bool item_at(const AttnParams& p, int g, int u, Item&
 }
 
 // k-th item of this CTA: snake order over the group's members.
-__device__ __forceinline__ bool cta_item(const AttnParams& p, int k, Item& it) {
+__device__ __forceinline__ bool cta_item(const AttnParams& p, const NoLists&, int k, Item& it) {
   const int g = blockIdx.x / p.ctas_per_group;
   const int m = blockIdx.x % p.ctas_per_group;
   if (g >= p.groups) return false;
   const int G = p.ctas_per_group;
   const int u = k * G + ((k & 1) ? (G - 1 - m) : m);
   return item_at(p, g, u, it);
+}
+
+// k-th item of this CTA from its work list.
+__device__ __forceinline__ bool cta_item(const AttnParams& p, const WorkLists& wl, int k,
+                                         Item& it) {
+  const int g = blockIdx.x / p.ctas_per_group;
+  if (g >= p.groups) return false;
+  const int idx = wl.start[blockIdx.x] + k;
+  if (idx >= wl.start[blockIdx.x + 1]) return false;
+  return item_at(p, g, wl.item[idx], it);
 }
 
 // The key tiles met by a query-tile pair, in ring order.  Per block the two
@@ -358,10 +394,11 @@ __device__ __forceinline__ size_t out_row(const AttnParams& p, int bh, int j, in
   return (size_t)bh * p.N + t;
 }
 
-template <int D, bool ZZ>
+template <int D, bool ZZ, class Lists>
 __global__ void __launch_bounds__(320, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+                const __grid_constant__ CUtensorMap tmV, const AttnParams p,
+                const __grid_constant__ Lists wl) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -424,7 +461,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       uint32_t n_loads = 0;
       Item it;
       bool ok = true;
-      for (int k = 0; ok && cta_item(p, k, it); ++k) {
+      for (int k = 0; ok && cta_item(p, wl, k, it); ++k) {
         if (!mbar_wait(bar_q_empty, (k & 1) ^ 1, abort_flag, p.timeout_ns)) { ok = false; break; }
         mbar_arrive_expect_tx(bar_q_full, 2 * C::kTileBytes);
         const int x0 = it.pair * 2 * kBM;
@@ -487,7 +524,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       uint32_t of0 = 0, of1 = 0;
       Item it;
       bool ok = true;
-      for (int k = 0; ok && cta_item(p, k, it); ++k) {
+      for (int k = 0; ok && cta_item(p, wl, k, it); ++k) {
         if (!wmbar_wait(bar_q_full, k & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
         TileSeq<ZZ> seq;
         seq.init(p, it);
@@ -609,7 +646,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     uint32_t s_cnt = 0;
     Item it;
     bool ok = true;
-    for (int k = 0; ok && cta_item(p, k, it); ++k) {
+    for (int k = 0; ok && cta_item(p, wl, k, it); ++k) {
       TileSeq<ZZ> seq;
       seq.init(p, it);
       const int x = it.pair * 2 * kBM + t * kBM + row;   // local query row in shard
@@ -814,6 +851,91 @@ static bool encode_qkv_map(CUtensorMap* map, const void* base, int64_t BH, int64
   return r == CUDA_SUCCESS;
 }
 
+// Key-tile steps of a work item (the MMA warp's iterations): for each round
+// (each chunk pair in the zigzag layout) the larger of the two query tiles'
+// PARTIAL/FULL spans.  Mirrors TileSeq::next.
+static long long item_steps(const AttnParams& p, int j, int pair, bool zz) {
+  const int x0 = pair * 2 * kBM;
+  long long steps = 0;
+  if (zz) {
+    const int h = p.c >> 1;
+    for (int r = 0; r < 2 * p.P; ++r) {
+      const int kb = key_block(j, r >> 1, p.P);
+      const int hk = r & 1;
+      const int zx = x0 < h ? 0 : h;
+      const BlockMask bm = chunk_mask(zz_chunk(j, x0, h, p.P), hk ? 2 * p.P - 1 - kb : kb,
+                                      p.causal);
+      const TileSpan s0 = tile_span(bm, x0 - zx, h), s1 = tile_span(bm, x0 - zx + kBM, h);
+      steps += s0.part_end > s1.part_end ? s0.part_end : s1.part_end;
+    }
+  } else {
+    for (int r = 0; r < p.P; ++r) {
+      const BlockMask bm = block_mask(j, key_block(j, r, p.P), p.striped, p.causal);
+      const TileSpan s0 = tile_span(bm, x0, p.c), s1 = tile_span(bm, x0 + kBM, p.c);
+      steps += s0.part_end > s1.part_end ? s0.part_end : s1.part_end;
+    }
+  }
+  return steps;
+}
+
+// Per-CTA work lists of the owner schedule by longest-processing-time-first
+// list scheduling: every item of a group, heaviest first (head order kept
+// among equal weights), goes to the group's least-loaded CTA.  Used when the
+// items fit the parameter block; a snake deal of the head-major item order
+// leaves the CTAs of small problems unevenly loaded (at N = 8192 with 18
+// CTAs per group the busiest CTA gets 160 key-tile steps where 142 is the
+// mean; the lists bring it to 144).
+static bool build_lists(const AttnParams& p, bool zz, WorkLists& wl) {
+  const int G = p.ctas_per_group;
+  if (p.groups * G > kMaxListCtas) return false;
+  const int n_sh_max = (p.P + p.groups - 1) / p.groups;
+  const long long per_group_max = (long long)p.npairs * n_sh_max * p.BH;
+  if (per_group_max * p.groups > kMaxListItems) return false;
+  int pos = 0;
+  std::vector<long long> w;
+  std::vector<int> ord;
+  std::vector<std::vector<int>> lists(G);
+  for (int g = 0; g < p.groups; ++g) {
+    const int n_sh = (p.P - g + p.groups - 1) / p.groups;
+    const int n = p.npairs * n_sh * p.BH;
+    w.assign(n, 0);
+    for (int u = 0; u < n; ++u) {
+      // the same mapping as item_at (head-major)
+      const int per_head = p.npairs * n_sh;
+      const int rem = u % per_head;
+      int j, pair;
+      if (p.causal && !p.striped && !zz) {
+        const int sh_rank = rem / p.npairs;
+        j = g + (n_sh - 1 - sh_rank) * p.groups;
+        pair = p.npairs - 1 - (rem - sh_rank * p.npairs);
+      } else {
+        const int pr = rem / n_sh;
+        pair = p.npairs - 1 - pr;
+        j = g + (rem - pr * n_sh) * p.groups;
+      }
+      w[u] = item_steps(p, j, pair, zz);
+    }
+    ord.resize(n);
+    for (int u = 0; u < n; ++u) ord[u] = u;
+    std::stable_sort(ord.begin(), ord.end(), [&](int x, int y) { return w[x] > w[y]; });
+    std::vector<long long> load(G, 0);
+    for (auto& l : lists) l.clear();
+    for (int u : ord) {
+      int best = 0;
+      for (int m = 1; m < G; ++m)
+        if (load[m] < load[best]) best = m;
+      load[best] += w[u];
+      lists[best].push_back(u);
+    }
+    for (int m = 0; m < G; ++m) {
+      wl.start[g * G + m] = (uint16_t)pos;
+      for (int u : lists[m]) wl.item[pos++] = (uint16_t)u;
+    }
+  }
+  wl.start[p.groups * G] = (uint16_t)pos;
+  return true;
+}
+
 template <int D, bool ZZ>
 static ra_status launch(const AttnLaunch& a) {
   using C = Cfg<D>;
@@ -825,8 +947,10 @@ static ra_status launch(const AttnLaunch& a) {
       !encode_qkv_map(&tv, a.v, a.BH, a.N, c, a.P, D, mode))
     return RA_ERR_CUDA;
   static int attr_set[64] = {0};
+  static int attr_list_set[64] = {0};
   if (a.device < 64 && !attr_set[a.device]) {
-    if (cudaFuncSetAttribute(attn_fwd_kernel<D, ZZ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(attn_fwd_kernel<D, ZZ, NoLists>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmemBytes) != cudaSuccess)
       return RA_ERR_CUDA;
     attr_set[a.device] = 1;
@@ -866,8 +990,42 @@ static ra_status launch(const AttnLaunch& a) {
     p.ctas_per_group = G;
     grid = G * p.groups;
   }
-  attn_fwd_kernel<D, ZZ><<<grid, C::kThreads, C::kSmemBytes, (cudaStream_t)a.stream>>>(tq, tk, tv,
-                                                                                        p);
+  // Work lists for small causal problems of the striped layout (whose items
+  // differ in weight by pair index; measured at N = 8192, H = 16, P = 8:
+  // +11 % striped, while the zigzag and contiguous layouts measured equal or
+  // slower with them); they depend only on the shape and are built once per
+  // shape.
+  if (!a.sched_free && a.blk_kb < 0 && a.causal && a.striped && items_total <= kListItemsUsed) {
+    static std::mutex mu;
+    static std::map<std::vector<long long>, std::shared_ptr<WorkLists>> cache;
+    const std::vector<long long> key = {p.BH, p.N, p.P, p.striped, p.zigzag, p.causal,
+                                        p.groups, p.ctas_per_group};
+    std::shared_ptr<WorkLists> wl;
+    {
+      std::lock_guard<std::mutex> lock(mu);
+      auto found = cache.find(key);
+      if (found == cache.end()) {
+        auto built = std::make_shared<WorkLists>();
+        if (!build_lists(p, ZZ, *built)) built.reset();
+        found = cache.emplace(key, built).first;
+      }
+      wl = found->second;
+    }
+    if (wl) {
+      if (a.device < 64 && !attr_list_set[a.device]) {
+        if (cudaFuncSetAttribute(attn_fwd_kernel<D, ZZ, WorkLists>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::kSmemBytes) != cudaSuccess)
+          return RA_ERR_CUDA;
+        attr_list_set[a.device] = 1;
+      }
+      attn_fwd_kernel<D, ZZ, WorkLists>
+          <<<grid, C::kThreads, C::kSmemBytes, (cudaStream_t)a.stream>>>(tq, tk, tv, p, *wl);
+      return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+    }
+  }
+  attn_fwd_kernel<D, ZZ, NoLists>
+      <<<grid, C::kThreads, C::kSmemBytes, (cudaStream_t)a.stream>>>(tq, tk, tv, p, NoLists{});
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
