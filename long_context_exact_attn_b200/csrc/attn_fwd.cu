@@ -9,13 +9,15 @@
 // and O is divided by l once at the end.  Tiles that the block's causal
 // mask hides completely are never loaded or computed.
 //
-// Kernel organisation (one persistent CTA per SM, 320 threads):
+// Kernel organisation (one persistent CTA per SM, 384 threads):
 //   warps 0-3  softmax warpgroup for query tile 0 of the CTA's tile pair
 //   warps 4-7  softmax warpgroup for query tile 1
 //   warp  8    TMA producer: Q tile pair once per work item, then K and V
 //              tiles into a ring of shared-memory slots
 //   warp  9    tcgen05 issuer (warp-uniform, one elected lane issues) and
 //              TMEM owner
+//   warps 10-11 idle: with warps 8-9 they form the warpgroup that hands
+//              registers to the softmax warpgroups (setmaxnreg)
 // Variants of the same kernel: the zigzag layout (template parameter ZZ:
 // each key block walked as its two chunks), token-order addressing (the
 // layout's permutation applied in the TMA coordinates and the epilogue's
@@ -118,7 +120,16 @@ struct Cfg {
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 384;
+  // Register split (setmaxnreg, per warpgroup): the CTA is launched with
+  // 384 x kRegsLaunch registers; the warpgroup of producer, MMA and two idle
+  // warps gives some back (down to kRegsLow) and the two softmax warpgroups
+  // take them (up to kRegsHigh).  The split may not need more than the launch
+  // holds, or the softmax warpgroups' request would wait forever; the host
+  // checks the built kernel's register count before the first launch.
+  static constexpr int kRegsLaunch = 168, kRegsLow = 112, kRegsHigh = 192;
+  static_assert(256 * kRegsHigh + 128 * kRegsLow <= kThreads * kRegsLaunch,
+                "register split must fit in the launched registers");
 };
 
 // ------------------------------------------------------------ work items
@@ -394,8 +405,19 @@ __device__ __forceinline__ size_t out_row(const AttnParams& p, int bh, int j, in
   return (size_t)bh * p.N + t;
 }
 
+// Per-warpgroup register budget (setmaxnreg; every warp of the warpgroup
+// executes the same instruction).
+template <int N>
+__device__ __forceinline__ void reg_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void reg_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 template <int D, bool ZZ, class Lists>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const AttnParams p,
                 const __grid_constant__ Lists wl) {
@@ -455,6 +477,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // Register budgets: each warpgroup executes one setmaxnreg, all its warps
+  // at the same instruction, at the top of the branch that holds all of its
+  // code (so that the compiler allocates every branch within its budget).
+  // Warps 10 and 11 only complete the third warpgroup.
+  if (warp >= 8) {
+  reg_dealloc<C::kRegsLow>();
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -629,8 +657,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       wmbar_wait(bar_drain, 0, &no_abort, p.drain_timeout_ns);
     }
     __syncwarp();
+  }
   } else {
     // ----------------------------------------------------- softmax warpgroups
+    reg_alloc<C::kRegsHigh>();
     const int t = warp / 4;                 // query tile of the pair
     const int wq = warp % 4;                // TMEM lane quarter
     const int row = wq * 32 + lane;         // row within the query tile
@@ -730,8 +760,23 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
           }
           tmem_st16(tS + ch * 16, pk);
-          if (ch == 1 && !(rescale && acc)) {
-            // keys 0-63 of P are in TMEM: let P V start on them
+          if (ch == 1) {
+            if (rescale && acc) {
+              // O (the previous tiles' P V: complete, since this tile's
+              // scores were committed after it) moves to the new max before
+              // this tile's P V adds to it; 32 columns at a time, while the
+              // scores of keys 64-127 are still held
+              const uint64_t a2 = f2(alpha, alpha);
+#pragma unroll 1
+              for (int q4 = 0; q4 < D / 32; ++q4) {
+                uint32_t o32[32];
+                tmem_ld32(tO + q4 * 32, o32);
+                tmem_wait_ld();
+                scale_row32(o32, a2);
+                tmem_st32(tO + q4 * 32, o32);
+              }
+            }
+            // keys 0-63 of P (and a rescaled O) are in TMEM: let P V start
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -743,27 +788,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           unf2(fadd2(fadd2(sum_e[0], sum_e[1]), fadd2(sum_e[2], sum_e[3])), a, b);
           l += a + b;
         }
-        if (rescale && acc) {
-          uint32_t o0[32], o1[32], o2[32], o3[32];
-          tmem_ld32(tO + 0, o0);
-          if (D > 32) tmem_ld32(tO + 32, o1);
-          if (D > 64) tmem_ld32(tO + 64, o2);
-          if (D > 96) tmem_ld32(tO + 96, o3);
-          tmem_wait_ld();
-          const uint64_t a2 = f2(alpha, alpha);
-          scale_row32(o0, a2);
-          tmem_st32(tO + 0, o0);
-          if (D > 32) { scale_row32(o1, a2); tmem_st32(tO + 32, o1); }
-          if (D > 64) { scale_row32(o2, a2); tmem_st32(tO + 64, o2); }
-          if (D > 96) { scale_row32(o3, a2); tmem_st32(tO + 96, o3); }
-        }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          if (rescale && acc) mbar_arrive(my_p_full);   // O had to be rescaled first
-          mbar_arrive(my_p_full2);
-        }
+        if (lane == 0) mbar_arrive(my_p_full2);
         acc = true;
       }
       if (!ok) break;
@@ -936,6 +964,17 @@ static bool build_lists(const AttnParams& p, bool zz, WorkLists& wl) {
   return true;
 }
 
+// The softmax warpgroups' setmaxnreg.inc waits until the other warpgroup's
+// .dec has freed enough of the registers the CTA was launched with: a build
+// whose register count would leave it waiting is never launched.
+template <int D, class K>
+static bool register_split_fits(K kernel) {
+  using C = Cfg<D>;
+  cudaFuncAttributes fa;
+  return cudaFuncGetAttributes(&fa, kernel) == cudaSuccess &&
+         fa.numRegs * C::kThreads >= 256 * C::kRegsHigh + 128 * C::kRegsLow;
+}
+
 template <int D, bool ZZ>
 static ra_status launch(const AttnLaunch& a) {
   using C = Cfg<D>;
@@ -951,7 +990,8 @@ static ra_status launch(const AttnLaunch& a) {
   if (a.device < 64 && !attr_set[a.device]) {
     if (cudaFuncSetAttribute(attn_fwd_kernel<D, ZZ, NoLists>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kSmemBytes) != cudaSuccess)
+                             C::kSmemBytes) != cudaSuccess ||
+        !register_split_fits<D>(attn_fwd_kernel<D, ZZ, NoLists>))
       return RA_ERR_CUDA;
     attr_set[a.device] = 1;
   }
@@ -1015,7 +1055,8 @@ static ra_status launch(const AttnLaunch& a) {
       if (a.device < 64 && !attr_list_set[a.device]) {
         if (cudaFuncSetAttribute(attn_fwd_kernel<D, ZZ, WorkLists>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::kSmemBytes) != cudaSuccess)
+                                 C::kSmemBytes) != cudaSuccess ||
+            !register_split_fits<D>(attn_fwd_kernel<D, ZZ, WorkLists>))
           return RA_ERR_CUDA;
         attr_list_set[a.device] = 1;
       }
