@@ -70,6 +70,7 @@ struct AttnParams {
   __nv_bfloat16* o;
   float* lse;
   int o_f32;          // O written as float32 (o then points to float rows)
+  int o_v8;           // o is 32-byte aligned: O rows written in 32-byte stores
   int tok;            // q, k, v, o, lse in token order: the layout's permutation
                       // is applied in the TMA coordinates and the epilogue
   int BH;             // B * H
@@ -403,6 +404,13 @@ __device__ __forceinline__ size_t out_row(const AttnParams& p, int bh, int j, in
     t = (size_t)j * p.c + x;
   }
   return (size_t)bh * p.N + t;
+}
+
+// 32 bytes (8 words) to global memory in one store; dst 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void* dst, const uint32_t* w) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(w[0]),
+               "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
 }
 
 // Per-warpgroup register budget (setmaxnreg; every warp of the warpgroup
@@ -814,23 +822,38 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           for (int i = 0; i < 32; ++i) orow[i] = 0u;
         }
         if (valid && p.o_f32) {
-          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.o) + grow * D + q * 32);
+          float* dstf = reinterpret_cast<float*>(p.o) + grow * D + q * 32;
+          if (p.o_v8) {
+            uint32_t w[32];
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(__uint_as_float(orow[4 * i]) * inv_l,
-                                 __uint_as_float(orow[4 * i + 1]) * inv_l,
-                                 __uint_as_float(orow[4 * i + 2]) * inv_l,
-                                 __uint_as_float(orow[4 * i + 3]) * inv_l);
+            for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(orow[i]) * inv_l);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) st_global_v8(dstf + 8 * i, w + 8 * i);
+          } else {
+            float4* dst = reinterpret_cast<float4*>(dstf);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(orow[4 * i]) * inv_l,
+                                   __uint_as_float(orow[4 * i + 1]) * inv_l,
+                                   __uint_as_float(orow[4 * i + 2]) * inv_l,
+                                   __uint_as_float(orow[4 * i + 3]) * inv_l);
+          }
         } else if (valid) {
           uint32_t w[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             w[i] = pack_bf16x2(__uint_as_float(orow[2 * i]) * inv_l,
                                __uint_as_float(orow[2 * i + 1]) * inv_l);
-          uint4* dst = reinterpret_cast<uint4*>(orow_g + q * 32);
+          if (p.o_v8) {
+            // 32-byte stores: every store fills whole 32-byte sectors
+            st_global_v8(orow_g + q * 32, w);
+            st_global_v8(orow_g + q * 32 + 16, w + 8);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(orow_g + q * 32);
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          }
         }
       }
       if (valid) p.lse[grow] = (acc && l > 0.f) ? (m2 + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
@@ -998,6 +1021,7 @@ static ra_status launch(const AttnLaunch& a) {
   AttnParams p;
   p.o = reinterpret_cast<__nv_bfloat16*>(a.o);
   p.o_f32 = a.o_f32;
+  p.o_v8 = (reinterpret_cast<uintptr_t>(a.o) % 32) == 0;
   p.tok = a.tok;
   p.lse = a.lse;
   p.BH = (int)a.BH;

@@ -388,3 +388,25 @@ def test_token_order_is_bit_identical_to_partitioned_path(case):
     assert torch.equal(o_t, o_r)
     assert torch.equal(l_t, l_r)
     assert torch.equal(o32.to(torch.bfloat16), o_t)
+
+
+@pytest.mark.parametrize("o_f32", [False, True])
+def test_output_alignment_16_and_32_bytes_give_identical_results(o_f32):
+    """O rows are written with 32-byte stores when the output is 32-byte
+    aligned and with 16-byte stores otherwise (the ABI asks 16); both paths
+    give the same bits."""
+    w = W.Workload("align", 1, 2, 2048, 128, 4, W.STRIPED, True, 19, qk_scale_up=3.0)
+    q, k, v = (t.cuda() for t in W.make_qkv(w))
+    dt = torch.float32 if o_f32 else torch.bfloat16
+    esz = 4 if o_f32 else 2
+    n = q.numel()
+    big = torch.empty(n + 32 // esz, dtype=dt, device="cuda")
+    o_32 = big[:n].view(q.shape)
+    o_16 = big[16 // esz:16 // esz + n].view(q.shape)
+    assert o_32.data_ptr() % 32 == 0 and o_16.data_ptr() % 32 == 16
+    o1, l1 = ops.attn_fwd(q, k, v, w.P, w.layout, True, out=o_32, o_f32=o_f32)
+    r1, rl1 = o1.clone(), l1.clone()
+    o2, l2 = ops.attn_fwd(q, k, v, w.P, w.layout, True, out=o_16, o_f32=o_f32)
+    torch.cuda.synchronize()
+    assert ops.device_fault() == 0
+    assert torch.equal(r1, o2) and torch.equal(rl1, l2)
