@@ -83,6 +83,8 @@ struct AttnParams {
   int causal;
   int groups;         // shard groups (owner schedule) or 1 (free schedule)
   int ctas_per_group;
+  int helpers;        // owner schedule: CTAs on the SMs left over by the groups
+  int ceded;          // items at the end of every group's list that the helpers take
   float c2;           // scale * log2(e)
   unsigned long long timeout_ns;        // limit of every main-loop wait
   unsigned long long drain_timeout_ns;  // limit of the waits that drain the CTA's own
@@ -161,13 +163,28 @@ __device__ __forceinline__ bool item_at(const AttnParams& p, int g, int u, Item&
   return true;
 }
 
-// k-th item of this CTA: snake order over the group's members.
+// Items of group g.
+__device__ __forceinline__ int group_items(const AttnParams& p, int g) {
+  return p.npairs * ((p.P - g + p.groups - 1) / p.groups) * p.BH;
+}
+
+// k-th item of this CTA: snake order over the group's members, except the
+// group's last `ceded` items (its lightest), which go to the helper CTAs.
+// Helper h takes them from groups h, h + helpers, h + 2 helpers, ...
 __device__ __forceinline__ bool cta_item(const AttnParams& p, const NoLists&, int k, Item& it) {
-  const int g = blockIdx.x / p.ctas_per_group;
-  const int m = blockIdx.x % p.ctas_per_group;
-  if (g >= p.groups) return false;
   const int G = p.ctas_per_group;
+  const int base = p.groups * G;
+  if ((int)blockIdx.x >= base) {
+    if (p.ceded == 0) return false;
+    const int gi = k / p.ceded;
+    const int g = (int)blockIdx.x - base + gi * p.helpers;
+    if (g >= p.groups) return false;
+    return item_at(p, g, group_items(p, g) - p.ceded + (k - gi * p.ceded), it);
+  }
+  const int g = blockIdx.x / G;
+  const int m = blockIdx.x % G;
   const int u = k * G + ((k & 1) ? (G - 1 - m) : m);
+  if (u >= group_items(p, g) - p.ceded) return false;
   return item_at(p, g, u, it);
 }
 
@@ -955,7 +972,7 @@ static bool build_lists(const AttnParams& p, bool zz, WorkLists& wl) {
       const int per_head = p.npairs * n_sh;
       const int rem = u % per_head;
       int j, pair;
-      if (p.causal && !p.striped && !zz) {
+      if (p.causal && !p.striped) {
         const int sh_rank = rem / p.npairs;
         j = g + (n_sh - 1 - sh_rank) * p.groups;
         pair = p.npairs - 1 - (rem - sh_rank * p.npairs);
@@ -996,6 +1013,72 @@ static bool register_split_fits(K kernel) {
   cudaFuncAttributes fa;
   return cudaFuncGetAttributes(&fa, kernel) == cudaSuccess &&
          fa.numRegs * C::kThreads >= 256 * C::kRegsHigh + 128 * C::kRegsLow;
+}
+
+// Items each owner group cedes to the helper CTAs (the SMs left over after
+// groups x G): the count that minimises the busiest CTA's key-tile steps,
+// with the groups' CTAs dealing the rest of their lists in snake order and
+// helper h taking the ceded items of groups h, h + E, ...  The same count
+// for every group; 0 when ceding does not help.
+static int plan_ceded(const AttnParams& p, bool zz, int E) {
+  const int G = p.ctas_per_group;
+  if (E <= 0) return 0;
+  int n_min = INT32_MAX;
+  for (int g = 0; g < p.groups; ++g) {
+    const int n_sh = (p.P - g + p.groups - 1) / p.groups;
+    n_min = std::min(n_min, p.npairs * n_sh * p.BH);
+  }
+  const int t_max = n_min / 2;
+  if (t_max < 1) return 0;
+  // cta[g][m]: load of CTA m of group g with t items ceded; help[h]
+  std::vector<std::vector<long long>> cta(p.groups, std::vector<long long>(G, 0));
+  std::vector<std::vector<long long>> w(p.groups);
+  std::vector<long long> help(E, 0);
+  for (int g = 0; g < p.groups; ++g) {
+    const int n_sh = (p.P - g + p.groups - 1) / p.groups;
+    const int n = p.npairs * n_sh * p.BH;
+    const int per_head = p.npairs * n_sh;
+    w[g].resize(n);
+    for (int u = 0; u < n; ++u) {
+      const int rem = u % per_head;
+      int j, pair;
+      if (p.causal && !p.striped) {
+        const int sh_rank = rem / p.npairs;
+        j = g + (n_sh - 1 - sh_rank) * p.groups;
+        pair = p.npairs - 1 - (rem - sh_rank * p.npairs);
+      } else {
+        const int pr = rem / n_sh;
+        pair = p.npairs - 1 - pr;
+        j = g + (rem - pr * n_sh) * p.groups;
+      }
+      w[g][u] = item_steps(p, j, pair, zz);
+      const int k = u / G, r = u % G;
+      cta[g][(k & 1) ? (G - 1 - r) : r] += w[g][u];
+    }
+  }
+  auto makespan = [&]() {
+    long long mx = 0;
+    for (auto& row : cta)
+      for (long long v : row) mx = std::max(mx, v);
+    for (long long v : help) mx = std::max(mx, v);
+    return mx;
+  };
+  long long best = makespan();
+  int best_t = 0;
+  for (int t = 1; t <= t_max; ++t) {
+    for (int g = 0; g < p.groups; ++g) {
+      const int u = (int)w[g].size() - t;   // the item ceded at this step
+      const int k = u / G, r = u % G;
+      cta[g][(k & 1) ? (G - 1 - r) : r] -= w[g][u];
+      help[g % E] += w[g][u];
+    }
+    const long long ms = makespan();
+    if (ms < best) {
+      best = ms;
+      best_t = t;
+    }
+  }
+  return best_t;
 }
 
 template <int D, bool ZZ>
@@ -1054,6 +1137,8 @@ static ra_status launch(const AttnLaunch& a) {
     p.ctas_per_group = G;
     grid = G * p.groups;
   }
+  p.helpers = 0;
+  p.ceded = 0;
   // Work lists for small causal problems of the striped layout (whose items
   // differ in weight by pair index; measured at N = 8192, H = 16, P = 8:
   // +11 % striped, while the zigzag and contiguous layouts measured equal or
@@ -1087,6 +1172,27 @@ static ra_status launch(const AttnLaunch& a) {
       attn_fwd_kernel<D, ZZ, WorkLists>
           <<<grid, C::kThreads, C::kSmemBytes, (cudaStream_t)a.stream>>>(tq, tk, tv, p, *wl);
       return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+    }
+  }
+  // Owner schedule: the SMs left over by the groups become helper CTAs that
+  // take the lightest items of every group (planned once per shape).
+  if (!a.sched_free && a.blk_kb < 0 && a.num_sms - grid > 0 && p.groups > 1) {
+    const int E = std::min(a.num_sms - grid, p.groups);
+    static std::mutex mu;
+    static std::map<std::vector<long long>, int> cache;
+    const std::vector<long long> key = {p.BH, p.N, p.P, p.striped, p.zigzag, p.causal,
+                                        p.groups, p.ctas_per_group, E};
+    int t;
+    {
+      std::lock_guard<std::mutex> lock(mu);
+      auto found = cache.find(key);
+      if (found == cache.end()) found = cache.emplace(key, plan_ceded(p, ZZ, E)).first;
+      t = found->second;
+    }
+    if (t > 0) {
+      p.helpers = E;
+      p.ceded = t;
+      grid += E;
     }
   }
   attn_fwd_kernel<D, ZZ, NoLists>
