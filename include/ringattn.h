@@ -96,6 +96,18 @@ typedef int ra_status;
  * load-balanced schedule; same results, same tile skipping). */
 #define RA_SCHED_FREE 0x100
 
+/* Optional kernel flag for ra_attn_fwd, OR-ed into `layout`: RA_CTA_PAIR
+ * runs the forward on pairs of SMs (clusters of two CTAs sharing each
+ * tensor-core MMA, M = 256; each SM loads half of every key/value tile).
+ * It applies to d = 128 in layout order (not RA_TOKEN_ORDER, not RA_ZIGZAG);
+ * elsewhere it is ignored.  Same results (bit-identical on the shapes
+ * tested): each row is the same online softmax over the same key tiles.
+ * On B200 it measured slower than the default kernel at every benchmark
+ * shape (717 against 1023 TFLOP/s at N = 131072, H = 8, P = 8 striped): the
+ * MMA issuer waits for the softmax of both SMs, across the pair, on every
+ * tile.  Not recommended for speed; it exists as the tested two-SM form. */
+#define RA_CTA_PAIR 0x800
+
 /* Optional output flag for ra_attn_fwd, OR-ed into `layout`: O is written as
  * float32 [B, H, N, d] (o must hold 4 bytes per element) instead of bf16,
  * e.g. for callers that merge partial results or want O before rounding. */

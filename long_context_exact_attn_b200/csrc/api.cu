@@ -206,7 +206,8 @@ static ra_status fwd_prepare(const void* q, const void* k, const void* v, void* 
                              int64_t B, int64_t H, int64_t N, int64_t d, int P, int layout,
                              int causal, float scale, void* stream, AttnLaunch* out) {
   if (!q || !k || !v || !o || !lse) return RA_ERR_NULL;
-  if (layout & ~(0xff | RA_SCHED_FREE | RA_O_F32 | RA_TOKEN_ORDER)) return RA_ERR_LAYOUT;
+  if (layout & ~(0xff | RA_SCHED_FREE | RA_O_F32 | RA_TOKEN_ORDER | RA_CTA_PAIR))
+    return RA_ERR_LAYOUT;
   const int base = layout & 0xff;
   if (base != RA_CONTIGUOUS && base != RA_STRIPED && base != RA_ZIGZAG) return RA_ERR_LAYOUT;
   if (d != 64 && d != 128) return RA_ERR_HEADDIM;
@@ -237,6 +238,7 @@ static ra_status fwd_prepare(const void* q, const void* k, const void* v, void* 
   a.sched_free = (layout & RA_SCHED_FREE) != 0;
   a.o_f32 = o_f32;
   a.tok = (layout & RA_TOKEN_ORDER) != 0;
+  a.pair = (layout & RA_CTA_PAIR) != 0;
   a.scale = scale;
   a.device = dev;
   a.num_sms = info.num_sms;

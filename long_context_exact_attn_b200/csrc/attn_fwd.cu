@@ -292,6 +292,20 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
+// Max of 128 scores: eight independent chains of 3-input max.
+__device__ __forceinline__ float row_max128(const float (&s)[128]) {
+  float mx8[8];
+#pragma unroll
+  for (int a = 0; a < 8; ++a) {
+    float acc = fmax3(s[a], s[a + 8], s[a + 16]);
+#pragma unroll
+    for (int kq = 3; kq < 15; kq += 2) acc = fmax3(acc, s[a + 8 * kq], s[a + 8 * kq + 8]);
+    mx8[a] = fmaxf(acc, s[a + 120]);
+  }
+  return fmaxf(fmax3(mx8[0], mx8[1], mx8[2]),
+               fmaxf(fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+}
+
 // Packed pairs of fp32 (sm_100 f32x2 arithmetic: one instruction, two lanes).
 __device__ __forceinline__ uint64_t f2(float lo, float hi) {
   uint64_t r;
@@ -889,17 +903,563 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   }
 }
 
+// ===================================================== CTA-pair forward
+// The same method with the tensor-core work of two SMs fused: a cluster of
+// two CTAs issues M = 256 tcgen05 MMAs (cta_group::2).  CTA r of the pair
+// holds query tiles 4q+2r and 4q+2r+1 of its item (query tiles 4q..4q+3 of
+// one shard), and of every key/value tile only its half: key rows
+// [64r, 64r+64) of K and value columns [64r, 64r+64) of V.  Each SM thus
+// reads half of the B operand from its shared memory per MMA and loads half
+// of every K/V tile, and its ring of half-tile slots looks twice as far
+// ahead.  MMA slot t multiplies the pair's tiles 4q+t (rows 0-127, CTA 0)
+// and 4q+2+t (rows 128-255, CTA 1); each CTA's softmax warpgroup t handles
+// its own 128 rows of slot t in its own tensor memory, exactly as in the
+// single-CTA kernel.  CTA 0 issues every MMA; the barriers that gather both
+// CTAs' inputs (loaded tiles, published P, released O) live in CTA 0, and
+// each of CTA 0's commits is sent to the matching barrier of both CTAs.
+template <int D>
+struct PairCfg {
+  static constexpr int kTileBytes = kBM * D * 2;      // one query tile of this CTA
+  static constexpr int kHalfBytes = kTileBytes / 2;   // this CTA's half of a K or V tile
+  static constexpr int kChunks = D / 64;
+  static constexpr int kSlots = 10;                   // half-tile ring slots
+  static constexpr int kQOff = 0;
+  static constexpr int kRingOff = 2 * kTileBytes;
+  static constexpr int kBarOff = kRingOff + kSlots * kHalfBytes;
+  // barriers: q_full, q_empty, full[kSlots], empty[kSlots], s_full[2],
+  // p_full[2], p_full2[2], o_full[2], o_free[2], drain
+  static constexpr int kNumBars = 2 + 2 * kSlots + 10 + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
+  static constexpr int kThreads = 384;
+  static constexpr int kRegsLaunch = 168, kRegsLow = 112, kRegsHigh = 192;
+};
+
+// Items of the pair kernel are (b*h, shard, quad of query tiles); the
+// schedule is the single-CTA one over clusters (npairs counts quads).
+__device__ __forceinline__ bool pair_item(const AttnParams& p, int k, Item& it) {
+  const int ci = blockIdx.x >> 1;
+  const int G = p.ctas_per_group;
+  const int base = p.groups * G;
+  if (ci >= base) {
+    if (p.ceded == 0) return false;
+    const int gi = k / p.ceded;
+    const int g = ci - base + gi * p.helpers;
+    if (g >= p.groups) return false;
+    return item_at(p, g, group_items(p, g) - p.ceded + (k - gi * p.ceded), it);
+  }
+  const int g = ci / G;
+  const int m = ci % G;
+  const int u = k * G + ((k & 1) ? (G - 1 - m) : m);
+  if (u >= group_items(p, g) - p.ceded) return false;
+  return item_at(p, g, u, it);
+}
+
+// The key tiles met by a quad of query tiles, in ring order (the union of
+// the four tiles' spans); kind[i] is the kind of tile 4q+i.
+struct TileSeqQuad {
+  int j, P, c, striped, causal;
+  int x0;
+  int r, kt, kend;
+  TileSpan sp[4];
+  BlockMask bm;
+  int kb;
+  __device__ __forceinline__ void init(const AttnParams& p, const Item& it) {
+    j = it.j; P = p.P; c = p.c; striped = p.striped; causal = p.causal;
+    x0 = it.pair * 4 * kBM;
+    r = -1; kt = 0; kend = 0;
+  }
+  __device__ __forceinline__ bool next(int& kb_out, int& y0, int (&kind)[4], BlockMask& m) {
+    while (kt >= kend) {
+      if (++r >= P) return false;
+      kb = key_block(j, r, P);
+      bm = block_mask(j, kb, striped, causal);
+      kend = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        sp[i] = tile_span(bm, x0 + i * kBM, c);
+        kend = sp[i].part_end > kend ? sp[i].part_end : kend;
+      }
+      kt = 0;
+    }
+    kb_out = kb;
+    y0 = kt * kBN;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) kind[i] = tile_kind_at(sp[i], kt);
+    m = bm;
+    ++kt;
+    return true;
+  }
+};
+
+// Bounded wait against a deadline shared by several waits (drains).
+__device__ __forceinline__ bool mbar_wait_until(uint32_t bar, uint32_t parity,
+                                                unsigned long long deadline);
+__device__ __forceinline__ bool wmbar_wait_until(uint32_t bar, uint32_t parity,
+                                                 unsigned long long deadline) {
+  return __all_sync(0xffffffffu, mbar_wait_until(bar, parity, deadline));
+}
+__device__ __forceinline__ bool mbar_wait_until(uint32_t bar, uint32_t parity,
+                                                unsigned long long deadline) {
+  while (!mbar_try_wait(bar, parity))
+    if (global_timer_ns() > deadline) return false;
+  return true;
+}
+
+template <int D>
+__device__ __forceinline__ void pair_mma_qk(uint32_t s_tmem, uint32_t qa, uint32_t ka) {
+  constexpr uint32_t idesc = idesc_bf16_f32(2 * kBM, kBN, 0, 0);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk)
+    pair::mma_ss_w(s_tmem, smem_desc_sw128(qa + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024),
+                   smem_desc_sw128(ka + (kk / 4) * 8192 + (kk % 4) * 32, 16, 1024), idesc, kk > 0);
+}
+
+template <int D, int KK0, int KK1>
+__device__ __forceinline__ void pair_mma_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t va,
+                                            uint32_t acc) {
+  constexpr uint32_t idesc = idesc_bf16_f32(2 * kBM, D, 0, 1);
+#pragma unroll
+  for (int kk = KK0; kk < KK1; ++kk)
+    pair::mma_ts_w(o_tmem, p_tmem + kk * 8, smem_desc_sw128(va + kk * 2048, 16384, 1024), idesc,
+                   (acc | (uint32_t)kk) != 0);
+}
+
+template <int D>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
+attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
+                     const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+  using C = PairCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase + C::kQOff;
+  const uint32_t sRing = sbase + C::kRingOff;
+  const uint32_t bars = sbase + C::kBarOff;
+  const uint32_t bar_q_full = bars + 0 * 8;
+  const uint32_t bar_q_empty = bars + 1 * 8;
+  auto bar_full = [&](int s) { return bars + (2 + s) * 8; };
+  auto bar_empty = [&](int s) { return bars + (2 + C::kSlots + s) * 8; };
+  const uint32_t bar_s_full = bars + (2 + 2 * C::kSlots) * 8;   // [2]
+  const uint32_t bar_p_full = bar_s_full + 16;                  // [2]
+  const uint32_t bar_p_full2 = bar_p_full + 16;                 // [2]
+  const uint32_t bar_o_full = bar_p_full2 + 16;                 // [2]
+  const uint32_t bar_o_free = bar_o_full + 16;                  // [2]
+  const uint32_t bar_drain = bar_o_free + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const uint32_t rank = pair::cta_rank();
+  const bool leader = rank == 0;
+  // the even CTA's copy of a barrier, and the odd CTA's
+  auto at0 = [&](uint32_t bar) { return pair::map_to(bar, 0); };
+  auto at1 = [&](uint32_t bar) { return pair::map_to(bar, 1); };
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q_full, 1);
+    mbar_init(bar_q_empty, 1);
+    for (int s = 0; s < C::kSlots; ++s) {
+      mbar_init(bar_full(s), 1);
+      mbar_init(bar_empty(s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar_s_full + 8 * t, 1);
+      mbar_init(bar_p_full + 8 * t, 8);     // four softmax warps of each CTA
+      mbar_init(bar_p_full2 + 8 * t, 8);
+      mbar_init(bar_o_full + 8 * t, 1);
+      mbar_init(bar_o_free + 8 * t, 8);
+    }
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    pair::tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    pair::tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  tc_fence_before();
+  // both CTAs' barriers are initialised and tensor memory is allocated
+  // before either CTA touches the other's barriers
+  pair::cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp >= 8) {
+  reg_dealloc<C::kRegsLow>();
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t n_loads = 0;
+      Item it;
+      bool ok = true;
+      for (int k = 0; ok && pair_item(p, k, it); ++k) {
+        if (!mbar_wait(bar_q_empty, (k & 1) ^ 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+        if (leader) mbar_arrive_expect_tx(bar_q_full, 4 * C::kTileBytes);
+        const int x0 = it.pair * 4 * kBM + (int)rank * 2 * kBM;
+        for (int t = 0; t < 2; ++t)
+          for (int ch = 0; ch < C::kChunks; ++ch)
+            pair::tma_load_4d(sQ + t * C::kTileBytes + ch * 16384, &tmQ, at0(bar_q_full), ch * 64,
+                              x0 + t * kBM, it.j, it.bh);
+        TileSeqQuad seq;
+        seq.init(p, it);
+        int kb, y0, kind[4];
+        BlockMask bm;
+        while (seq.next(kb, y0, kind, bm)) {
+          for (int kv = 0; kv < 2; ++kv) {
+            const int s = n_loads % C::kSlots;
+            const uint32_t ph = (n_loads / C::kSlots) & 1;
+            if (!mbar_wait(bar_empty(s), ph ^ 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+            if (leader) mbar_arrive_expect_tx(bar_full(s), 2 * C::kHalfBytes);
+            const uint32_t dst = sRing + s * C::kHalfBytes;
+            if (kv == 0) {
+              // key rows [64 rank, 64 rank + 64) of the tile, all d
+              for (int ch = 0; ch < C::kChunks; ++ch)
+                pair::tma_load_4d(dst + ch * (C::kHalfBytes / C::kChunks), &tmK, at0(bar_full(s)),
+                                  ch * 64, y0 + (int)rank * (kBN / 2), kb, it.bh);
+            } else {
+              // value columns [64 rank, 64 rank + 64) of the tile, all keys
+              pair::tma_load_4d(dst, &tmV, at0(bar_full(s)), (int)rank * 64, y0, kb, it.bh);
+            }
+            ++n_loads;
+          }
+          if (!ok) break;
+        }
+      }
+      if (leader) {
+        // Every load issued (by both CTAs) lands on this CTA's barriers;
+        // wait for the ones not consumed yet, under one deadline.
+        const unsigned long long deadline = global_timer_ns() + p.drain_timeout_ns;
+        const uint32_t first = n_loads > (uint32_t)C::kSlots ? n_loads - C::kSlots : 0;
+        for (uint32_t n = first; n < n_loads; ++n)
+          if (!mbar_wait_until(bar_full(n % C::kSlots), (n / C::kSlots) & 1, deadline)) break;
+      } else if (!ok) {
+        // after an abort the even CTA may never count these loads: give
+        // them time to land before this CTA can exit
+        const unsigned long long until = global_timer_ns() + 200000ull;
+        while (global_timer_ns() < until) {
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9 && leader) {
+    // ------------------------------------------------ MMA issuer (CTA 0)
+    {
+      const uint32_t tS0 = tmem + C::kColS0, tS1 = tmem + C::kColS1;
+      const uint32_t tO0 = tmem + C::kColO0, tO1 = tmem + C::kColO1;
+      const uint32_t sQ0 = sQ, sQ1 = sQ + C::kTileBytes;
+      const uint32_t s_full0 = bar_s_full, s_full1 = bar_s_full + 8;
+      const uint32_t p_full0 = bar_p_full, p_full1 = bar_p_full + 8;
+      const uint32_t p_full2_0 = bar_p_full2, p_full2_1 = bar_p_full2 + 8;
+      const uint32_t o_free0 = bar_o_free, o_free1 = bar_o_free + 8;
+      bool withhold = p.withhold_first_s != 0;
+      // a commit reaches the barrier of both CTAs
+      auto commit2 = [&](uint32_t bar) {
+        pair::mma_commit_w(bar);
+        pair::mma_commit_w(at1(bar));
+      };
+      uint32_t slot = 0, phase = 0;
+      uint32_t pc0 = 0, pc1 = 0;
+      uint32_t of0 = 0, of1 = 0;
+      Item it;
+      bool ok = true;
+      for (int k = 0; ok && pair_item(p, k, it); ++k) {
+        if (!pair::wmbar_wait(bar_q_full, k & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+        TileSeqQuad seq;
+        seq.init(p, it);
+        int kb, y0, kind[4];
+        BlockMask bm;
+        bool have = seq.next(kb, y0, kind, bm);
+        // slot t computes when either CTA's tile of it is visible
+        bool c0 = have && (kind[0] != TILE_SKIP || kind[2] != TILE_SKIP);
+        bool c1 = have && (kind[1] != TILE_SKIP || kind[3] != TILE_SKIP);
+        uint32_t acc0 = 0, acc1 = 0;
+        if (!have) {
+          bool okw = true;
+          while (okw && of0 < (uint32_t)k) okw = pair::wmbar_wait(o_free0, of0++ & 1, abort_flag, p.timeout_ns);
+          while (okw && of1 < (uint32_t)k) okw = pair::wmbar_wait(o_free1, of1++ & 1, abort_flag, p.timeout_ns);
+          if (!okw) { ok = false; break; }
+          commit2(bar_o_full + 0);
+          commit2(bar_o_full + 8);
+          commit2(bar_q_empty);
+          continue;
+        }
+        uint32_t kslot = slot;
+        if (!pair::wmbar_wait(bar_full(kslot), phase, abort_flag, p.timeout_ns)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t ka0 = sRing + kslot * C::kHalfBytes;
+        if (c0) {
+          pair_mma_qk<D>(tS0, sQ0, ka0);
+          if (!withhold) commit2(s_full0);
+          withhold = false;
+        }
+        if (c1) { pair_mma_qk<D>(tS1, sQ1, ka0); commit2(s_full1); }
+        commit2(bar_empty(kslot));
+        if (++slot == C::kSlots) { slot = 0; phase ^= 1; }
+        while (have) {
+          int nkind[4];
+          const bool more = seq.next(kb, y0, nkind, bm);
+          const bool n0 = more && (nkind[0] != TILE_SKIP || nkind[2] != TILE_SKIP);
+          const bool n1 = more && (nkind[1] != TILE_SKIP || nkind[3] != TILE_SKIP);
+          const uint32_t vslot = slot, vph = phase;
+          if (++slot == C::kSlots) { slot = 0; phase ^= 1; }
+          uint32_t nkslot = 0;
+          if (more) {
+            nkslot = slot;
+            if (!pair::wmbar_wait(bar_full(nkslot), phase, abort_flag, p.timeout_ns)) { ok = false; break; }
+            if (++slot == C::kSlots) { slot = 0; phase ^= 1; }
+          }
+          if (!pair::wmbar_wait(bar_full(vslot), vph, abort_flag, p.timeout_ns)) { ok = false; break; }
+          const uint32_t va = sRing + vslot * C::kHalfBytes;
+          const uint32_t nka = sRing + nkslot * C::kHalfBytes;
+          if (c0) {
+            bool okw = true;
+            while (okw && of0 < (uint32_t)k) okw = pair::wmbar_wait(o_free0, of0++ & 1, abort_flag, p.timeout_ns);
+            if (!okw) { ok = false; break; }
+            if (!pair::wmbar_wait(p_full0, pc0 & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+            tc_fence_after();
+            pair_mma_pv<D, 0, 4>(tO0, tS0, va, acc0);
+            if (!pair::wmbar_wait(p_full2_0, pc0 & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+            ++pc0;
+            tc_fence_after();
+            pair_mma_pv<D, 4, 8>(tO0, tS0, va, 1);
+            acc0 = 1;
+          }
+          if (n0) { tc_fence_after(); pair_mma_qk<D>(tS0, sQ0, nka); commit2(s_full0); }
+          if (c1) {
+            bool okw = true;
+            while (okw && of1 < (uint32_t)k) okw = pair::wmbar_wait(o_free1, of1++ & 1, abort_flag, p.timeout_ns);
+            if (!okw) { ok = false; break; }
+            if (!pair::wmbar_wait(p_full1, pc1 & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+            tc_fence_after();
+            pair_mma_pv<D, 0, 4>(tO1, tS1, va, acc1);
+            if (!pair::wmbar_wait(p_full2_1, pc1 & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+            ++pc1;
+            tc_fence_after();
+            pair_mma_pv<D, 4, 8>(tO1, tS1, va, 1);
+            acc1 = 1;
+          }
+          commit2(bar_empty(vslot));
+          if (n1) { tc_fence_after(); pair_mma_qk<D>(tS1, sQ1, nka); commit2(s_full1); }
+          if (more) commit2(bar_empty(nkslot));
+          have = more;
+          c0 = n0;
+          c1 = n1;
+        }
+        if (!ok) break;
+        {
+          bool okw = true;
+          while (okw && of0 < (uint32_t)k) okw = pair::wmbar_wait(o_free0, of0++ & 1, abort_flag, p.timeout_ns);
+          while (okw && of1 < (uint32_t)k) okw = pair::wmbar_wait(o_free1, of1++ & 1, abort_flag, p.timeout_ns);
+          if (!okw) { ok = false; break; }
+        }
+        commit2(bar_o_full + 0);
+        commit2(bar_o_full + 8);
+        commit2(bar_q_empty);
+      }
+      // Every pair MMA must be complete before either CTA frees its TMEM.
+      pair::mma_commit_w(bar_drain);
+      wmbar_wait_until(bar_drain, 0, global_timer_ns() + p.drain_timeout_ns);
+    }
+    __syncwarp();
+  }
+  } else {
+    // ----------------------------------------------------- softmax warpgroups
+    reg_alloc<C::kRegsHigh>();
+    const int t = warp / 4;                 // MMA slot; this CTA's tile 2 rank + t of the quad
+    const int wq = warp % 4;                // TMEM lane quarter
+    const int row = wq * 32 + lane;         // row within the query tile
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + (t ? C::kColS1 : C::kColS0) + lane_off;
+    const uint32_t tO = tmem + (t ? C::kColO1 : C::kColO0) + lane_off;
+    const uint32_t my_s_full = bar_s_full + 8 * t;
+    const uint32_t their_p_full = at0(bar_p_full + 8 * t);
+    const uint32_t their_p_full2 = at0(bar_p_full2 + 8 * t);
+    const uint32_t my_o_full = bar_o_full + 8 * t;
+    const uint32_t their_o_free = at0(bar_o_free + 8 * t);
+    const int mine = 2 * (int)rank + t;     // this warpgroup's tile of the quad
+    const float c2 = p.c2;
+    uint32_t s_cnt = 0;
+    Item it;
+    bool ok = true;
+    for (int k = 0; ok && pair_item(p, k, it); ++k) {
+      TileSeqQuad seq;
+      seq.init(p, it);
+      const int x = it.pair * 4 * kBM + mine * kBM + row;   // local query row in shard
+      float m2 = -INFINITY;
+      float l = 0.f;
+      bool acc = false;
+      int kb, y0, kind[4];
+      BlockMask bm;
+      while (seq.next(kb, y0, kind, bm)) {
+        if (kind[t] == TILE_SKIP && kind[2 + t] == TILE_SKIP) continue;   // slot not computed
+        const int my_kind = kind[mine];
+        if (!wmbar_wait(my_s_full, s_cnt & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+        ++s_cnt;
+        tc_fence_after();
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, sr[q]);
+        tmem_wait_ld();
+        float s[128];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[q * 32 + i] = __uint_as_float(sr[q][i]);
+        if (my_kind != TILE_FULL) {
+          // this CTA's tile of the slot is partial, or hidden entirely
+          // (the other CTA's tile needed the MMA): mask by the row limit
+          const int lim = my_kind == TILE_SKIP ? 0 : row_limit(bm, x, y0, p.c);
+#pragma unroll
+          for (int i = 0; i < 128; ++i)
+            if (i >= lim) s[i] = -INFINITY;
+        }
+        const float mx = row_max128(s);
+        const float m_cand = fmaxf(m2, mx * c2);
+        const bool rescale = __any_sync(0xffffffffu, m_cand > m2);
+        float alpha = 1.f;
+        if (rescale) {
+          alpha = (m_cand == -INFINITY) ? 1.f : ex2(m2 - m_cand);
+          l *= alpha;
+          m2 = m_cand;
+        }
+        const float msub = (m2 == -INFINITY) ? 0.f : m2;
+        const uint64_t c2x2 = f2(c2, c2);
+        const uint64_t nm2 = f2(-msub, -msub);
+        uint64_t sum_e[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int e = ch * 32 + 2 * i;
+            const uint64_t x2 = ffma2(f2(s[e], s[e + 1]), c2x2, nm2);
+            float a0, a1;
+            unf2(x2, a0, a1);
+            const float p0 = ex2(a0), p1 = ex2(a1);
+            pk[i] = pack_bf16x2(p0, p1);
+            sum_e[i & 3] = fadd2(sum_e[i & 3], f2(p0, p1));
+          }
+          tmem_st16(tS + ch * 16, pk);
+          if (ch == 1) {
+            if (rescale && acc) {
+              const uint64_t a2 = f2(alpha, alpha);
+#pragma unroll 1
+              for (int q4 = 0; q4 < D / 32; ++q4) {
+                uint32_t o32[32];
+                tmem_ld32(tO + q4 * 32, o32);
+                tmem_wait_ld();
+                scale_row32(o32, a2);
+                tmem_st32(tO + q4 * 32, o32);
+              }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) pair::mbar_arrive_cluster(their_p_full);
+          }
+        }
+        {
+          float a, b;
+          unf2(fadd2(fadd2(sum_e[0], sum_e[1]), fadd2(sum_e[2], sum_e[3])), a, b);
+          l += a + b;
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) pair::mbar_arrive_cluster(their_p_full2);
+        acc = true;
+      }
+      if (!ok) break;
+      if (!wmbar_wait(my_o_full, k & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+      tc_fence_after();
+      const bool valid = x < p.c;
+      const float inv_l = (acc && l > 0.f) ? 1.f / l : 0.f;
+      const size_t grow = out_row<false>(p, it.bh, it.j, valid ? x : 0);
+      __nv_bfloat16* orow_g = p.o + grow * D;
+#pragma unroll 1
+      for (int q = 0; q < D / 32; ++q) {
+        uint32_t orow[32];
+        tmem_ld32(tO + q * 32, orow);
+        tmem_wait_ld();
+        if (!acc) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) orow[i] = 0u;
+        }
+        if (valid && p.o_f32) {
+          float* dstf = reinterpret_cast<float*>(p.o) + grow * D + q * 32;
+          if (p.o_v8) {
+            uint32_t w[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(__uint_as_float(orow[i]) * inv_l);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) st_global_v8(dstf + 8 * i, w + 8 * i);
+          } else {
+            float4* dst = reinterpret_cast<float4*>(dstf);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(orow[4 * i]) * inv_l,
+                                   __uint_as_float(orow[4 * i + 1]) * inv_l,
+                                   __uint_as_float(orow[4 * i + 2]) * inv_l,
+                                   __uint_as_float(orow[4 * i + 3]) * inv_l);
+          }
+        } else if (valid) {
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            w[i] = pack_bf16x2(__uint_as_float(orow[2 * i]) * inv_l,
+                               __uint_as_float(orow[2 * i + 1]) * inv_l);
+          if (p.o_v8) {
+            st_global_v8(orow_g + q * 32, w);
+            st_global_v8(orow_g + q * 32 + 16, w + 8);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(orow_g + q * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          }
+        }
+      }
+      if (valid) p.lse[grow] = (acc && l > 0.f) ? (m2 + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) pair::mbar_arrive_cluster(their_o_free);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) atomicOr(&g_device_fault, 1u);
+  // CTA 0's MMAs (which write both CTAs' tensor memory) are complete: both
+  // CTAs may free their columns
+  pair::cluster_sync();
+  if (warp == 9) {
+    tc_fence_after();
+    pair::tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
 // ------------------------------------------------------------------ host
 // mode 0: [BH, P, c, d] (layout order, or token order of the contiguous
 // layout); mode 1: striped token order as [BH, c, P, d] (box over c);
 // mode 2: zigzag token order as [BH, 2P, c/2, d].
 static bool encode_qkv_map(CUtensorMap* map, const void* base, int64_t BH, int64_t N, int64_t c,
-                           int P, int d, int mode = 0) {
+                           int P, int d, int mode = 0, int box_rows = kBM) {
   PFN_encodeTiled enc = get_encode_tiled();
   if (!enc) return false;
   cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)c, (cuuint64_t)P, (cuuint64_t)BH};
   cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)c * d * 2, (cuuint64_t)N * d * 2};
-  cuuint32_t box[4] = {64, (cuuint32_t)kBM, 1, 1};
+  cuuint32_t box[4] = {64, (cuuint32_t)box_rows, 1, 1};
   if (mode == 1) {
     dims[1] = (cuuint64_t)P;
     dims[2] = (cuuint64_t)c;
@@ -1013,6 +1573,10 @@ static bool register_split_fits(K kernel) {
   cudaFuncAttributes fa;
   return cudaFuncGetAttributes(&fa, kernel) == cudaSuccess &&
          fa.numRegs * C::kThreads >= 256 * C::kRegsHigh + 128 * C::kRegsLow;
+}
+
+static int group_items_host(const AttnParams& p, int g) {
+  return p.npairs * ((p.P - g + p.groups - 1) / p.groups) * p.BH;
 }
 
 // Items each owner group cedes to the helper CTAs (the SMs left over after
@@ -1200,7 +1764,176 @@ static ra_status launch(const AttnLaunch& a) {
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
+// Key-tile steps of a quad of query tiles in the pair kernel (the union of
+// the four tiles' spans per round).  Mirrors TileSeqQuad::next.
+static long long quad_steps(const AttnParams& p, int j, int quad) {
+  long long steps = 0;
+  for (int r = 0; r < p.P; ++r) {
+    const BlockMask bm = block_mask(j, key_block(j, r, p.P), p.striped, p.causal);
+    int kend = 0;
+    for (int i = 0; i < 4; ++i) {
+      const TileSpan sp = tile_span(bm, quad * 4 * kBM + i * kBM, p.c);
+      kend = sp.part_end > kend ? sp.part_end : kend;
+    }
+    steps += kend;
+  }
+  return steps;
+}
+
+// Helper planning of the pair kernel: as plan_ceded, over clusters and quads.
+static int plan_ceded_quads(const AttnParams& p, int E) {
+  const int G = p.ctas_per_group;
+  if (E <= 0) return 0;
+  int n_min = INT32_MAX;
+  for (int g = 0; g < p.groups; ++g) n_min = std::min(n_min, group_items_host(p, g));
+  const int t_max = n_min / 2;
+  if (t_max < 1) return 0;
+  std::vector<std::vector<long long>> cta(p.groups, std::vector<long long>(G, 0));
+  std::vector<std::vector<long long>> w(p.groups);
+  std::vector<long long> help(E, 0);
+  for (int g = 0; g < p.groups; ++g) {
+    const int n = group_items_host(p, g);
+    const int n_sh = (p.P - g + p.groups - 1) / p.groups;
+    const int per_head = p.npairs * n_sh;
+    w[g].resize(n);
+    for (int u = 0; u < n; ++u) {
+      const int rem = u % per_head;
+      int j, quad;
+      if (p.causal && !p.striped) {
+        const int sh_rank = rem / p.npairs;
+        j = g + (n_sh - 1 - sh_rank) * p.groups;
+        quad = p.npairs - 1 - (rem - sh_rank * p.npairs);
+      } else {
+        const int pr = rem / n_sh;
+        quad = p.npairs - 1 - pr;
+        j = g + (rem - pr * n_sh) * p.groups;
+      }
+      w[g][u] = quad_steps(p, j, quad);
+      const int k = u / G, r = u % G;
+      cta[g][(k & 1) ? (G - 1 - r) : r] += w[g][u];
+    }
+  }
+  auto makespan = [&]() {
+    long long mx = 0;
+    for (auto& row : cta)
+      for (long long v : row) mx = std::max(mx, v);
+    for (long long v : help) mx = std::max(mx, v);
+    return mx;
+  };
+  long long best = makespan();
+  int best_t = 0;
+  for (int t = 1; t <= t_max; ++t) {
+    for (int g = 0; g < p.groups; ++g) {
+      const int u = (int)w[g].size() - t;
+      const int k = u / G, r = u % G;
+      cta[g][(k & 1) ? (G - 1 - r) : r] -= w[g][u];
+      help[g % E] += w[g][u];
+    }
+    const long long ms = makespan();
+    if (ms < best) {
+      best = ms;
+      best_t = t;
+    }
+  }
+  return best_t;
+}
+
+// The CTA-pair kernel: d = 128, layout order (no token-order addressing),
+// not zigzag, not the single-block mode.
+static ra_status launch_pair(const AttnLaunch& a) {
+  constexpr int D = 128;
+  using C = PairCfg<D>;
+  CUtensorMap tq, tk, tv;
+  const int64_t c = a.N / a.P;
+  if (!encode_qkv_map(&tq, a.q, a.BH, a.N, c, a.P, D, 0, kBM) ||
+      !encode_qkv_map(&tk, a.k, a.BH, a.N, c, a.P, D, 0, kBN / 2) ||
+      !encode_qkv_map(&tv, a.v, a.BH, a.N, c, a.P, D, 0, kBN))
+    return RA_ERR_CUDA;
+  static int attr_set[64] = {0};
+  static int clusters[64] = {0};
+  if (a.device < 64 && !attr_set[a.device]) {
+    if (cudaFuncSetAttribute(attn_fwd_pair_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes) != cudaSuccess)
+      return RA_ERR_CUDA;
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, attn_fwd_pair_kernel<D>) != cudaSuccess ||
+        fa.numRegs * C::kThreads < 256 * C::kRegsHigh + 128 * C::kRegsLow)
+      return RA_ERR_CUDA;
+    // clusters of two that can be resident at once (one CTA per SM)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (a.num_sms / 2), 1, 1);
+    cfg.blockDim = dim3(C::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, attn_fwd_pair_kernel<D>, &cfg) != cudaSuccess || n < 1)
+      return RA_ERR_CUDA;
+    clusters[a.device] = n;
+    attr_set[a.device] = 1;
+  }
+  const int n_clusters = a.device < 64 ? clusters[a.device] : 1;
+  AttnParams p;
+  p.o = reinterpret_cast<__nv_bfloat16*>(a.o);
+  p.o_f32 = a.o_f32;
+  p.o_v8 = (reinterpret_cast<uintptr_t>(a.o) % 32) == 0;
+  p.tok = 0;
+  p.lse = a.lse;
+  p.BH = (int)a.BH;
+  p.N = (int)a.N;
+  p.c = (int)c;
+  p.P = a.P;
+  const int T = (int)((c + kBM - 1) / kBM);
+  p.npairs = (T + 3) / 4;                // quads of query tiles
+  p.striped = a.striped;
+  p.zigzag = 0;
+  p.causal = a.causal;
+  p.c2 = (float)((double)a.scale * 1.4426950408889634074);
+  p.drain_timeout_ns = 2000000000ull;
+  p.timeout_ns = a.main_limit_ns > 0 ? (unsigned long long)a.main_limit_ns : p.drain_timeout_ns;
+  p.withhold_first_s = a.withhold_first_s;
+  p.blk_j = -1;
+  p.blk_kb = -1;
+  p.helpers = 0;
+  p.ceded = 0;
+  const long long items_total = (long long)p.npairs * a.P * a.BH;
+  int used;
+  if (a.sched_free) {
+    p.groups = 1;
+    used = (int)(items_total < n_clusters ? items_total : n_clusters);
+    p.ctas_per_group = used;
+  } else {
+    p.groups = a.P < n_clusters ? a.P : n_clusters;
+    int G = n_clusters / p.groups;
+    const long long per_group =
+        (long long)p.npairs * a.BH * ((a.P + p.groups - 1) / p.groups);
+    if (per_group < G) G = (int)per_group;
+    p.ctas_per_group = G;
+    used = G * p.groups;
+    const int E = std::min(n_clusters - used, p.groups);
+    if (E > 0 && p.groups > 1) {
+      static std::mutex mu;
+      static std::map<std::vector<long long>, int> cache;
+      const std::vector<long long> key = {p.BH, p.N, p.P, p.striped, p.causal, p.groups, G, E};
+      int t;
+      {
+        std::lock_guard<std::mutex> lock(mu);
+        auto found = cache.find(key);
+        if (found == cache.end()) found = cache.emplace(key, plan_ceded_quads(p, E)).first;
+        t = found->second;
+      }
+      if (t > 0) {
+        p.helpers = E;
+        p.ceded = t;
+        used += E;
+      }
+    }
+  }
+  attn_fwd_pair_kernel<D><<<2 * used, C::kThreads, C::kSmemBytes, (cudaStream_t)a.stream>>>(
+      tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
 ra_status attn_fwd_launch(const AttnLaunch& a) {
+  if (a.pair && a.d == 128 && !a.zigzag && !a.tok && a.blk_kb < 0) return launch_pair(a);
   if (a.zigzag) {
     if (a.d == 128) return launch<128, true>(a);
     if (a.d == 64) return launch<64, true>(a);

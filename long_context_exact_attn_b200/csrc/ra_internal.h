@@ -33,6 +33,7 @@ struct AttnLaunch {
   int zigzag = 0;                // zigzag layout (striped == 0)
   int o_f32 = 0;                 // write O as float32
   int tok = 0;                   // q, k, v, o, lse in token order
+  int pair = 0;                  // the CTA-pair (two-SM MMA) kernel where it applies
   int64_t main_limit_ns = 0;     // > 0: limit of the main-loop waits (abort self-test)
   int withhold_first_s = 0;      // abort self-test: first S-ready signal never sent
 };

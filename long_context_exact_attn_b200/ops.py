@@ -21,6 +21,7 @@ ZIGZAG = 2
 SCHED_FREE = 0x100
 O_F32 = 0x200
 TOKEN_ORDER = 0x400
+CTA_PAIR = 0x800
 
 BF16 = 0
 F32 = 1
@@ -159,12 +160,14 @@ def partition(x, P, layout, inverse=False, out=None):
 
 
 def attn_fwd(q, k, v, P, layout, causal=True, scale=None, sched_free=False, out=None, lse=None,
-             o_f32=False, token_order=False):
+             o_f32=False, token_order=False, cta_pair=False):
     """Exact blockwise attention forward; q, k, v: [B, H, N, d] bf16 CUDA
     tensors in LAYOUT order (in token order with ``token_order``: the
     kernel applies the layout's permutation itself).  Returns (o [B, H, N, d]
     bf16, or float32 with ``o_f32``, lse [B, H, N] float32), in the same
-    order as the inputs."""
+    order as the inputs.  ``cta_pair`` selects the two-SM (cluster of two)
+    form of the kernel where it applies (RA_CTA_PAIR: same results, slower
+    on the shapes measured)."""
     for n, t in (("q", q), ("k", k), ("v", v)):
         _cuda_contig(t, n)
         if t.dtype != torch.bfloat16:
@@ -181,7 +184,7 @@ def attn_fwd(q, k, v, P, layout, causal=True, scale=None, sched_free=False, out=
     lse = (torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None
            else _like(lse, "lse", (B, H, N), torch.float32, q.device))
     lay = (int(layout) | (SCHED_FREE if sched_free else 0) | (O_F32 if o_f32 else 0)
-           | (TOKEN_ORDER if token_order else 0))
+           | (TOKEN_ORDER if token_order else 0) | (CTA_PAIR if cta_pair else 0))
     _launch("ra_attn_fwd", q, lib().ra_attn_fwd, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
             B, H, N, d, int(P), lay, int(bool(causal)), float(scale), _stream(q))
     return out, lse

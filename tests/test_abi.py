@@ -68,7 +68,7 @@ def attn(L, q=A, k=Bp, v=Cp, o=Op, lse=Lp, B=1, H=2, N=1024, d=128, P=4, layout=
     (dict(q=A + 8), 2), (dict(o=Op + 2), 2), (dict(lse=Lp + 4), 2),
     (dict(N=1000, P=3), 3), (dict(P=0), 3), (dict(N=0), 3), (dict(B=0), 3),
     (dict(d=96), 4), (dict(d=256), 4),
-    (dict(layout=3), 5), (dict(layout=0x800), 5), (dict(layout=0x1201), 5),
+    (dict(layout=3), 5), (dict(layout=0x1000), 5), (dict(layout=0x1201), 5),
     (dict(scale=0.0), 6), (dict(scale=float("inf")), 6), (dict(scale=float("nan")), 6),
     (dict(scale=-1.0), 6),
     (dict(o=A), 8), (dict(lse=Op + 64), 8),
