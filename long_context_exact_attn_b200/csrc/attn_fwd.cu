@@ -803,16 +803,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             if (rescale && acc) {
               // O (the previous tiles' P V: complete, since this tile's
               // scores were committed after it) moves to the new max before
-              // this tile's P V adds to it; 32 columns at a time, while the
-              // scores of keys 64-127 are still held
+              // this tile's P V adds to it; 64 columns per TMEM round trip
+              // (one wait for two loads), while the scores of keys 64-127
+              // are still held
               const uint64_t a2 = f2(alpha, alpha);
 #pragma unroll 1
-              for (int q4 = 0; q4 < D / 32; ++q4) {
-                uint32_t o32[32];
+              for (int q4 = 0; q4 < D / 32; q4 += 2) {
+                uint32_t o32[32], o32b[32];
                 tmem_ld32(tO + q4 * 32, o32);
+                tmem_ld32(tO + q4 * 32 + 32, o32b);
                 tmem_wait_ld();
                 scale_row32(o32, a2);
+                scale_row32(o32b, a2);
                 tmem_st32(tO + q4 * 32, o32);
+                tmem_st32(tO + q4 * 32 + 32, o32b);
               }
             }
             // keys 0-63 of P (and a rescaled O) are in TMEM: let P V start
