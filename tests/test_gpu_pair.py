@@ -23,11 +23,12 @@ def _lib():
     assert ops.device_fault() == 0
 
 
-def run(q, k, v, P, layout, causal, sched_free, pair):
+def run(q, k, v, P, layout, causal, sched_free, pair, o_f32=False):
     dq, dk, dv = (t.cuda() for t in (q, k, v))
     if layout != W.CONTIGUOUS:
         dq, dk, dv = (ops.partition(t, P, layout) for t in (dq, dk, dv))
-    o, lse = ops.attn_fwd(dq, dk, dv, P, layout, causal, sched_free=sched_free, cta_pair=pair)
+    o, lse = ops.attn_fwd(dq, dk, dv, P, layout, causal, sched_free=sched_free, cta_pair=pair,
+                          o_f32=o_f32)
     if layout != W.CONTIGUOUS:
         o = ops.partition(o, P, layout, inverse=True)
         lse = ops.partition(lse, P, layout, inverse=True)
@@ -74,3 +75,16 @@ def test_pair_workloads_sampled(w):
                                            v[0, h].float().numpy(), w.scale, True, rows)
         assert_close(o[0, h, rows], lse[0, h, rows], o_ref, lse_ref, f"pair {w.name} h{h}")
     assert np.array_equal(o[0, :, 0], v[0, :, 0].float().numpy())
+
+
+def test_pair_float32_output_rounds_to_bf16_output():
+    """RA_O_F32 with the pair kernel: the float32 O rounds to the bf16 O bit
+    for bit, and matches the single-CTA kernel's float32 O."""
+    w = W.Workload("pair_f32", 1, 2, 2048, 128, 4, W.STRIPED, True, seed=77, qk_scale_up=3.0)
+    q, k, v = W.make_qkv(w)
+    o32, lse32 = run(q, k, v, w.P, w.layout, True, False, True, o_f32=True)
+    o16, lse16 = run(q, k, v, w.P, w.layout, True, False, True)
+    rounded = torch.from_numpy(o32).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(rounded, o16) and np.array_equal(lse32, lse16)
+    o32s, _ = run(q, k, v, w.P, w.layout, True, False, False, o_f32=True)
+    assert np.abs(o32 - o32s).max() <= 1e-3
