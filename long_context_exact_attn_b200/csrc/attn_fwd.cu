@@ -764,9 +764,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         // nothing (a lazy threshold lets it reach 2^t with an uncovered
         // rounding error of up to 2^-8 of the dominant term).
         const bool need = m_cand > m2;
-        // The O rescale itself is deferred until after the exps: it only has
-        // to land before this tile's P V, and by then the scores are dead, so
-        // the whole O row can be loaded at once.
+        // The O rescale itself comes after the exps of keys 0-63: it only has
+        // to land before this tile's P V, and by then half of the scores are
+        // dead, which leaves the registers for 64 columns of O per round trip.
         const bool rescale = __any_sync(0xffffffffu, need);
         float alpha = 1.f;
         if (rescale) {
