@@ -290,8 +290,10 @@ ra_status ra_attn_bwd_noalloc(const void* q, const void* k, const void* v, const
  * caller's device workspace (each chunk runs the attention with
  * RA_TOKEN_ORDER, so only q, k, v, o, lse are staged): the host-to-device
  * copy of chunk i+1 and the device-to-host copy of chunk i-1 run on the
- * library's own copy streams while chunk i computes on `stream`.  Host
- * buffers should be page-locked (pinned) for the copies to overlap.
+ * library's own copy streams while chunk i computes on `stream`.  The first
+ * and last chunks take half as many heads as the others (their copies in
+ * and out overlap no compute).  Host buffers should be page-locked (pinned)
+ * for the copies to overlap.
  *
  *   q, k, v     host bf16 [B, H, N, d], token order.
  *   o, lse      host bf16 [B, H, N, d] and float32 [B, H, N], token order.

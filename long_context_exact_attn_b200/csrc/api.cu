@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include <mutex>
+#include <vector>
 
 #include "ra_internal.h"
 #include "ra_bwd.h"
@@ -486,10 +487,32 @@ ra_status ra_attn_fwd_host(const void* q, const void* k, const void* v, void* o,
     return RA_ERR_CUDA;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const int64_t T = round256(hp.tok) * G;
-  const int64_t nch = (BH + G - 1) / G;
-  for (int64_t i = 0; i < nch; ++i) {
+  // Chunk sizes: the first chunk's copy in and the last chunk's copy out
+  // overlap no compute, so both take half a chunk (when there are heads to
+  // spare); the chunks between take G heads.
+  std::vector<int64_t> sizes;
+  {
+    const int64_t half = G > 1 ? G / 2 : 1;
+    int64_t rem = BH;
+    int64_t last = 0;
+    if (rem > 2 * half) {
+      sizes.push_back(half);
+      rem -= half;
+      last = half;
+      rem -= last;
+    }
+    while (rem > 0) {
+      const int64_t g = rem < G ? rem : G;
+      sizes.push_back(g);
+      rem -= g;
+    }
+    if (last) sizes.push_back(last);
+  }
+  const int64_t nch = (int64_t)sizes.size();
+  int64_t h0 = 0;
+  for (int64_t i = 0; i < nch; h0 += sizes[i], ++i) {
     const int s = (int)(i & 1);
-    const int64_t h0 = i * G, g = (BH - h0 < G) ? BH - h0 : G;
+    const int64_t g = sizes[i];
     const int64_t tb = g * hp.tok, lb = g * hp.lsz;
     uint8_t* slot = ws + s * G * hp.per_head;
     uint8_t *dq = slot, *dk = dq + T, *dv = dk + T, *dout = dv + T;

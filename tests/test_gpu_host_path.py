@@ -37,6 +37,7 @@ CASES = [
     (2, 3, 1200, 128, 3, W.STRIPED, True, 1),
     (1, 5, 2048, 64, 4, W.CONTIGUOUS, True, 2),
     (1, 2, 1024, 128, 2, W.STRIPED, False, 8),
+    (1, 7, 2048, 128, 4, W.STRIPED, True, 4),      # chunks of 1, 2, 2, 1, 1 heads
 ]
 
 
