@@ -26,6 +26,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "ra_internal.h"
@@ -938,14 +939,16 @@ static ra_status launch_bwd(const BwdLaunch& a) {
       !encode_map(&tv, a.v, a.BH, a.N, c, a.P, D, mode) ||
       !encode_map(&tdo, a.dout, a.BH, a.N, c, a.P, D, mode))
     return RA_ERR_CUDA;
-  static int attr_set[64] = {0};
-  if (a.device < 64 && !attr_set[a.device]) {
+  // once per device (setting the attribute again is harmless; the flag only
+  // saves the calls)
+  static std::atomic<int> attr_set[64];
+  if (a.device < 64 && !attr_set[a.device].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(bwd_dkdv_kernel<D, ZZ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmem) != cudaSuccess ||
         cudaFuncSetAttribute(bwd_dq_kernel<D, ZZ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmem) != cudaSuccess)
       return RA_ERR_CUDA;
-    attr_set[a.device] = 1;
+    attr_set[a.device].store(1, std::memory_order_release);
   }
   BwdParams p;
   p.o = reinterpret_cast<const __nv_bfloat16*>(a.o);
@@ -1015,8 +1018,8 @@ ra_status attn_bwd_noalloc_launch(BwdLaunch a) {
       if (cudaGetSymbolAddress(&ptr, g_bwd_scratch) != cudaSuccess || !ptr) return RA_ERR_CUDA;
       addr[a.device] = reinterpret_cast<float*>(ptr);
     }
+    a.workspace = addr[a.device];
   }
-  a.workspace = addr[a.device];
   return attn_bwd_launch(a);
 }
 

@@ -42,6 +42,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstring>
 #include <map>
 #include <memory>
@@ -1659,15 +1660,17 @@ static ra_status launch(const AttnLaunch& a) {
       !encode_qkv_map(&tk, a.k, a.BH, a.N, c, a.P, D, mode) ||
       !encode_qkv_map(&tv, a.v, a.BH, a.N, c, a.P, D, mode))
     return RA_ERR_CUDA;
-  static int attr_set[64] = {0};
-  static int attr_list_set[64] = {0};
-  if (a.device < 64 && !attr_set[a.device]) {
+  // once per device and instance (setting the attribute again is harmless;
+  // the flags only save the calls)
+  static std::atomic<int> attr_set[64];
+  static std::atomic<int> attr_list_set[64];
+  if (a.device < 64 && !attr_set[a.device].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(attn_fwd_kernel<D, ZZ, NoLists>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmemBytes) != cudaSuccess ||
         !register_split_fits<D>(attn_fwd_kernel<D, ZZ, NoLists>))
       return RA_ERR_CUDA;
-    attr_set[a.device] = 1;
+    attr_set[a.device].store(1, std::memory_order_release);
   }
   AttnParams p;
   p.o = reinterpret_cast<__nv_bfloat16*>(a.o);
@@ -1729,13 +1732,13 @@ static ra_status launch(const AttnLaunch& a) {
       wl = found->second;
     }
     if (wl) {
-      if (a.device < 64 && !attr_list_set[a.device]) {
+      if (a.device < 64 && !attr_list_set[a.device].load(std::memory_order_acquire)) {
         if (cudaFuncSetAttribute(attn_fwd_kernel<D, ZZ, WorkLists>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::kSmemBytes) != cudaSuccess ||
             !register_split_fits<D>(attn_fwd_kernel<D, ZZ, WorkLists>))
           return RA_ERR_CUDA;
-        attr_list_set[a.device] = 1;
+        attr_list_set[a.device].store(1, std::memory_order_release);
       }
       attn_fwd_kernel<D, ZZ, WorkLists>
           <<<grid, C::kThreads, C::kSmemBytes, (cudaStream_t)a.stream>>>(tq, tk, tv, p, *wl);
@@ -1853,28 +1856,36 @@ static ra_status launch_pair(const AttnLaunch& a) {
       !encode_qkv_map(&tk, a.k, a.BH, a.N, c, a.P, D, 0, kBN / 2) ||
       !encode_qkv_map(&tv, a.v, a.BH, a.N, c, a.P, D, 0, kBN))
     return RA_ERR_CUDA;
-  static int attr_set[64] = {0};
+  // Per device, once (under a lock: the cluster count is read by every
+  // launch): the shared-memory attribute, the register check, and the number
+  // of clusters of two that can be resident at once (one CTA per SM).
+  if (a.device < 0 || a.device >= 64) return RA_ERR_DEVICE;
+  static std::mutex init_mu;
   static int clusters[64] = {0};
-  if (a.device < 64 && !attr_set[a.device]) {
-    if (cudaFuncSetAttribute(attn_fwd_pair_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kSmemBytes) != cudaSuccess)
-      return RA_ERR_CUDA;
-    cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, attn_fwd_pair_kernel<D>) != cudaSuccess ||
-        fa.numRegs * C::kThreads < 256 * C::kRegsHigh + 128 * C::kRegsLow)
-      return RA_ERR_CUDA;
-    // clusters of two that can be resident at once (one CTA per SM)
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * (a.num_sms / 2), 1, 1);
-    cfg.blockDim = dim3(C::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = C::kSmemBytes;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, attn_fwd_pair_kernel<D>, &cfg) != cudaSuccess || n < 1)
-      return RA_ERR_CUDA;
-    clusters[a.device] = n;
-    attr_set[a.device] = 1;
+  int n_clusters;
+  {
+    std::lock_guard<std::mutex> lock(init_mu);
+    if (!clusters[a.device]) {
+      if (cudaFuncSetAttribute(attn_fwd_pair_kernel<D>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               C::kSmemBytes) != cudaSuccess)
+        return RA_ERR_CUDA;
+      cudaFuncAttributes fa;
+      if (cudaFuncGetAttributes(&fa, attn_fwd_pair_kernel<D>) != cudaSuccess ||
+          fa.numRegs * C::kThreads < 256 * C::kRegsHigh + 128 * C::kRegsLow)
+        return RA_ERR_CUDA;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2 * (a.num_sms / 2), 1, 1);
+      cfg.blockDim = dim3(C::kThreads, 1, 1);
+      cfg.dynamicSmemBytes = C::kSmemBytes;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, attn_fwd_pair_kernel<D>, &cfg) != cudaSuccess ||
+          n < 1)
+        return RA_ERR_CUDA;
+      clusters[a.device] = n;
+    }
+    n_clusters = clusters[a.device];
   }
-  const int n_clusters = a.device < 64 ? clusters[a.device] : 1;
   AttnParams p;
   p.o = reinterpret_cast<__nv_bfloat16*>(a.o);
   p.o_f32 = a.o_f32;
@@ -1976,8 +1987,10 @@ ra_status wait_selftest_launch(int64_t limit_ns, void* stream) {
 // without relocatable device code).
 unsigned int* device_fault_word() {
   static unsigned int* cache[64] = {nullptr};
+  static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
   if (!cache[dev]) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_device_fault) != cudaSuccess) return nullptr;
