@@ -78,6 +78,7 @@ typedef int ra_status;
                              /* ra_attn_bwd_noalloc (B*H*N > 1048576)          */
 #define RA_ERR_ROPE 13       /* unknown RoPE pairing, or base not > 1 / finite */
 #define RA_ERR_WORKSPACE 14  /* device workspace too small                     */
+#define RA_ERR_NOPROFILE 15  /* library built without the phase profile        */
 
 /* Layouts (low byte of `layout`). */
 #define RA_CONTIGUOUS 0      /* shard j = tokens [j*c, (j+1)*c)  (Ring)        */
@@ -424,6 +425,31 @@ ra_status ra_tile_census(int64_t N, int P, int layout, int causal, int64_t* out,
  * Returns RA_ERR_DEVICE_FAULT if the word was non-zero, RA_OK otherwise.
  */
 ra_status ra_device_fault(int* code);
+
+/*
+ * ra_fwd_phase_profile -- read and clear the forward kernel's phase counters.
+ *
+ * Not an operation of the pages: a diagnostic of where the attention kernel
+ * spends its cycles.  Only a library built with RA_PROFILE=1 (`python -m
+ * long_context_exact_attn_b200.build --profile` writes libringattn_prof.so)
+ * keeps counters; the regular library returns RA_ERR_NOPROFILE.  In the
+ * profiling build every ra_attn_fwd launch adds, for each of its first 160
+ * CTAs, the clock64 cycles that each softmax warp (slots 0-7) and the MMA
+ * warp (slot 8) spent in each phase of its loop; slot 9 is unused.  Softmax
+ * phases: 0 loop, skipped tiles and epilogue, 1 waiting for S, 2 loading S
+ * from tensor memory, 3 row max and rescale decision, 4 exps of keys 0-63
+ * with the O rescale and the first publication of P, 5 exps of keys 64-127
+ * and the last publication, 6 unused, 7 tiles processed.  MMA phases: 0
+ * issuing, 1 waiting for the next K tile, 2 for the V tile, 3 for the first
+ * half of P, 4 for its second half, 5 for a released O (epilogue), 6
+ * unused, 7 key-tile steps.  The timers themselves cost a few per cent.
+ * This call synchronises the current device, copies the counters to
+ * host memory as uint64 [160][10][8] and clears them.
+ *
+ *   out       host array of at least 160 * 10 * 8 = 12800 uint64 values.
+ *   capacity  its length; smaller: RA_ERR_SHAPE.
+ */
+ra_status ra_fwd_phase_profile(uint64_t* out, int64_t capacity);
 
 /*
  * ra_wait_selftest -- exercise the bounded-wait and fault-reporting path.

@@ -146,6 +146,7 @@ const char* ra_status_string(ra_status s) {
     case RA_ERR_DEVICE_FAULT: return "a kernel gave up a bounded wait; outputs incomplete";
     case RA_ERR_ROPE: return "unknown RoPE pairing, or RoPE base not finite and > 1";
     case RA_ERR_WORKSPACE: return "device workspace too small (see ra_attn_fwd_host_workspace)";
+    case RA_ERR_NOPROFILE: return "library built without the phase profile (RA_PROFILE)";
     case RA_ERR_SCRATCH:
       return "B*H*N exceeds the built-in scratch of ra_attn_bwd_noalloc (1048576 rows); "
              "use ra_attn_bwd with a workspace";
@@ -603,6 +604,11 @@ ra_status ra_wait_selftest(int64_t limit_ns, void* stream) {
 ra_status ra_device_fault(int* code) {
   if (!code) return RA_ERR_NULL;
   return read_device_fault(code);
+}
+
+ra_status ra_fwd_phase_profile(uint64_t* out, int64_t capacity) {
+  if (!out) return RA_ERR_NULL;
+  return fwd_profile_read(reinterpret_cast<unsigned long long*>(out), capacity);
 }
 
 }  // extern "C"

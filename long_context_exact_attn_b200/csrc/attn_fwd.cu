@@ -58,6 +58,52 @@ namespace ra {
 
 __device__ unsigned int g_device_fault = 0;
 
+// Phase profile (profiling build only: RA_PROFILE=1, a library of its own).
+// Each softmax warp (slots 0-7) and the MMA warp (slot 8) of the first
+// kProfCtas CTAs accumulate clock64 cycles per phase of their loop; the
+// counters are read and cleared through ra_fwd_phase_profile.  Without
+// RA_PROFILE every marker below compiles to nothing.
+#ifndef RA_PROFILE
+#define RA_PROFILE 0
+#endif
+#if RA_PROFILE
+__device__ unsigned long long g_fwd_profile[kProfCtas * kProfSlots * kProfPhases];
+// 32-bit counts per launch and warp (a warp's launch is far below 2^32
+// cycles), added into the 64-bit counters at the end: fewer registers.
+struct PhaseClock {
+  uint32_t acc[kProfPhases];
+  uint32_t last;
+  __device__ __forceinline__ void start() {
+#pragma unroll
+    for (int i = 0; i < kProfPhases; ++i) acc[i] = 0;
+    last = (uint32_t)clock64();
+  }
+  __device__ __forceinline__ void mark(int i) {
+    const uint32_t t = (uint32_t)clock64();
+    acc[i] += t - last;
+    last = t;
+  }
+  __device__ __forceinline__ void count() { acc[kProfPhases - 1] += 1; }
+  __device__ __forceinline__ void store(int slot) {
+    if ((threadIdx.x % 32) == 0 && blockIdx.x < kProfCtas)
+#pragma unroll
+      for (int i = 0; i < kProfPhases; ++i)
+        atomicAdd(&g_fwd_profile[(blockIdx.x * kProfSlots + slot) * kProfPhases + i],
+                  (unsigned long long)acc[i]);
+  }
+};
+#define RA_PHASE_START(c) (c).start()
+#define RA_PHASE(c, i) (c).mark(i)
+#define RA_PHASE_COUNT(c) (c).count()
+#define RA_PHASE_STORE(c, slot) (c).store(slot)
+#else
+struct PhaseClock {};
+#define RA_PHASE_START(c) ((void)0)
+#define RA_PHASE(c, i) ((void)0)
+#define RA_PHASE_COUNT(c) ((void)0)
+#define RA_PHASE_STORE(c, slot) ((void)0)
+#endif
+
 // Work lists for small problems (see WorkLists): capacity, and the largest
 // problem (items of all heads and shards) that uses them.  At N = 8192
 // (512 items) the whole K/V fits in L2 and the lists only rebalance work;
@@ -590,6 +636,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       // at a time: a parity wait is only unambiguous one phase ahead, and a
       // query tile without key tiles in an item skips its lazy wait.
       uint32_t of0 = 0, of1 = 0;
+      PhaseClock mc;
+      (void)mc;
+      RA_PHASE_START(mc);
       Item it;
       bool ok = true;
       for (int k = 0; ok && cta_item(p, wl, k, it); ++k) {
@@ -632,25 +681,33 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           const uint32_t vslot = slot, vph = phase;
           if (++slot == C::kSlots) { slot = 0; phase ^= 1; }
           uint32_t nkslot = 0;
+          RA_PHASE(mc, 0);
           if (more) {
             nkslot = slot;
             if (!wmbar_wait(full0 + 8 * nkslot, phase, abort_flag, p.timeout_ns)) { ok = false; break; }
             if (++slot == C::kSlots) { slot = 0; phase ^= 1; }
           }
+          RA_PHASE(mc, 1);
           if (!wmbar_wait(full0 + 8 * vslot, vph, abort_flag, p.timeout_ns)) { ok = false; break; }
+          RA_PHASE(mc, 2);
           const uint32_t va = sRing + vslot * C::kTileBytes;
           const uint32_t nka = sRing + nkslot * C::kTileBytes;
           // query tile 0: P0 V, then the next Q0 K^T into the freed S0/P0 columns
           if (c0 != TILE_SKIP) {
             bool okw = true;
+            RA_PHASE(mc, 0);
             while (okw && of0 < (uint32_t)k) okw = wmbar_wait(o_free0, of0++ & 1, abort_flag, p.timeout_ns);
             if (!okw) { ok = false; break; }
+            RA_PHASE(mc, 5);
             // P in two halves: the first 4 k-steps (keys 0-63) start while the
             // softmax is still producing keys 64-127.
             if (!wmbar_wait(p_full0, pc0 & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+            RA_PHASE(mc, 3);
             tc_fence_after();
             mma_pv<D, 0, 4>(tO0, tS0, va, acc0);
+            RA_PHASE(mc, 0);
             if (!wmbar_wait(p_full2_0, pc0 & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+            RA_PHASE(mc, 4);
             ++pc0;
             tc_fence_after();
             mma_pv<D, 4, 8>(tO0, tS0, va, 1);
@@ -660,14 +717,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           // query tile 1
           if (c1 != TILE_SKIP) {
             bool okw = true;
+            RA_PHASE(mc, 0);
             while (okw && of1 < (uint32_t)k) okw = wmbar_wait(o_free1, of1++ & 1, abort_flag, p.timeout_ns);
             if (!okw) { ok = false; break; }
+            RA_PHASE(mc, 5);
             // P in two halves: the first 4 k-steps (keys 0-63) start while the
             // softmax is still producing keys 64-127.
             if (!wmbar_wait(p_full1, pc1 & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+            RA_PHASE(mc, 3);
             tc_fence_after();
             mma_pv<D, 0, 4>(tO1, tS1, va, acc1);
+            RA_PHASE(mc, 0);
             if (!wmbar_wait(p_full2_1, pc1 & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
+            RA_PHASE(mc, 4);
             ++pc1;
             tc_fence_after();
             mma_pv<D, 4, 8>(tO1, tS1, va, 1);
@@ -679,6 +741,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           have = more;
           c0 = n0;
           c1 = n1;
+          RA_PHASE(mc, 0);
+          RA_PHASE_COUNT(mc);
         }
         if (!ok) break;
         {
@@ -691,6 +755,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         mma_commit_w(bar_o_full + 8);
         mma_commit_w(bar_q_empty);
       }
+      RA_PHASE(mc, 0);
+      RA_PHASE_STORE(mc, 8);
       // All MMAs issued by this thread must be complete before TMEM is freed.
       mma_commit_w(bar_drain);
       volatile int no_abort = 0;
@@ -714,6 +780,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const uint32_t my_o_free = bar_o_free + 8 * t;
     const float c2 = p.c2;
     uint32_t s_cnt = 0;
+    PhaseClock pc;
+    (void)pc;
+    RA_PHASE_START(pc);
     Item it;
     bool ok = true;
     for (int k = 0; ok && cta_item(p, wl, k, it); ++k) {
@@ -730,8 +799,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (kind == TILE_SKIP) continue;
         // warp-uniform: a lane that gives up makes the whole warp give up, so
         // the warp-collective TMEM accesses and votes below never diverge
+        RA_PHASE(pc, 0);
         if (!wmbar_wait(my_s_full, s_cnt & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
         ++s_cnt;
+        RA_PHASE(pc, 1);
         tc_fence_after();
         uint32_t sr[4][32];
 #pragma unroll
@@ -742,6 +813,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (int q = 0; q < 4; ++q)
 #pragma unroll
           for (int i = 0; i < 32; ++i) s[q * 32 + i] = __uint_as_float(sr[q][i]);
+        RA_PHASE(pc, 2);
         if (kind == TILE_PARTIAL) {
           const int lim = row_limit(bm, x - seq.mxo(), y0 - seq.myo(), seq.mc());
 #pragma unroll
@@ -778,6 +850,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const float msub = (m2 == -INFINITY) ? 0.f : m2;
         const uint64_t c2x2 = f2(c2, c2);
         const uint64_t nm2 = f2(-msub, -msub);
+        RA_PHASE(pc, 3);
         uint64_t sum_e[4] = {0, 0, 0, 0};   // row sum of the probabilities
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
@@ -825,6 +898,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(my_p_full);
+            RA_PHASE(pc, 4);
           }
         }
         {
@@ -836,6 +910,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(my_p_full2);
+        RA_PHASE(pc, 5);
+        RA_PHASE_COUNT(pc);
         acc = true;
       }
       if (!ok) break;
@@ -897,6 +973,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       __syncwarp();
       if (lane == 0) mbar_arrive(my_o_free);
     }
+    RA_PHASE(pc, 0);
+    RA_PHASE_STORE(pc, warp);
   }
 
   tc_fence_before();
@@ -1997,6 +2075,23 @@ unsigned int* device_fault_word() {
     cache[dev] = reinterpret_cast<unsigned int*>(ptr);
   }
   return cache[dev];
+}
+
+ra_status fwd_profile_read(unsigned long long* host, int64_t capacity) {
+#if RA_PROFILE
+  const int64_t n = (int64_t)kProfCtas * kProfSlots * kProfPhases;
+  if (capacity < n) return RA_ERR_SHAPE;
+  if (cudaDeviceSynchronize() != cudaSuccess) return RA_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(host, g_fwd_profile, n * sizeof(unsigned long long)) != cudaSuccess)
+    return RA_ERR_CUDA;
+  static const unsigned long long zeros[kProfCtas * kProfSlots * kProfPhases] = {};
+  if (cudaMemcpyToSymbol(g_fwd_profile, zeros, sizeof(zeros)) != cudaSuccess) return RA_ERR_CUDA;
+  return RA_OK;
+#else
+  (void)host;
+  (void)capacity;
+  return RA_ERR_NOPROFILE;
+#endif
 }
 
 ra_status read_device_fault(int* code) {

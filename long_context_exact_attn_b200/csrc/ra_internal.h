@@ -42,6 +42,12 @@ ra_status attn_fwd_launch(const AttnLaunch& a);
 
 ra_status read_device_fault(int* code);
 unsigned int* device_fault_word();
+
+// Phase profile of the forward kernel (profiling build only): counters per
+// CTA (the first kProfCtas), role slot (softmax warps 0-7, MMA warp 8, one
+// spare) and phase (the last phase counts tiles).
+constexpr int kProfCtas = 160, kProfSlots = 10, kProfPhases = 8;
+ra_status fwd_profile_read(unsigned long long* host, int64_t capacity);
 ra_status wait_selftest_launch(int64_t limit_ns, void* stream);
 
 ra_status partition_launch(const void* src, void* dst, int64_t rows_outer, int64_t N, int64_t P,

@@ -38,6 +38,15 @@ class RingAttnError(RuntimeError):
         super().__init__(f"{where}: status {status} ({status_string(status)})")
 
 
+def use_library(path):
+    """Load the C library from `path` instead of the default (before the first
+    call; e.g. the profiling build libringattn_prof.so)."""
+    global LIB_PATH
+    if _lib is not None and os.path.abspath(path) != os.path.abspath(LIB_PATH):
+        raise RuntimeError("the library is already loaded from " + LIB_PATH)
+    LIB_PATH = path
+
+
 def lib():
     """The loaded C library (loaded on first use; raises if it is missing)."""
     global _lib
@@ -84,6 +93,8 @@ def lib():
                                              i32, f32, i64, vp]
         L.ra_device_fault.restype = i32
         L.ra_device_fault.argtypes = [ctypes.POINTER(ctypes.c_int)]
+        L.ra_fwd_phase_profile.restype = i32
+        L.ra_fwd_phase_profile.argtypes = [ctypes.POINTER(ctypes.c_uint64), i64]
         _lib = L
     return _lib
 
@@ -409,6 +420,21 @@ def attn_abort_selftest(q, k, v, P, layout, causal=True, limit_ns=1_000_000, out
             _ptr(out), _ptr(lse), B, H, N, d, int(P), int(layout), int(bool(causal)),
             float(d ** -0.5), int(limit_ns), _stream(q))
     return out, lse
+
+
+PROFILE_SHAPE = (160, 10, 8)   # CTAs, role slots, phases (see ra_fwd_phase_profile)
+
+
+def fwd_phase_profile():
+    """Read and clear the forward kernel's phase counters (profiling build
+    only; the regular library raises RingAttnError with RA_ERR_NOPROFILE).
+    Returns a nested list [cta][slot][phase] of cycle counts (phase 7: tiles)."""
+    n = PROFILE_SHAPE[0] * PROFILE_SHAPE[1] * PROFILE_SHAPE[2]
+    buf = (ctypes.c_uint64 * n)()
+    _check(lib().ra_fwd_phase_profile(buf, n), "ra_fwd_phase_profile")
+    c, sl, ph = PROFILE_SHAPE
+    return [[[int(buf[(i * sl + j) * ph + k]) for k in range(ph)] for j in range(sl)]
+            for i in range(c)]
 
 
 def device_fault():

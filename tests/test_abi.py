@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(L):
 
 def test_status_strings(L):
     assert ops.status_string(0) == "ok"
-    for code in range(1, 15):
+    for code in range(1, 16):
         assert ops.status_string(code) not in ("", "unknown status")
     assert ops.status_string(999) == "unknown status"
     assert L.ra_version() >= 100
@@ -309,3 +309,13 @@ def test_header_is_plain_c_and_links(L, tmp_path):
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0, (r.returncode, r.stderr)
     assert r.stdout.strip() == ops.status_string(3)
+
+
+def test_phase_profile_needs_the_profiling_build(L):
+    """The regular library keeps no phase counters: RA_ERR_NOPROFILE (15)
+    without touching the device; a NULL output is refused first."""
+    buf = (ctypes.c_uint64 * (160 * 10 * 8))()
+    assert L.ra_fwd_phase_profile(buf, len(buf)) == 15
+    assert L.ra_fwd_phase_profile(None, len(buf)) == 1
+    with pytest.raises(ops.RingAttnError):
+        ops.fwd_phase_profile()
