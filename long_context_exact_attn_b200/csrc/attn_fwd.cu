@@ -47,6 +47,7 @@
 #include <map>
 #include <memory>
 #include <mutex>
+#include <type_traits>
 #include <vector>
 
 #include "exp2_poly.h"
@@ -163,7 +164,7 @@ struct Cfg {
   static constexpr int kRingOff = 2 * kTileBytes;
   static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
   // barriers: q_full, q_empty, full[kSlots], empty[kSlots], s_full[2],
-  // p_full[2] (P columns of keys 0-63 ready), p_full2[2] (keys 64-127),
+  // p_full[2] (first part of P ready), p_full2[2] (the rest),
   // o_full[2], o_free[2], drain
   static constexpr int kNumBars = 2 + 2 * kSlots + 10 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
@@ -508,6 +509,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 const __grid_constant__ CUtensorMap tmV, const AttnParams p,
                 const __grid_constant__ Lists wl) {
   using C = Cfg<D>;
+  // P is published in two parts: keys [0, 32 kPub) and the rest; P V runs
+  // in the same two parts (2 kPub and 8 - 2 kPub k-steps of 16 keys).  The
+  // work-list instance (small striped problems: short rows, where the O
+  // rescale before the first part is frequent) publishes after 96 keys, the
+  // other instances after 64 (measured: +1.3 % and -0.5 % respectively with
+  // 96 at N = 8192 and N = 262144).
+  constexpr int kPub = std::is_same<Lists, WorkLists>::value ? 3 : 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -699,18 +707,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             while (okw && of0 < (uint32_t)k) okw = wmbar_wait(o_free0, of0++ & 1, abort_flag, p.timeout_ns);
             if (!okw) { ok = false; break; }
             RA_PHASE(mc, 5);
-            // P in two halves: the first 4 k-steps (keys 0-63) start while the
-            // softmax is still producing keys 64-127.
+            // P in two parts: the first 2 kPub k-steps start while the
+            // softmax is still producing the rest.
             if (!wmbar_wait(p_full0, pc0 & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
             RA_PHASE(mc, 3);
             tc_fence_after();
-            mma_pv<D, 0, 4>(tO0, tS0, va, acc0);
+            mma_pv<D, 0, 2 * kPub>(tO0, tS0, va, acc0);
             RA_PHASE(mc, 0);
             if (!wmbar_wait(p_full2_0, pc0 & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
             RA_PHASE(mc, 4);
             ++pc0;
             tc_fence_after();
-            mma_pv<D, 4, 8>(tO0, tS0, va, 1);
+            mma_pv<D, 2 * kPub, 8>(tO0, tS0, va, 1);
             acc0 = 1;
           }
           if (more && n0 != TILE_SKIP) { tc_fence_after(); mma_qk<D>(tS0, sQ0, nka); mma_commit_w(s_full0); }
@@ -721,18 +729,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             while (okw && of1 < (uint32_t)k) okw = wmbar_wait(o_free1, of1++ & 1, abort_flag, p.timeout_ns);
             if (!okw) { ok = false; break; }
             RA_PHASE(mc, 5);
-            // P in two halves: the first 4 k-steps (keys 0-63) start while the
-            // softmax is still producing keys 64-127.
+            // P in two parts: the first 2 kPub k-steps start while the
+            // softmax is still producing the rest.
             if (!wmbar_wait(p_full1, pc1 & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
             RA_PHASE(mc, 3);
             tc_fence_after();
-            mma_pv<D, 0, 4>(tO1, tS1, va, acc1);
+            mma_pv<D, 0, 2 * kPub>(tO1, tS1, va, acc1);
             RA_PHASE(mc, 0);
             if (!wmbar_wait(p_full2_1, pc1 & 1, abort_flag, p.timeout_ns)) { ok = false; break; }
             RA_PHASE(mc, 4);
             ++pc1;
             tc_fence_after();
-            mma_pv<D, 4, 8>(tO1, tS1, va, 1);
+            mma_pv<D, 2 * kPub, 8>(tO1, tS1, va, 1);
             acc1 = 1;
           }
           mma_commit_w(empty0 + 8 * vslot);
@@ -837,9 +845,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         // nothing (a lazy threshold lets it reach 2^t with an uncovered
         // rounding error of up to 2^-8 of the dominant term).
         const bool need = m_cand > m2;
-        // The O rescale itself comes after the exps of keys 0-63: it only has
-        // to land before this tile's P V, and by then half of the scores are
-        // dead, which leaves the registers for 64 columns of O per round trip.
+        // The O rescale itself comes after the exps of the first part of P:
+        // it only has to land before this tile's P V, and by then those
+        // scores are dead, which leaves the registers for 64 columns of O per
+        // round trip.
         const bool rescale = __any_sync(0xffffffffu, need);
         float alpha = 1.f;
         if (rescale) {
@@ -873,13 +882,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
           }
           tmem_st16(tS + ch * 16, pk);
-          if (ch == 1) {
+          if (ch == kPub - 1) {
             if (rescale && acc) {
               // O (the previous tiles' P V: complete, since this tile's
               // scores were committed after it) moves to the new max before
               // this tile's P V adds to it; 64 columns per TMEM round trip
-              // (one wait for two loads), while the scores of keys 64-127
-              // are still held
+              // (one wait for two loads), while the scores of the second
+              // part are still held
               const uint64_t a2 = f2(alpha, alpha);
 #pragma unroll 1
               for (int q4 = 0; q4 < D / 32; q4 += 2) {
@@ -893,7 +902,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 tmem_st32(tO + q4 * 32 + 32, o32b);
               }
             }
-            // keys 0-63 of P (and a rescaled O) are in TMEM: let P V start
+            // the first part of P (and a rescaled O) is in TMEM: let P V start
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
