@@ -678,8 +678,10 @@ def main():
             l_blk = torch.empty(w.B, w.H, c, dtype=torch.float32, device="cuda")
             acc = torch.empty(o_blk.shape, dtype=torch.float32, device="cuda")
             lacc = torch.empty_like(l_blk)
-            t = [[0.0] * w.P for _ in range(w.P)]
-            for rep in range(2):                       # first pass warms up
+            # first pass warms up; each block's time is the median of the
+            # three passes after it (one slow launch must not set a round)
+            samples = [[[] for _ in range(w.P)] for _ in range(w.P)]
+            for rep in range(4):
                 for j in range(w.P):
                     for r in range(w.P):
                         kb = (j - r) % w.P
@@ -691,7 +693,9 @@ def main():
                         ops.lse_merge_acc(acc, lacc, o_blk, l_blk, first=(r == 0))
                         e1.record()
                         e1.synchronize()
-                        t[j][r] = e0.elapsed_time(e1)
+                        if rep:
+                            samples[j][r].append(e0.elapsed_time(e1))
+            t = [[statistics.median(samples[j][r]) for r in range(w.P)] for j in range(w.P)]
             del shards, o_blk, l_blk, acc, lacc
             torch.cuda.empty_cache()
             round_max = [max(t[j][r] for j in range(w.P)) for r in range(w.P)]
@@ -710,8 +714,8 @@ def main():
         ring["contiguous_over_striped"] = round(
             ring["contiguous"]["predicted_ring_ms"] / ring["striped"]["predicted_ring_ms"], 3)
         ring["note"] = ("per-round block (float32 partial) + merge kernels of every rank run "
-                        "one at a time on this GPU; P GPUs would run each round's ranks "
-                        "concurrently")
+                        "one at a time on this GPU (median of 3 timings each); P GPUs would "
+                        "run each round's ranks concurrently")
 
     # ---- stripe + RoPE of q and k (memory-bound side path, not in the step)
     rope = None

@@ -437,11 +437,12 @@ ra_status ra_device_fault(int* code);
  * CTAs, the clock64 cycles that each softmax warp (slots 0-7) and the MMA
  * warp (slot 8) spent in each phase of its loop; slot 9 is unused.  Softmax
  * phases: 0 loop, skipped tiles and epilogue, 1 waiting for S, 2 loading S
- * from tensor memory, 3 row max and rescale decision, 4 exps of keys 0-63
- * with the O rescale and the first publication of P, 5 exps of keys 64-127
- * and the last publication, 6 unused, 7 tiles processed.  MMA phases: 0
- * issuing, 1 waiting for the next K tile, 2 for the V tile, 3 for the first
- * half of P, 4 for its second half, 5 for a released O (epilogue), 6
+ * from tensor memory, 3 row max and rescale decision, 4 exps of the first
+ * part of P (keys 0-63; 0-95 when the work-list schedule of small striped
+ * problems runs) with the O rescale and the first publication of P, 5 exps
+ * of the rest and the last publication, 6 unused, 7 tiles processed.  MMA
+ * phases: 0 issuing, 1 waiting for the next K tile, 2 for the V tile, 3 for
+ * the first part of P, 4 for the rest, 5 for a released O (epilogue), 6
  * unused, 7 key-tile steps.  The timers themselves cost a few per cent.
  * This call synchronises the current device, copies the counters to
  * host memory as uint64 [160][10][8] and clears them.

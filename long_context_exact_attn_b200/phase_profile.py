@@ -18,9 +18,11 @@ import torch
 from . import build, ops
 from . import workloads as W
 
+# The first part of P is keys 0-63, or 0-95 in the work-list instance
+# (small striped problems).
 SOFTMAX_PHASES = ["loop, skips, epilogue", "wait for S", "load S", "row max and decision",
-                  "exps 0-63, O rescale, publish", "exps 64-127, publish"]
-MMA_PHASES = ["issue", "wait next K", "wait V", "wait P (keys 0-63)", "wait P (keys 64-127)",
+                  "exps of P's first part, O rescale, publish", "exps of the rest, publish"]
+MMA_PHASES = ["issue", "wait next K", "wait V", "wait P (first part)", "wait P (rest)",
               "wait released O"]
 
 
